@@ -1,0 +1,88 @@
+"""ctypes view of ``libsvdq.so`` (the C ABI declared in ``include/svdq.h``).
+
+Loading fails loudly when the library is missing: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, Structure, c_char_p, c_int, c_int64, c_size_t, c_uint32, c_void_p
+
+from .build import LIB_PATH
+
+SVDQ_OK = 0
+SVDQ_ERR_INVALID_ARG = 1
+SVDQ_ERR_UNSUPPORTED = 2
+SVDQ_ERR_MISALIGNED = 3
+SVDQ_ERR_CUDA = 4
+SVDQ_ERR_TIMEOUT = 5
+SVDQ_ERR_NO_DEVICE = 6
+
+
+class SvdqSeg(Structure):
+    _fields_ = [("begin", c_int64), ("end", c_int64)]
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, call: str, status: int, text: str):
+        super().__init__(f"{call} failed: {text} (status {status})")
+        self.status = status
+
+
+# name -> (restype, argtypes); mirrors include/svdq.h
+SIGNATURES = {
+    "svdq_status_string": (c_char_p, [c_int]),
+    "svdq_version": (c_int, []),
+    "svdq_sf_bytes": (c_size_t, [c_int64, c_int64]),
+    "svdq_calib_lambda": (c_int, [c_void_p, c_int64, c_int64, c_int64, POINTER(SvdqSeg), c_int,
+                                  c_void_p, c_int64, c_int64,
+                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "svdq_quantize_act": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p,
+                                  c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "svdq_linear": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                            c_void_p, c_int64, c_int, c_int64, c_int64, c_int64, c_void_p]),
+    "svdq_score_workspace_bytes": (c_size_t, [POINTER(SvdqSeg), c_int, c_int64]),
+    "svdq_score_lambda": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int64, POINTER(SvdqSeg), c_int,
+                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "svdq_residual": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_int,
+                              c_void_p, c_void_p]),
+    "svdq_device_error": (c_int, [c_void_p, POINTER(c_uint32)]),
+}
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load (once) and return the library with every signature declared."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with `python -m bit_w4a4_quantized_svdq_b200.build` "
+            "(the CUDA library is the only implementation; there is no fallback)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_text(status: int) -> str:
+    return load().svdq_status_string(status).decode()
+
+
+def check(call: str, status: int) -> None:
+    if status != SVDQ_OK:
+        raise SvdqError(call, status, status_text(status))
+
+
+def seg_array(segs):
+    """Host array of svdq_seg from [(begin, end), ...]; (None, 0) for None."""
+    if segs is None:
+        return None, 0
+    arr = (SvdqSeg * len(segs))(*[SvdqSeg(int(b), int(e)) for b, e in segs])
+    return arr, len(segs)

@@ -1,0 +1,65 @@
+// common.cuh -- host-side helpers shared by the C-ABI entry points:
+// argument checks, the per-device error word, TMA descriptor encoding.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/svdq.h"
+
+namespace svdq {
+
+// Row ranges handed to kernels by value (host segments are copied in).
+constexpr int kMaxSegments = 64;
+
+struct SegTable {
+    int n;
+    int64_t begin[kMaxSegments];
+    int64_t prefix[kMaxSegments + 1];   // prefix[s] = rows in segments before s
+};
+
+// Validate host segments against [0, M) and fill a SegTable.  NULL/0 selects all rows.
+inline int make_seg_table(const svdq_seg* segs, int n_seg, int64_t M, SegTable* t) {
+    if (n_seg < 0 || n_seg > kMaxSegments) return SVDQ_ERR_INVALID_ARG;
+    if (n_seg > 0 && segs == nullptr) return SVDQ_ERR_INVALID_ARG;
+    if (segs == nullptr) {
+        t->n = 1;
+        t->begin[0] = 0;
+        t->prefix[0] = 0;
+        t->prefix[1] = M;
+        return SVDQ_OK;
+    }
+    t->n = n_seg;
+    t->prefix[0] = 0;
+    for (int s = 0; s < n_seg; ++s) {
+        if (segs[s].begin < 0 || segs[s].end < segs[s].begin || segs[s].end > M) return SVDQ_ERR_INVALID_ARG;
+        t->begin[s] = segs[s].begin;
+        t->prefix[s + 1] = t->prefix[s] + (segs[s].end - segs[s].begin);
+    }
+    return SVDQ_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device's error word (a __device__ variable of this library).
+uint32_t* device_error_word();
+
+// Current device is sm_100 (B200 class)?  Cached per device.
+bool device_is_sm100();
+
+// Number of SMs of the current device (cached).
+int device_sm_count();
+
+// Encode a 2-D tiled tensor map (dims/strides in elements of `dtype`).
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t elem_bytes,
+                    const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
+                    uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
+inline int launch_status(cudaError_t e) {
+    if (e == cudaSuccess) return SVDQ_OK;
+    return SVDQ_ERR_CUDA;
+}
+
+}  // namespace svdq

@@ -1,0 +1,441 @@
+// linear.cu -- the fused W4A4 linear: block-scaled NVFP4 GEMM on the tcgen05
+// tensor cores with the low-rank up-projection, the tensor scales and the bias
+// in the same accumulator / epilogue.
+//
+// "MiniMax-H3 . SVDQuant W4A4 (int4, rank 32, GPTQ)", opening section: 4-bit
+// activations times the 4-bit residual weight plus the 16-bit rank-32 branch,
+// executed as one fused kernel (the "Measured" table contrasts it with an
+// unfused dequantise-then-GEMM path).  "MiniMax-H3 NVFP4 -- what the smoothing
+// scale should be calibrated on", section "Why": one E4M3 scale per 16
+// consecutive channels.
+//
+//   Y[m, n] = alpha * (sum_k A[m,k] B[n,k] + sum_j D'[m,j] up[n,j]) + bias[n]
+//   alpha   = s_g_act * s_g_w,   D' = D / alpha (split into bf16 hi + lo)
+//
+// One persistent CTA per SM walks 128 x 256 output tiles (M fastest).  Warps:
+//   0     TMA producer: per 256-channel stage, A codes 128 x 128 B and B codes
+//         256 x 128 B (128-byte swizzle) plus 2 + 4 KB of scale atoms (bulk copies)
+//   1     tcgen05 issuer and tensor-memory owner: per tile 4 kind::f16 MMAs for
+//         the low-rank term (K = 64: 32 ranks of D'_hi then 32 of D'_lo against
+//         up twice), then per stage: scale atoms -> tensor memory (tcgen05.cp),
+//         4 kind::mxf4nvf4 block16 MMAs (K = 64 each) into one fp32 accumulator
+//   2     low-rank operand builder: D' hi/lo and the duplicated up tile written
+//         into the swizzled operand layout in shared memory
+//   3..6  epilogue: tensor memory -> registers, alpha and bias, bf16 (or fp32)
+//         rows to global memory; the accumulator is released as soon as it has
+//         been read, so the stores overlap the next tile's main loop.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace svdq {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBKBytes = 128;                 // packed FP4 bytes per row per stage (256 channels)
+constexpr int kBK = 256;                      // channels per stage
+constexpr int kStages = 3;
+constexpr int kThreads = 224;
+constexpr int kEpiWarp0 = 3;
+constexpr int kEpiWarps = 4;
+
+constexpr uint32_t kATile = kBM * kBKBytes;          // 16 KB
+constexpr uint32_t kBTile = kBN * kBKBytes;          // 32 KB
+constexpr uint32_t kSfaTile = kBM * (kBK / 16);      // 2 KB: 4 atoms of 512 B
+constexpr uint32_t kSfbTile = kBN * (kBK / 16);      // 4 KB: 2 row blocks x 4 atoms
+constexpr uint32_t kStageBytes = kATile + kBTile + kSfaTile + kSfbTile;
+constexpr uint32_t kLrA = kBM * 128;                 // 128 rows x 64 bf16
+constexpr uint32_t kLrB = kBN * 128;                 // 256 rows x 64 bf16
+
+constexpr uint32_t kOffStages = 0;
+constexpr uint32_t kOffLrA = kStages * kStageBytes;  // multiple of 1024
+constexpr uint32_t kOffLrB = kOffLrA + kLrA;
+constexpr uint32_t kOffBar = kOffLrB + kLrB;
+constexpr uint32_t kSmemBytes = kOffBar + 256;
+
+// Tensor-memory columns: accumulator [0, 256), block scales after it.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemSfa = 256;                   // 4 columns per MMA, 4 MMAs per stage
+constexpr uint32_t kTmemSfb = 272;                   // 8 columns per MMA
+
+struct LinearArgs {
+    const uint8_t* a_sf;
+    const uint8_t* w_sf;
+    const float* D;
+    const uint16_t* up;
+    const uint16_t* bias;
+    void* Y;
+    int64_t ldy;
+    int64_t M, N, K;
+    const float* s_g_act;
+    const float* s_g_w;
+    int r;
+    int m_tiles, n_tiles;
+    uint32_t* err;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    return l | (h << 16);
+}
+
+template <bool kOutF32>
+__global__ void __launch_bounds__(kThreads, 1)
+linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+              LinearArgs args) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* empty = full + kStages;
+    uint64_t* acc_full = empty + kStages;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* lr_full = acc_empty + 1;
+    uint64_t* lr_empty = lr_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lr_empty + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const uint32_t lane = threadIdx.x & 31;
+    const int num_tiles = args.m_tiles * args.n_tiles;
+    const int k_stages = static_cast<int>(args.K / kBK);
+    const bool has_lr = args.r > 0;
+    const float alpha = __fmul_rn(__ldg(args.s_g_act), __ldg(args.s_g_w));
+    const float inv_alpha = __frcp_rn(alpha);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kEpiWarps);
+        mbar_init(lr_full, 1);
+        mbar_init(lr_empty, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmap_a);
+            prefetch_tmap(&tmap_b);
+            const int64_t atoms_k = args.K / 64;
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m_blk = tile % args.m_tiles;
+                const int n_blk = tile / args.m_tiles;
+                for (int kb = 0; kb < k_stages; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) { ok = false; break; }
+                    uint8_t* st = smem + kOffStages + s * kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], kStageBytes);
+                    tma_load_2d(st, &tmap_a, &full[s], kb * kBKBytes, m_blk * kBM);
+                    tma_load_2d(st + kATile, &tmap_b, &full[s], kb * kBKBytes, n_blk * kBN);
+                    bulk_load(st + kATile + kBTile, args.a_sf + (static_cast<int64_t>(m_blk) * atoms_k + kb * 4) * 512,
+                              kSfaTile, &full[s]);
+                    const uint8_t* sfb0 = args.w_sf + (static_cast<int64_t>(2 * n_blk) * atoms_k + kb * 4) * 512;
+                    bulk_load(st + kATile + kBTile + kSfaTile, sfb0, kSfbTile / 2, &full[s]);
+                    bulk_load(st + kATile + kBTile + kSfaTile + kSfbTile / 2, sfb0 + atoms_k * 512, kSfbTile / 2,
+                              &full[s]);
+                }
+            }
+            // Bounded drain of the copies still in flight.
+            for (int i = (it > kStages ? it - kStages : 0); i < it; ++i) {
+                const long long t0 = clock64();
+                while (!mbar_try_wait(&full[i % kStages], (i / kStages) & 1) && clock64() - t0 < kWaitLimitCycles) {}
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_f4 = idesc_nvf4(kBM, kBN);
+            const uint32_t idesc_lr = idesc_bf16(kBM, kBN);
+            int it = 0;
+            int local = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+                if (!mbar_wait(acc_empty, (local & 1) ^ 1, abort_flag, args.err, kErrWaitAccum)) break;
+                tc_fence_after();
+                bool first = true;
+                if (has_lr) {
+                    if (!mbar_wait(lr_full, local & 1, abort_flag, args.err, kErrWaitLowRank)) break;
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + kOffLrA);
+                    const uint32_t b0 = smem_u32(smem + kOffLrB);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc_lr,
+                                 kk > 0 ? 1u : 0u);
+                    tc_commit(lr_empty);
+                    first = false;
+                }
+                for (int kb = 0; kb < k_stages; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) { ok = false; break; }
+                    tc_fence_after();
+                    uint8_t* st = smem + kOffStages + s * kStageBytes;
+                    const uint32_t sfa = smem_u32(st + kATile + kBTile);
+                    const uint32_t sfb = sfa + kSfaTile;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        tc_cp_32x128b_x4(tmem + kTmemSfa + 4 * j, desc_sf_block(sfa + 512 * j));
+                        tc_cp_32x128b_x4(tmem + kTmemSfb + 8 * j, desc_sf_block(sfb + 512 * j));
+                        tc_cp_32x128b_x4(tmem + kTmemSfb + 8 * j + 4, desc_sf_block(sfb + kSfbTile / 2 + 512 * j));
+                    }
+                    const uint32_t a0 = smem_u32(st);
+                    const uint32_t b0 = smem_u32(st + kATile);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        mma_nvf4(tmem, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc_f4,
+                                 tmem + kTmemSfa + 4 * kk, tmem + kTmemSfb + 8 * kk, (first && kk == 0) ? 0u : 1u);
+                    }
+                    first = false;
+                    tc_commit(&empty[s]);
+                }
+                tc_commit(acc_full);
+            }
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ low-rank operand builder
+        if (has_lr) {
+            int local = 0;
+            const int r = args.r;
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+                const int m_blk = tile % args.m_tiles;
+                const int n_blk = tile / args.m_tiles;
+                if (!mbar_wait(lr_empty, (local & 1) ^ 1, abort_flag, args.err, kErrWaitLowRank)) break;
+                uint8_t* la = smem + kOffLrA;
+                uint8_t* lb = smem + kOffLrB;
+                // A: row = D'[m] as bf16 hi (channels 0..31) and lo (32..63)
+                for (int row = lane; row < kBM; row += 32) {
+                    const int64_t gm = static_cast<int64_t>(m_blk) * kBM + row;
+                    float dv[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) dv[j] = 0.0f;
+                    if (gm < args.M) {
+                        const float4* src = reinterpret_cast<const float4*>(args.D + gm * r);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (q * 4 < r) {
+                                const float4 v = __ldg(src + q);
+                                dv[4 * q] = v.x; dv[4 * q + 1] = v.y; dv[4 * q + 2] = v.z; dv[4 * q + 3] = v.w;
+                            }
+                        }
+                    }
+                    uint32_t hi[16], lo[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float x0 = __fmul_rn(dv[2 * j], inv_alpha);
+                        const float x1 = __fmul_rn(dv[2 * j + 1], inv_alpha);
+                        const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+                        const float r0 = __fsub_rn(x0, __bfloat162float(h0));
+                        const float r1 = __fsub_rn(x1, __bfloat162float(h1));
+                        hi[j] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                                (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+                        lo[j] = pack_bf16x2(r0, r1);
+                    }
+                    uint8_t* rowp = la + row * 128;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        *reinterpret_cast<uint4*>(rowp + ((c ^ (row & 7)) << 4)) =
+                            make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+                        *reinterpret_cast<uint4*>(rowp + (((c + 4) ^ (row & 7)) << 4)) =
+                            make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+                    }
+                }
+                // B: row n = [up[n, 0..31] | up[n, 0..31]] (zero beyond r)
+                for (int row = lane; row < kBN; row += 32) {
+                    const int64_t gn = static_cast<int64_t>(n_blk) * kBN + row;
+                    uint4 u[4];
+                    const uint4* src = reinterpret_cast<const uint4*>(args.up + gn * r);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) u[c] = (c * 8 < r) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+                    uint8_t* rowp = lb + row * 128;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        *reinterpret_cast<uint4*>(rowp + ((c ^ (row & 7)) << 4)) = u[c];
+                        *reinterpret_cast<uint4*>(rowp + (((c + 4) ^ (row & 7)) << 4)) = u[c];
+                    }
+                }
+                fence_async_shared();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(lr_full);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;                       // tensor-memory lane quarter of this warp
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            const int m_blk = tile % args.m_tiles;
+            const int n_blk = tile / args.m_tiles;
+            if (!mbar_wait(acc_full, local & 1, abort_flag, args.err, kErrWaitMma)) break;
+            tc_fence_after();
+            const int64_t row = static_cast<int64_t>(m_blk) * kBM + quarter * 32 + lane;
+            const int64_t col0 = static_cast<int64_t>(n_blk) * kBN;
+            const bool row_ok = row < args.M;
+            if constexpr (!kOutF32) {
+                uint32_t packed[kBN / 2];
+#pragma unroll
+                for (int c = 0; c < kBN / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase + c * 32, v);
+                    tmem_ld_wait();
+                    float b[32];
+                    if (args.bias) {
+                        const uint4* bp = reinterpret_cast<const uint4*>(args.bias + col0 + c * 32);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint4 w = __ldg(bp + q);
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                b[8 * q + 2 * e] = bf16_lo(ws[e]);
+                                b[8 * q + 2 * e + 1] = bf16_hi(ws[e]);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) b[j] = 0.0f;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float y0 = fmaf(alpha, __uint_as_float(v[2 * j]), b[2 * j]);
+                        const float y1 = fmaf(alpha, __uint_as_float(v[2 * j + 1]), b[2 * j + 1]);
+                        packed[c * 16 + j] = pack_bf16x2(y0, y1);
+                    }
+                }
+                // The accumulator has been read: let the next tile's MMAs start.
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty);
+                if (row_ok) {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(args.Y) + row * args.ldy + col0);
+#pragma unroll
+                    for (int q = 0; q < kBN / 8; ++q)
+                        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < kBN / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase + c * 32, v);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        float* dst = static_cast<float*>(args.Y) + row * args.ldy + col0 + c * 32;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            float y[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = 4 * q + e;
+                                const float bj = args.bias
+                                    ? __uint_as_float(static_cast<uint32_t>(args.bias[col0 + c * 32 + j]) << 16) : 0.0f;
+                                y[e] = fmaf(alpha, __uint_as_float(v[j]), bj);
+                            }
+                            reinterpret_cast<float4*>(dst)[q] = make_float4(y[0], y[1], y[2], y[3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty);
+            }
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <bool kOutF32>
+int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const LinearArgs& a, cudaStream_t st) {
+    const uint32_t smem = kSmemBytes + 1024;
+    auto kern = linear_kernel<kOutF32>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return SVDQ_ERR_CUDA;
+    const int tiles = a.m_tiles * a.n_tiles;
+    const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+    const int grid = tiles < sms ? tiles : sms;
+    kern<<<grid, kThreads, smem, st>>>(ta, tb, a);
+    return launch_status(cudaGetLastError());
+}
+
+}  // namespace
+}  // namespace svdq
+
+extern "C" int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g_act,
+                           const float* D, int r,
+                           const uint8_t* w_codes, const uint8_t* w_sf, const float* s_g_w,
+                           const void* up, const void* bias,
+                           void* Y, int64_t ldy, int out_dtype,
+                           int64_t M, int64_t N, int64_t K, void* stream) {
+    using namespace svdq;
+    if (a_codes == nullptr || a_sf == nullptr || w_codes == nullptr || w_sf == nullptr || Y == nullptr ||
+        s_g_act == nullptr || s_g_w == nullptr)
+        return SVDQ_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < 1 || ldy < N) return SVDQ_ERR_INVALID_ARG;
+    if (out_dtype != 0 && out_dtype != 1) return SVDQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(s_g_act) & 3u) || (reinterpret_cast<uintptr_t>(s_g_w) & 3u))
+        return SVDQ_ERR_MISALIGNED;
+    if (r != 0 && r != 16 && r != 32) return SVDQ_ERR_UNSUPPORTED;
+    if ((r > 0) != (D != nullptr) || (r > 0) != (up != nullptr)) return SVDQ_ERR_INVALID_ARG;
+    if (K % 256 != 0 || N % 256 != 0) return SVDQ_ERR_UNSUPPORTED;
+    if (M > (int64_t(1) << 31) - 128 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 30))
+        return SVDQ_ERR_UNSUPPORTED;
+    const int64_t m_tiles = (M + 127) / 128, n_tiles = N / 256;
+    if (m_tiles * n_tiles > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(Y))
+        return SVDQ_ERR_MISALIGNED;
+    if ((ldy * (out_dtype ? 4 : 2)) % 16 != 0) return SVDQ_ERR_MISALIGNED;
+    if (r > 0 && (!aligned16(D) || !aligned16(up))) return SVDQ_ERR_MISALIGNED;
+    if (bias && !aligned16(bias)) return SVDQ_ERR_MISALIGNED;
+    if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    uint32_t* err = device_error_word();
+    if (err == nullptr) return SVDQ_ERR_CUDA;
+
+    CUtensorMap ta, tb;
+    if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a_codes, K / 2, M, K / 2, 128, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_codes, K / 2, N, K / 2, 128, 256,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return SVDQ_ERR_CUDA;
+    LinearArgs a{};
+    a.a_sf = a_sf;
+    a.w_sf = w_sf;
+    a.D = D;
+    a.up = static_cast<const uint16_t*>(up);
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.Y = Y;
+    a.ldy = ldy;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.s_g_act = s_g_act;
+    a.s_g_w = s_g_w;
+    a.r = r;
+    a.m_tiles = static_cast<int>(m_tiles);
+    a.n_tiles = static_cast<int>(n_tiles);
+    a.err = err;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return out_dtype ? launch_linear<true>(ta, tb, a, st) : launch_linear<false>(ta, tb, a, st);
+}

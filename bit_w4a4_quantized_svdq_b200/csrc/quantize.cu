@@ -1,0 +1,373 @@
+// quantize.cu -- per-token NVFP4 quantisation of smoothed activations, fused
+// with the low-rank down-projection D = X down^T = (X / lambda) L1.
+//
+// "MiniMax-H3 NVFP4 -- what the smoothing scale should be calibrated on",
+// section "Why": 16 consecutive input channels share one FP8 (E4M3) scale set
+// by the group absmax, and the kernel sees X / lambda.  "MiniMax-H3 . SVDQuant
+// W4A4 (int4, rank 32, GPTQ)", opening section: activations are quantised per
+// token at run time and a 16-bit rank-32 branch carries the outliers.
+// "DeltaQuant on MiniMax-H3", section "The activation scale bound held": the
+// tensor scale is static and saturated groups are counted at run time.
+//
+// Layout of one CTA (6 warps) over a 128-row tile and a slice of K:
+//   warp 4      TMA producer: 128 x 64 bf16 tiles of X (128-byte swizzle) and
+//               the matching r x 64 tile of the down weight into a 4-stage ring
+//   warp 5      tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
+//   warps 0..3  quantisers: read the swizzled tile from shared memory, 2 lanes
+//               per 16-element group (amax by one shuffle), E4M3 scale and E2M1
+//               codes through the hardware RNE conversions, coalesced stores;
+//               finally read D_partial from tensor memory.
+// K is split across the CTAs of a thread-block cluster (up to 8); the partial
+// D tiles are summed in a fixed order through distributed shared memory, so D
+// is deterministic.  Memory traffic per element: 2 bytes in, 0.5625 out.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace svdq {
+namespace {
+
+constexpr int kBM = 128;               // rows per CTA tile
+constexpr int kBK = 64;                // channels per stage (128 bytes of bf16)
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kQuantWarps = 4;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kMaxSplit = 8;
+constexpr uint32_t kXTileBytes = kBM * kBK * 2;  // 16 KB
+
+template <int R>
+struct QSmem {
+    static constexpr uint32_t kDownTileBytes = R * kBK * 2;
+    static constexpr uint32_t kXOff = 0;
+    static constexpr uint32_t kDownOff = kStages * kXTileBytes;
+    static constexpr uint32_t kPartOff = kDownOff + kStages * kDownTileBytes;     // D partial [R][128] fp32
+    static constexpr uint32_t kBarOff = kPartOff + R * kBM * 4;
+    static constexpr uint32_t kBytes = kBarOff + 256;
+};
+
+struct QuantArgs {
+    const float* inv_lambda;
+    const float* s_g;
+    int64_t M, K;
+    uint8_t* codes;
+    uint8_t* sf;
+    float* D;
+    uint32_t* sat_count;
+    uint32_t* err;
+    int n_chunks;      // K / 64
+    int split;         // CTAs along K (cluster size when R > 0)
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads)
+quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_down,
+                    QuantArgs args) {
+    using L = QSmem<R>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+    uint64_t* empty = full + kStages;
+    uint64_t* dfull = empty + kStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dfull + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const uint32_t lane = threadIdx.x & 31;
+    const int m_blk = blockIdx.x;
+    const int ky = blockIdx.y;
+    const int c_begin = static_cast<int>(static_cast<int64_t>(ky) * args.n_chunks / args.split);
+    const int c_end = static_cast<int>(static_cast<int64_t>(ky + 1) * args.n_chunks / args.split);
+    const int n_local = c_end - c_begin;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kQuantWarps + (R > 0 ? 1 : 0));
+        }
+        mbar_init(dfull, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (R > 0 && warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, 32);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = (R > 0) ? *tmem_slot : 0u;
+
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            prefetch_tmap(&tmap_x);
+            if (R > 0) prefetch_tmap(&tmap_down);
+            int issued = 0;
+            for (int i = 0; i < n_local; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) break;
+                mbar_arrive_expect_tx(&full[s], kXTileBytes + L::kDownTileBytes);
+                const int col = (c_begin + i) * kBK;
+                tma_load_2d(smem + L::kXOff + s * kXTileBytes, &tmap_x, &full[s], col, m_blk * kBM);
+                if (R > 0)
+                    tma_load_2d(smem + L::kDownOff + s * L::kDownTileBytes, &tmap_down, &full[s], col, 0);
+                ++issued;
+            }
+            // Wait (bounded) for the copies still in flight before the CTA may exit.
+            for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i) {
+                const long long t0 = clock64();
+                while (!mbar_try_wait(&full[i % kStages], (i / kStages) & 1) && clock64() - t0 < kWaitLimitCycles) {}
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (R > 0 && lane == 0) {
+            const uint32_t idesc = idesc_bf16(kBM, R);
+            for (int i = 0; i < n_local; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(smem + L::kXOff + s * kXTileBytes);
+                const uint32_t b0 = smem_u32(smem + L::kDownOff + s * L::kDownTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)
+                    mma_bf16(tmem_d, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc,
+                             (i > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&empty[s]);
+            }
+            tc_commit(dfull);
+        }
+    } else {
+        // ------------------------------------------------------------ quantisers
+        const float s_g = __ldg(args.s_g);
+        const float d = __fmul_rn(6.0f, s_g);
+        const int64_t M = args.M, K = args.K;
+        const int64_t half_k = K >> 1;
+        const int64_t atoms_k = K >> 6;
+        uint32_t sat = 0;
+        const int c8 = lane & 7;           // 16-byte chunk of the 128-byte row this lane reads
+        const int rsub = lane >> 3;        // which of 4 rows this iteration
+        for (int i = 0; i < n_local; ++i) {
+            const int s = i % kStages;
+            const uint32_t ph = (i / kStages) & 1;
+            if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
+            const int chunk = c_begin + i;
+            const int64_t k0 = static_cast<int64_t>(chunk) * kBK + c8 * 8;
+            float il[8];
+            if (args.inv_lambda) {
+                const float4 a = __ldg(reinterpret_cast<const float4*>(args.inv_lambda + k0));
+                const float4 b = __ldg(reinterpret_cast<const float4*>(args.inv_lambda + k0 + 4));
+                il[0] = a.x; il[1] = a.y; il[2] = a.z; il[3] = a.w;
+                il[4] = b.x; il[5] = b.y; il[6] = b.z; il[7] = b.w;
+            }
+            const uint8_t* tile = smem + L::kXOff + s * kXTileBytes;
+#pragma unroll 2
+            for (int it = 0; it < 8; ++it) {
+                const int row = warp * 32 + it * 4 + rsub;                // row inside the tile
+                const uint4 v = *reinterpret_cast<const uint4*>(tile + row * 128 + ((c8 ^ (row & 7)) << 4));
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                float xs[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    xs[2 * j] = bf16_lo(w[j]);
+                    xs[2 * j + 1] = bf16_hi(w[j]);
+                }
+                if (args.inv_lambda) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) xs[j] = __fmul_rn(xs[j], il[j]);
+                }
+                float a = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(xs[j]));
+                a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));            // the other half of the group
+                const float t = __fdiv_rn(a, d);
+                const uint32_t sfb = cvt_e4m3(t);
+                const float S = __fmul_rn(e4m3_to_f32(sfb), s_g);
+                const float rS = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+                float q[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) q[j] = __fmul_rn(xs[j], rS);
+                const uint32_t packed = cvt_e2m1x8(q);
+                if ((c8 & 1) == 0 && t > 448.0f) ++sat;
+                // 4 scale bytes of this row and chunk -> one 32-bit word (lane c8 == 0 of the row)
+                uint32_t sfw = sfb;
+                sfw |= __shfl_down_sync(0xffffffffu, sfb, 2) << 8;
+                sfw |= __shfl_down_sync(0xffffffffu, sfb, 4) << 16;
+                sfw |= __shfl_down_sync(0xffffffffu, sfb, 6) << 24;
+                const int64_t grow = static_cast<int64_t>(m_blk) * kBM + row;
+                if (grow < M)
+                    *reinterpret_cast<uint32_t*>(args.codes + grow * half_k + chunk * (kBK / 2) + c8 * 4) = packed;
+                if (c8 == 0) {
+                    const int64_t off = (static_cast<int64_t>(m_blk) * atoms_k + chunk) * 512 + (row & 31) * 16 +
+                                        ((row >> 5) & 3) * 4;
+                    *reinterpret_cast<uint32_t*>(args.sf + off) = sfw;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        // saturation count: one atomic per warp
+        for (int o = 16; o > 0; o >>= 1) sat += __shfl_xor_sync(0xffffffffu, sat, o);
+        if (lane == 0 && sat && args.sat_count) atomicAdd(args.sat_count, sat);
+
+        if (R > 0) {
+            float* part = reinterpret_cast<float*>(smem + L::kPartOff);   // [R][128]
+            const int row = warp * 32 + lane;
+            if (mbar_wait(dfull, 0, abort_flag, args.err, kErrWaitMma)) {
+                tc_fence_after();
+                const uint32_t taddr = tmem_d + (static_cast<uint32_t>(warp * 32) << 16);
+                if constexpr (R == 32) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(taddr, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) part[j * kBM + row] = __uint_as_float(v[j]);
+                } else {
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(taddr, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) part[j * kBM + row] = __uint_as_float(v[j]);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < R; ++j) part[j * kBM + row] = 0.0f;
+            }
+            tc_fence_before();
+        }
+    }
+
+    __syncwarp();   // reconverge each warp before the warp-aligned cluster barrier
+    if constexpr (R > 0) {
+        // Sum the split-K partials in cluster-rank order (deterministic) on rank 0.
+        cluster_sync_all();
+        if (cluster_ctarank() == 0 && warp < kQuantWarps) {
+            const int row = warp * 32 + lane;
+            const int64_t grow = static_cast<int64_t>(m_blk) * kBM + row;
+            const uint32_t base = smem_u32(smem + L::kPartOff);
+            if (grow < args.M) {
+                float* dst = args.D + grow * R;
+#pragma unroll 4
+                for (int j = 0; j < R; j += 4) {
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int c = 0; c < args.split; ++c)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            acc[u] += ld_dsmem_f32(base + ((j + u) * kBM + row) * 4, c);
+                    *reinterpret_cast<float4*>(dst + j) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                }
+            }
+        }
+        cluster_sync_all();
+        if (warp == kMmaWarp) {
+            tc_fence_after();
+            tmem_dealloc(tmem_d, 32);
+        }
+    }
+}
+
+template <int R>
+int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const QuantArgs& base, const void* down,
+                    cudaStream_t st) {
+    CUtensorMap tx, td;
+    if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, K, M, ldx * 2, kBK, kBM,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return SVDQ_ERR_CUDA;
+    if (R > 0) {
+        if (!encode_tmap_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, down, K, R, K * 2, kBK, R,
+                            CU_TENSOR_MAP_SWIZZLE_128B))
+            return SVDQ_ERR_CUDA;
+    } else {
+        td = tx;
+    }
+    QuantArgs a = base;
+    a.n_chunks = static_cast<int>(K / kBK);
+    const int64_t m_tiles = (M + kBM - 1) / kBM;
+    // Split K so the grid covers the GPU about twice over, up to a cluster of 8.
+    const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+    int split = static_cast<int>((2 * sms + m_tiles - 1) / m_tiles);
+    split = split < 1 ? 1 : (split > kMaxSplit ? kMaxSplit : split);
+    if (split > a.n_chunks) split = a.n_chunks;
+    a.split = split;
+    if (m_tiles > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
+
+    const uint32_t smem = QSmem<R>::kBytes + 1024;
+    auto kern = quantize_act_kernel<R>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return SVDQ_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(m_tiles), static_cast<unsigned>(split), 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (R > 0) ? split : 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return launch_status(cudaLaunchKernelEx(&cfg, kern, tx, td, a));
+}
+
+}  // namespace
+}  // namespace svdq
+
+extern "C" int svdq_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx,
+                                 const float* inv_lambda, const float* s_g,
+                                 const void* down, int r,
+                                 uint8_t* codes, uint8_t* sf, float* D, uint32_t* sat_count,
+                                 void* stream) {
+    using namespace svdq;
+    if (X == nullptr || codes == nullptr || sf == nullptr || s_g == nullptr) return SVDQ_ERR_INVALID_ARG;
+    if (M < 1 || K < 64 || ldx < K) return SVDQ_ERR_INVALID_ARG;
+    if (K % 64 != 0) return SVDQ_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(s_g) & 3u) return SVDQ_ERR_MISALIGNED;
+    if (r != 0 && r != 16 && r != 32) return SVDQ_ERR_UNSUPPORTED;
+    if ((r > 0) != (down != nullptr) || (r > 0) != (D != nullptr)) return SVDQ_ERR_INVALID_ARG;
+    if (M > (int64_t(1) << 31) - 128 || K > (int64_t(1) << 30)) return SVDQ_ERR_UNSUPPORTED;
+    if (!aligned16(X) || (ldx * 2) % 16 != 0 || !aligned16(codes) || !aligned16(sf)) return SVDQ_ERR_MISALIGNED;
+    if (inv_lambda && !aligned16(inv_lambda)) return SVDQ_ERR_MISALIGNED;
+    if (r > 0 && (!aligned16(down) || !aligned16(D))) return SVDQ_ERR_MISALIGNED;
+    if (sat_count && (reinterpret_cast<uintptr_t>(sat_count) & 3u)) return SVDQ_ERR_MISALIGNED;
+    if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    uint32_t* err = device_error_word();
+    if (err == nullptr) return SVDQ_ERR_CUDA;
+    QuantArgs a{};
+    a.inv_lambda = inv_lambda;
+    a.s_g = s_g;
+    a.M = M;
+    a.K = K;
+    a.codes = codes;
+    a.sf = sf;
+    a.D = D;
+    a.sat_count = sat_count;
+    a.err = err;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // Rows of the last 128-row block beyond M hold zero scale bytes: the kernel
+    // writes every row of every tile (zero-filled by TMA), so no memset is needed.
+    switch (r) {
+        case 0: return launch_quantize<0>(X, M, K, ldx, a, down, st);
+        case 16: return launch_quantize<16>(X, M, K, ldx, a, down, st);
+        default: return launch_quantize<32>(X, M, K, ldx, a, down, st);
+    }
+}

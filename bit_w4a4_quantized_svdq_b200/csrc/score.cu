@@ -1,0 +1,190 @@
+// score.cu -- per-segment relative L2 error of a quantised layer output
+// against the bf16 layer ("MiniMax-H3 NVFP4 -- what the smoothing scale should
+// be calibrated on", section "The metric that picks the winner also hides the
+// cost": candidates scored by rel-L2 vs bf16 on proportional rows and on 4096
+// rows per modality).
+//
+// Bandwidth-bound two-pass reduction with a fixed order, so results are
+// bitwise reproducible: pass 1 gives every (segment, row chunk) one block that
+// writes fp64 partial sums to the caller's workspace; pass 2 sums each
+// segment's partials in index order and forms num, den and rel.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace svdq {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int64_t kElemsPerChunk = 1 << 17;        // elements a partial-sum block covers
+
+struct ChunkPlan {
+    int n;                                           // segments
+    int64_t begin[kMaxSegments];                     // first row of segment s
+    int64_t end[kMaxSegments];
+    int64_t rows_per_chunk;                          // rows one block sums
+    int64_t chunk_prefix[kMaxSegments + 1];          // first chunk index of segment s
+};
+
+inline int64_t rows_per_chunk_for(int64_t N) {
+    const int64_t r = kElemsPerChunk / (N > 0 ? N : 1);
+    return r < 1 ? 1 : r;
+}
+
+inline void make_plan(const svdq_seg* segs, int n_seg, int64_t N, ChunkPlan* p) {
+    p->n = n_seg;
+    p->rows_per_chunk = rows_per_chunk_for(N);
+    p->chunk_prefix[0] = 0;
+    for (int s = 0; s < n_seg; ++s) {
+        p->begin[s] = segs[s].begin;
+        p->end[s] = segs[s].end;
+        const int64_t rows = segs[s].end - segs[s].begin;
+        const int64_t chunks = rows > 0 ? (rows + p->rows_per_chunk - 1) / p->rows_per_chunk : 1;
+        p->chunk_prefix[s + 1] = p->chunk_prefix[s] + chunks;
+    }
+}
+
+__device__ __forceinline__ double block_sum(double v, double* sh) {
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) sh[w] = v;
+    __syncthreads();
+    v = (threadIdx.x < (kThreads >> 5)) ? sh[threadIdx.x] : 0.0;
+    if (w == 0)
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;   // valid in thread 0
+}
+
+__global__ void __launch_bounds__(kThreads)
+score_partial_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict__ yr, int64_t N, int64_t ld,
+                     ChunkPlan plan, double* __restrict__ partial) {
+    __shared__ double sh[kThreads / 32];
+    const int64_t chunk = blockIdx.x;
+    int s = 0;
+    while (s + 1 < plan.n && chunk >= plan.chunk_prefix[s + 1]) ++s;
+    const int64_t r0 = plan.begin[s] + (chunk - plan.chunk_prefix[s]) * plan.rows_per_chunk;
+    const int64_t r1 = min(r0 + plan.rows_per_chunk, plan.end[s]);
+    double num = 0.0, den = 0.0;
+    const bool vec = (N % 8 == 0);
+    for (int64_t row = r0; row < r1; ++row) {
+        const uint16_t* a = yq + row * ld;
+        const uint16_t* b = yr + row * ld;
+        if (vec) {
+            for (int64_t c = static_cast<int64_t>(threadIdx.x) * 8; c < N; c += kThreads * 8) {
+                const uint4 qa = *reinterpret_cast<const uint4*>(a + c);
+                const uint4 qb = *reinterpret_cast<const uint4*>(b + c);
+                const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
+                const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const double r_lo = bf16_lo(wb[i]), r_hi = bf16_hi(wb[i]);
+                    const double d_lo = static_cast<double>(bf16_lo(wa[i])) - r_lo;
+                    const double d_hi = static_cast<double>(bf16_hi(wa[i])) - r_hi;
+                    num = fma(d_lo, d_lo, num);
+                    num = fma(d_hi, d_hi, num);
+                    den = fma(r_lo, r_lo, den);
+                    den = fma(r_hi, r_hi, den);
+                }
+            }
+        } else {
+            for (int64_t c = threadIdx.x; c < N; c += kThreads) {
+                const double r = __uint_as_float(static_cast<uint32_t>(b[c]) << 16);
+                const double d = static_cast<double>(__uint_as_float(static_cast<uint32_t>(a[c]) << 16)) - r;
+                num = fma(d, d, num);
+                den = fma(r, r, den);
+            }
+        }
+    }
+    num = block_sum(num, sh);
+    den = block_sum(den, sh);
+    if (threadIdx.x == 0) {
+        partial[2 * chunk] = num;
+        partial[2 * chunk + 1] = den;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+score_finalize_kernel(ChunkPlan plan, const double* __restrict__ partial, double* __restrict__ num_out,
+                      double* __restrict__ den_out, double* __restrict__ rel_out) {
+    __shared__ double sh[kThreads / 32];
+    const int s = blockIdx.x;
+    double num = 0.0, den = 0.0;
+    for (int64_t c = plan.chunk_prefix[s] + threadIdx.x; c < plan.chunk_prefix[s + 1]; c += kThreads) {
+        num += partial[2 * c];
+        den += partial[2 * c + 1];
+    }
+    num = block_sum(num, sh);
+    den = block_sum(den, sh);
+    if (threadIdx.x == 0) {
+        num_out[s] = num;
+        den_out[s] = den;
+        double rel;
+        if (den > 0.0) rel = sqrt(num / den);
+        else rel = (num == 0.0) ? 0.0 : __longlong_as_double(0x7FF0000000000000LL);
+        rel_out[s] = rel;
+    }
+}
+
+}  // namespace
+
+// Shared by the entry point below; `partial` must hold 2 doubles per chunk.
+int score_lambda_launch(const void* Yq, const void* Yref, int64_t M, int64_t N, int64_t ld,
+                        const svdq_seg* segs, int n_seg, double* num, double* den, double* rel,
+                        double* partial, size_t partial_bytes, cudaStream_t cs) {
+    ChunkPlan plan;
+    make_plan(segs, n_seg, N, &plan);
+    const int64_t chunks = plan.chunk_prefix[n_seg];
+    if (partial_bytes < static_cast<size_t>(chunks) * 2 * sizeof(double)) return SVDQ_ERR_INVALID_ARG;
+    if (chunks > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
+    score_partial_kernel<<<static_cast<unsigned>(chunks), kThreads, 0, cs>>>(
+        static_cast<const uint16_t*>(Yq), static_cast<const uint16_t*>(Yref), N, ld, plan, partial);
+    if (cudaGetLastError() != cudaSuccess) return SVDQ_ERR_CUDA;
+    score_finalize_kernel<<<n_seg, kThreads, 0, cs>>>(plan, partial, num, den, rel);
+    return launch_status(cudaGetLastError());
+}
+
+int score_lambda_check(const void* Yq, const void* Yref, int64_t M, int64_t N, int64_t ld,
+                       const svdq_seg* segs, int n_seg, const double* num, const double* den,
+                       const double* rel) {
+    if (Yq == nullptr || Yref == nullptr || num == nullptr || den == nullptr || rel == nullptr)
+        return SVDQ_ERR_INVALID_ARG;
+    if (segs == nullptr || n_seg < 1 || n_seg > kMaxSegments) return SVDQ_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || ld < N) return SVDQ_ERR_INVALID_ARG;
+    for (int s = 0; s < n_seg; ++s)
+        if (segs[s].begin < 0 || segs[s].end < segs[s].begin || segs[s].end > M) return SVDQ_ERR_INVALID_ARG;
+    if (!aligned16(Yq) || !aligned16(Yref) || (ld * 2) % 16 != 0) return SVDQ_ERR_MISALIGNED;
+    return SVDQ_OK;
+}
+
+size_t score_partial_bytes(const svdq_seg* segs, int n_seg, int64_t N) {
+    if (segs == nullptr || n_seg < 1 || n_seg > kMaxSegments) return 0;
+    const int64_t rpc = rows_per_chunk_for(N);
+    int64_t chunks = 0;
+    for (int s = 0; s < n_seg; ++s) {
+        const int64_t rows = segs[s].end - segs[s].begin;
+        chunks += rows > 0 ? (rows + rpc - 1) / rpc : 1;
+    }
+    return static_cast<size_t>(chunks) * 2 * sizeof(double);
+}
+
+}  // namespace svdq
+
+extern "C" size_t svdq_score_workspace_bytes(const svdq_seg* segs, int n_seg, int64_t N) {
+    const size_t b = svdq::score_partial_bytes(segs, n_seg, N);
+    return b == 0 ? 0 : (b + 255) / 256 * 256;
+}
+
+extern "C" int svdq_score_lambda(const void* Yq, const void* Yref, int64_t M, int64_t N, int64_t ld,
+                                 const svdq_seg* segs, int n_seg,
+                                 double* num, double* den, double* rel,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    using namespace svdq;
+    int st = score_lambda_check(Yq, Yref, M, N, ld, segs, n_seg, num, den, rel);
+    if (st != SVDQ_OK) return st;
+    if (workspace == nullptr) return SVDQ_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return SVDQ_ERR_MISALIGNED;
+    if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    return score_lambda_launch(Yq, Yref, M, N, ld, segs, n_seg, num, den, rel,
+                               static_cast<double*>(workspace), workspace_bytes,
+                               static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,158 @@
+"""Python binding of the C ABI, one function per entry point, same names.
+
+Argument marshalling only: torch tensors provide device memory and the
+current CUDA stream; every computation runs in ``libsvdq.so``.  bf16 tensors
+may be ``torch.bfloat16`` or raw ``int16``/``uint16`` bit patterns.
+"""
+from __future__ import annotations
+
+from ctypes import byref, c_uint32
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+from . import _lib
+
+Segs = Optional[Sequence[Tuple[int, int]]]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check_bf16(t: torch.Tensor, name: str) -> None:
+    if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"{name} must be bf16 (or its 16-bit pattern), got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _row_stride(t: torch.Tensor, name: str) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a row-major 2-D tensor")
+    return t.stride(0)
+
+
+def sf_bytes(rows: int, k: int) -> int:
+    return int(_lib.load().svdq_sf_bytes(rows, k))
+
+
+def svdq_calib_lambda(x: torch.Tensor, segs: Segs = None, w: Optional[torch.Tensor] = None,
+                      stream=None) -> dict:
+    """Per-channel absmax, lambda, 1/lambda and the static tensor scale (device tensors)."""
+    lib = _lib.load()
+    _check_bf16(x, "x")
+    m, k = x.shape
+    ldx = _row_stride(x, "x")
+    dev = x.device
+    ax = torch.empty(k, dtype=torch.float32, device=dev)
+    aw = torch.empty(k, dtype=torch.float32, device=dev) if w is not None else None
+    lam = torch.empty(k, dtype=torch.float32, device=dev)
+    inv = torch.empty(k, dtype=torch.float32, device=dev)
+    s_g = torch.empty(1, dtype=torch.float32, device=dev)
+    if w is not None:
+        _check_bf16(w, "w")
+        n, ldw = w.shape[0], _row_stride(w, "w")
+    else:
+        n, ldw = 0, 0
+    arr, n_seg = _lib.seg_array(segs)
+    _lib.check("svdq_calib_lambda", lib.svdq_calib_lambda(
+        _ptr(x), m, k, ldx, arr, n_seg, _ptr(w), n, ldw,
+        _ptr(ax), _ptr(aw), _ptr(lam), _ptr(inv), _ptr(s_g), _stream(stream)))
+    return dict(amax_x=ax, amax_w=aw, lam=lam, inv_lam=inv, s_g=s_g)
+
+
+def svdq_quantize_act(x: torch.Tensor, inv_lambda: Optional[torch.Tensor], s_g: torch.Tensor,
+                      down: Optional[torch.Tensor] = None, sat_count: Optional[torch.Tensor] = None,
+                      out: Optional[dict] = None, stream=None) -> dict:
+    """NVFP4 codes, scale bytes (tensor-core layout) and D = x down^T."""
+    lib = _lib.load()
+    _check_bf16(x, "x")
+    m, k = x.shape
+    ldx = _row_stride(x, "x")
+    r = 0 if down is None else int(down.shape[0])
+    dev = x.device
+    if out is None:
+        out = dict(codes=torch.empty((m, k // 2), dtype=torch.uint8, device=dev),
+                   sf=torch.empty(sf_bytes(m, k), dtype=torch.uint8, device=dev),
+                   d=torch.empty((m, r), dtype=torch.float32, device=dev) if r else None)
+    _lib.check("svdq_quantize_act", lib.svdq_quantize_act(
+        _ptr(x), m, k, ldx, _ptr(inv_lambda), _ptr(s_g), _ptr(down), r,
+        _ptr(out["codes"]), _ptr(out["sf"]), _ptr(out["d"]), _ptr(sat_count), _stream(stream)))
+    return out
+
+
+def svdq_linear(a_codes: torch.Tensor, a_sf: torch.Tensor, s_g_act: torch.Tensor, d: Optional[torch.Tensor],
+                w_codes: torch.Tensor, w_sf: torch.Tensor, s_g_w: torch.Tensor, up: Optional[torch.Tensor],
+                bias: Optional[torch.Tensor], out_dtype: torch.dtype = torch.bfloat16,
+                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y = s_g_act s_g_w deq(A) deq(W)^T + D up^T + bias."""
+    lib = _lib.load()
+    m, kh = a_codes.shape
+    n = w_codes.shape[0]
+    k = 2 * kh
+    r = 0 if d is None else int(d.shape[1])
+    if out is None:
+        out = torch.empty((m, n), dtype=out_dtype, device=a_codes.device)
+    ldy = _row_stride(out, "out")
+    code = {torch.bfloat16: 0, torch.float32: 1}[out.dtype]
+    _lib.check("svdq_linear", lib.svdq_linear(
+        _ptr(a_codes), _ptr(a_sf), _ptr(s_g_act), _ptr(d), r, _ptr(w_codes), _ptr(w_sf), _ptr(s_g_w),
+        _ptr(up), _ptr(bias), _ptr(out), ldy, code, m, n, k, _stream(stream)))
+    return out
+
+
+def score_workspace_bytes(segs: Sequence[Tuple[int, int]], n: int) -> int:
+    arr, n_seg = _lib.seg_array(segs)
+    return int(_lib.load().svdq_score_workspace_bytes(arr, n_seg, n))
+
+
+def svdq_score_lambda(yq: torch.Tensor, yref: torch.Tensor, segs: Sequence[Tuple[int, int]],
+                      workspace: Optional[torch.Tensor] = None, stream=None):
+    """Per-segment (num, den, rel) fp64 device tensors."""
+    lib = _lib.load()
+    _check_bf16(yq, "yq")
+    _check_bf16(yref, "yref")
+    m, n = yq.shape
+    ld = _row_stride(yq, "yq")
+    if _row_stride(yref, "yref") != ld:
+        raise ValueError("yq and yref must share a row stride")
+    arr, n_seg = _lib.seg_array(segs)
+    dev = yq.device
+    num = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    den = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    rel = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    need = score_workspace_bytes(segs, n)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _lib.check("svdq_score_lambda", lib.svdq_score_lambda(
+        _ptr(yq), _ptr(yref), m, n, ld, arr, n_seg, _ptr(num), _ptr(den), _ptr(rel),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return num, den, rel
+
+
+def svdq_residual(w: torch.Tensor, lam: Optional[torch.Tensor], down: Optional[torch.Tensor],
+                  up: Optional[torch.Tensor], stream=None) -> torch.Tensor:
+    """R = bf16(W diag(lambda) - (diag(lambda) down^T up^T)^T), computed in fp64."""
+    lib = _lib.load()
+    _check_bf16(w, "w")
+    n, k = w.shape
+    r = 0 if down is None else int(down.shape[0])
+    out = torch.empty((n, k), dtype=torch.bfloat16, device=w.device)
+    _lib.check("svdq_residual", lib.svdq_residual(
+        _ptr(w), n, k, _row_stride(w, "w"), _ptr(lam), _ptr(down), _ptr(up), r, _ptr(out), _stream(stream)))
+    return out
+
+
+def svdq_device_error(stream=None) -> int:
+    """Synchronise and return (then clear) the device error word; 0 = no timeout."""
+    code = c_uint32(0)
+    st = _lib.load().svdq_device_error(_stream(stream), byref(code))
+    if st not in (_lib.SVDQ_OK, _lib.SVDQ_ERR_TIMEOUT):
+        _lib.check("svdq_device_error", st)
+    return int(code.value)

@@ -1,0 +1,224 @@
+/*
+ * svdq.h -- C ABI of the B200 (sm_100a) SVDQuant-style NVFP4 W4A4 linear layer.
+ *
+ * The layer computes
+ *
+ *     Y = (X / lambda) Q(W lambda - L1 L2)^T + (X / lambda) L1 L2 + b
+ *
+ * with activations quantised per token at run time to NVFP4 (E2M1 values, one
+ * E4M3 scale per 16 consecutive input channels, one FP32 tensor scale) and an
+ * NVFP4 residual weight.  Sources, by page title and section:
+ *   - "MiniMax-H3 NVFP4 -- what the smoothing scale should be calibrated on",
+ *     section "Why": 16 consecutive channels share one FP8 scale set by the
+ *     group absmax; the kernel sees X / lambda; W * lambda is shared.
+ *   - same page, section "Calibration": lambda from activation absmax
+ *     statistics accumulated under a modality (row) mask.
+ *   - same page, section "The metric that picks the winner also hides the
+ *     cost": candidates scored by relative L2 against bf16 on row sets.
+ *   - "MiniMax-H3 . SVDQuant W4A4 (int4, rank 32, GPTQ)", opening section:
+ *     16-bit rank-32 low-rank branch absorbs outliers, 4-bit residual,
+ *     per-token activation quantisation, one fused kernel.
+ *   - "DeltaQuant on MiniMax-H3", section "The activation scale bound held":
+ *     static activation global scale from a bound, saturated groups counted.
+ *
+ * Conventions for every call
+ *   - All pointers marked "device" are CUDA device pointers owned by the
+ *     caller; the library allocates no device memory.  Host pointers are read
+ *     during the call only.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; the return value reports
+ *     argument validation and launch errors only.
+ *   - Matrices are row-major; leading dimensions are in elements.  bf16
+ *     tensors are raw 16-bit patterns.  Device pointers must be 16-byte
+ *     aligned and row strides multiples of 16 bytes (SVDQ_ERR_MISALIGNED).
+ *   - Kernels bound every wait; a wait that runs out records a code in a
+ *     per-device error word, read (and cleared) by svdq_device_error().
+ *   - No exception crosses the ABI.  Status codes are svdq_status values.
+ *
+ * Storage formats
+ *   - Packed codes: uint8 [rows, K/2]; element 2i in the low nibble, 2i+1 in
+ *     the high nibble; E2M1 code = sign bit 3, magnitude codes 0..7 for
+ *     {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+ *   - Scale bytes (E4M3, OCP E4M3FN) in the tensor-core scale-factor layout:
+ *     rows padded to a multiple of 128; for each 128-row block and each group
+ *     of 4 scales along K (64 channels) one 512-byte atom holding row r's 4
+ *     bytes at (r % 32) * 16 + (r / 32 % 4) * 4; atoms ordered K-block fastest.
+ *     Size: svdq_sf_bytes(rows, K).  Pad rows are written as zero.
+ *   - Low-rank branch: "down" weight = L1s^T, bf16 [r, K], with lambda folded
+ *     in (L1s = diag(1/lambda) L1, so X down^T = (X / lambda) L1), and "up"
+ *     weight = L2^T, bf16 [N, r]; r is 0, 16 or 32.
+ */
+#ifndef SVDQ_H
+#define SVDQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SVDQ_OK = 0,
+    SVDQ_ERR_INVALID_ARG = 1,   /* null pointer required by the shape, bad size or value */
+    SVDQ_ERR_UNSUPPORTED = 2,   /* shape outside what the kernels implement */
+    SVDQ_ERR_MISALIGNED = 3,    /* pointer or row stride not 16-byte aligned */
+    SVDQ_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, attribute) */
+    SVDQ_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out */
+    SVDQ_ERR_NO_DEVICE = 6      /* no sm_100 device is current */
+} svdq_status;
+
+/* Half-open row range [begin, end) of X; a host array of these selects rows. */
+typedef struct {
+    int64_t begin;
+    int64_t end;
+} svdq_seg;
+
+/* Human-readable name of a status code (static string). */
+const char* svdq_status_string(int status);
+
+/* ABI version (major * 100 + minor). */
+int svdq_version(void);
+
+/* Bytes of a scale-factor buffer for `rows` rows of K channels:
+ * ceil(rows / 128) * 128 * K / 16.  Returns 0 if K is not a multiple of 64. */
+size_t svdq_sf_bytes(int64_t rows, int64_t K);
+
+/*
+ * svdq_calib_lambda -- per-channel absmax statistics, smoothing scale and the
+ * static activation tensor scale ("MiniMax-H3 NVFP4 ...", sections
+ * "Calibration" and "Why"; "DeltaQuant on MiniMax-H3", section "The
+ * activation scale bound held").
+ *
+ *   amax_x[j]    = max over the selected rows i of |X[i, j]|
+ *   amax_w[j]    = max over n of |W[n, j]|                  (if W != NULL)
+ *   lambda[j]    = RN32(sqrt(RN32(amax_x[j] / amax_w[j]))), or 1 if either is 0
+ *                  (lambda = 1 for every j when W == NULL)
+ *   inv_lambda[j]= RN32(1 / lambda[j])
+ *   s_g[0]       = RN32(max_j RN32(amax_x[j] * inv_lambda[j]) / 2688), or 1 if that max is 0
+ *
+ * X: device bf16 [M, K] with row stride ldx (elements).  segs: host array of
+ * n_seg row ranges selecting the calibration rows (segs == NULL and n_seg == 0
+ * selects all rows); ranges must lie in [0, M] and begin <= end; at most 64.
+ * W: device bf16 [N, K] with row stride ldw, or NULL.  Outputs (device fp32):
+ * amax_x [K], amax_w [K] (ignored and may be NULL when W is NULL), lambda [K],
+ * inv_lambda [K] (may be NULL), s_g [1].  K must be a multiple of 8.
+ * All reductions are exact (max), so results do not depend on launch shape.
+ */
+int svdq_calib_lambda(const void* X, int64_t M, int64_t K, int64_t ldx,
+                      const svdq_seg* segs, int n_seg,
+                      const void* W, int64_t N, int64_t ldw,
+                      float* amax_x, float* amax_w, float* lambda, float* inv_lambda,
+                      float* s_g, void* stream);
+
+/*
+ * svdq_quantize_act -- smooth and quantise activations per token to NVFP4 and
+ * produce the low-rank down-projection ("MiniMax-H3 NVFP4 ...", section "Why";
+ * "MiniMax-H3 . SVDQuant W4A4", opening section).
+ *
+ * For each row i and each group g of 16 consecutive channels:
+ *   xs   = RN32(X[i, k] * inv_lambda[k])            (inv_lambda == NULL: xs = X)
+ *   a    = max |xs| over the group;  t = RN32(a / RN32(6 * s_g))
+ *   sf   = E4M3 round-to-nearest-even of t, saturating at 448
+ *   S    = RN32(decode(sf) * s_g);  rS = S == 0 ? 0 : RN32(1 / S)
+ *   code = E2M1 round-to-nearest-even of RN32(xs * rS) (ties to even code,
+ *          |.| > 6 saturates, sign bit kept, so a zero scale gives signed zeros)
+ *   D[i, :] = sum_k X[i, k] * down[:, k]  (fp32 accumulation of bf16 products)
+ *
+ * X: device bf16 [M, K], row stride ldx.  inv_lambda: device fp32 [K] or NULL.
+ * s_g: device fp32 [1], the tensor scale (positive and finite; read by the
+ * kernel, so a value svdq_calib_lambda just wrote needs no host round trip).  down: device bf16 [r, K] (row stride K),
+ * NULL iff r == 0; r in {0, 16, 32}.  codes: device uint8 [M, K/2] (row stride
+ * K/2).  sf: device uint8 of svdq_sf_bytes(M, K) bytes.  D: device fp32
+ * [M, r] (row stride r), NULL iff r == 0.  sat_count: device uint32 (or NULL);
+ * the number of groups whose scale saturated (t > 448) is ADDED to it.
+ * K must be a multiple of 64; M >= 1.  Codes and scale bytes are
+ * deterministic; D's fp32 sums are deterministic for a given (M, K, r).
+ */
+int svdq_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx,
+                      const float* inv_lambda, const float* s_g,
+                      const void* down, int r,
+                      uint8_t* codes, uint8_t* sf, float* D, uint32_t* sat_count,
+                      void* stream);
+
+/*
+ * svdq_linear -- the fused W4A4 GEMM with the low-rank branch and bias in its
+ * epilogue ("MiniMax-H3 . SVDQuant W4A4", opening section and "Measured").
+ *
+ *   Y[m, n] = s_g_act * s_g_w * sum_k deq(A)[m, k] deq(Wq)[n, k]
+ *           + sum_j D[m, j] up[n, j] + bias[n]
+ *
+ * where deq() multiplies each E2M1 code by its E4M3 group scale.  The main
+ * product runs on the tcgen05 block-scaled FP4 tensor-core path with fp32
+ * accumulation in tensor memory; the low-rank term is added in the same
+ * accumulator (D split into two bf16 halves); bias and the tensor scales are
+ * applied in the epilogue.
+ *
+ * s_g_act, s_g_w: device fp32 [1] tensor scales (positive, finite); alpha =
+ * RN32(s_g_act * s_g_w) is formed on the device.
+ * a_codes: device uint8 [M, K/2]; a_sf: device scale bytes (svdq_sf_bytes(M, K));
+ * w_codes: device uint8 [N, K/2]; w_sf: device scale bytes (svdq_sf_bytes(N, K));
+ * D: device fp32 [M, r] (row stride r), NULL iff r == 0; up: device bf16 [N, r]
+ * (row stride r), NULL iff r == 0; bias: device bf16 [N] or NULL.
+ * Y: device [M, N] with row stride ldy; out_dtype 0 = bf16 (round to nearest
+ * even), 1 = fp32.  Requirements: K % 256 == 0, N % 256 == 0, M >= 1,
+ * r in {0, 16, 32}; otherwise SVDQ_ERR_UNSUPPORTED.
+ */
+int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g_act,
+                const float* D, int r,
+                const uint8_t* w_codes, const uint8_t* w_sf, const float* s_g_w,
+                const void* up, const void* bias,
+                void* Y, int64_t ldy, int out_dtype,
+                int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * svdq_score_workspace_bytes -- device workspace svdq_score_lambda needs for
+ * these segments and N columns (a multiple of 256 bytes, at least 256).
+ */
+size_t svdq_score_workspace_bytes(const svdq_seg* segs, int n_seg, int64_t N);
+
+/*
+ * svdq_score_lambda -- per-segment relative L2 error against the bf16 layer
+ * ("MiniMax-H3 NVFP4 ...", section "The metric that picks the winner also
+ * hides the cost").  For each segment s (rows [begin, end), all N columns):
+ *   num[s] = sum (Yq - Yref)^2,  den[s] = sum Yref^2,  rel[s] = sqrt(num / den)
+ * (rel = 0 when num == den == 0, +inf when only den == 0), accumulated in fp64.
+ *
+ * Yq, Yref: device bf16 [M, N] with row stride ld.  segs: host array (<= 64
+ * ranges inside [0, M]).  num, den, rel: device fp64 [n_seg].  workspace:
+ * device memory of at least svdq_score_workspace_bytes(segs, n_seg, N) bytes
+ * (scratch for per-block partial sums; contents on entry are ignored).
+ * The reduction order is fixed, so results are bitwise reproducible.
+ */
+int svdq_score_lambda(const void* Yq, const void* Yref, int64_t M, int64_t N, int64_t ld,
+                      const svdq_seg* segs, int n_seg,
+                      double* num, double* den, double* rel,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * svdq_residual -- offline weight conversion: the residual the 4-bit weight
+ * encodes ("MiniMax-H3 . SVDQuant W4A4", opening section):
+ *   R[n, k] = bf16(fp32( W[n, k] * lambda[k] - lambda[k] * sum_j down[j, k] * up[n, j] ))
+ * computed in fp64 with the j sum in order.  W: device bf16 [N, K] (row
+ * stride ldw); lambda: device fp32 [K] (NULL = 1); down: device bf16 [r, K];
+ * up: device bf16 [N, r]; r in [0, 32]; R: device bf16 [N, K] (row stride K).
+ * Quantise R with svdq_calib_lambda (W = NULL) and svdq_quantize_act
+ * (inv_lambda = NULL, r = 0) to obtain the weight codes, scales and s_g_w.
+ */
+int svdq_residual(const void* W, int64_t N, int64_t K, int64_t ldw, const float* lambda,
+                  const void* down, const void* up, int r, void* R, void* stream);
+
+/*
+ * svdq_device_error -- synchronise `stream`, then read and clear the current
+ * device's error word.  *code receives 0 when no bounded wait ran out since
+ * the last call, otherwise a nonzero code naming the wait.  Returns
+ * SVDQ_ERR_TIMEOUT if *code != 0, SVDQ_OK otherwise (SVDQ_ERR_CUDA if the
+ * synchronisation itself failed).
+ */
+int svdq_device_error(void* stream, uint32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H */

@@ -1,0 +1,132 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point ``include/svdq.h`` declares, sizes and status strings are
+right, and invalid arguments are rejected before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_w4a4_quantized_svdq_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "svdq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(svdq_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = _declared_functions()
+    assert len(names) >= 10
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_version_and_status_strings():
+    lib = _lib.load()
+    assert lib.svdq_version() == 100
+    assert lib.svdq_status_string(0) == b"ok"
+    assert lib.svdq_status_string(3) == b"misaligned pointer or stride"
+    assert lib.svdq_status_string(99) == b"unknown status"
+
+
+def test_sf_bytes():
+    lib = _lib.load()
+    assert lib.svdq_sf_bytes(1, 64) == 128 * 4
+    assert lib.svdq_sf_bytes(128, 512) == 128 * 32
+    assert lib.svdq_sf_bytes(129, 512) == 256 * 32
+    assert lib.svdq_sf_bytes(4096, 5120) == 4096 * 320
+    assert lib.svdq_sf_bytes(10, 48) == 0          # K not a multiple of 64
+
+
+def test_score_workspace_bytes():
+    lib = _lib.load()
+    segs, n = _lib.seg_array([(0, 29), (29, 4068), (4068, 4096)])
+    b = lib.svdq_score_workspace_bytes(segs, n, 5120)
+    assert b > 0 and b % 256 == 0
+    assert lib.svdq_score_workspace_bytes(None, 0, 5120) == 0
+
+
+FAKE = 0x10000  # an aligned non-null "device" pointer; never dereferenced on these paths
+
+
+def test_calib_rejects_bad_arguments():
+    lib = _lib.load()
+    z = ctypes.c_void_p
+    ok_ptr = z(FAKE)
+    # null X
+    assert lib.svdq_calib_lambda(None, 8, 64, 64, None, 0, None, 0, 0, ok_ptr, None, ok_ptr, None, ok_ptr,
+                                 None) == _lib.SVDQ_ERR_INVALID_ARG
+    # K not a multiple of 8
+    assert lib.svdq_calib_lambda(ok_ptr, 8, 60, 60, None, 0, None, 0, 0, ok_ptr, None, ok_ptr, None, ok_ptr,
+                                 None) == _lib.SVDQ_ERR_INVALID_ARG
+    # misaligned X
+    assert lib.svdq_calib_lambda(z(FAKE + 2), 8, 64, 64, None, 0, None, 0, 0, ok_ptr, None, ok_ptr, None,
+                                 ok_ptr, None) == _lib.SVDQ_ERR_MISALIGNED
+    # segment out of range
+    segs, n = _lib.seg_array([(0, 9)])
+    assert lib.svdq_calib_lambda(ok_ptr, 8, 64, 64, segs, n, None, 0, 0, ok_ptr, None, ok_ptr, None, ok_ptr,
+                                 None) == _lib.SVDQ_ERR_INVALID_ARG
+
+
+def test_quantize_rejects_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(FAKE)
+    # K not a multiple of 64
+    assert lib.svdq_quantize_act(p, 4, 96, 96, None, p, None, 0, p, p, None, None,
+                                 None) == _lib.SVDQ_ERR_UNSUPPORTED
+    # unsupported rank
+    assert lib.svdq_quantize_act(p, 4, 128, 128, None, p, p, 8, p, p, p, None,
+                                 None) == _lib.SVDQ_ERR_UNSUPPORTED
+    # rank without D
+    assert lib.svdq_quantize_act(p, 4, 128, 128, None, p, p, 16, p, p, None, None,
+                                 None) == _lib.SVDQ_ERR_INVALID_ARG
+    # null s_g
+    assert lib.svdq_quantize_act(p, 4, 128, 128, None, None, None, 0, p, p, None, None,
+                                 None) == _lib.SVDQ_ERR_INVALID_ARG
+    # misaligned codes
+    assert lib.svdq_quantize_act(p, 4, 128, 128, None, p, None, 0, ctypes.c_void_p(FAKE + 4), p, None, None,
+                                 None) == _lib.SVDQ_ERR_MISALIGNED
+
+
+def test_linear_rejects_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(FAKE)
+    args = dict(a=p, asf=p, sga=p, d=None, r=0, w=p, wsf=p, sgw=p, up=None, bias=None, y=p, ldy=512, dt=0,
+                m=128, n=512, k=512)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.svdq_linear(a["a"], a["asf"], a["sga"], a["d"], a["r"], a["w"], a["wsf"], a["sgw"], a["up"],
+                               a["bias"], a["y"], a["ldy"], a["dt"], a["m"], a["n"], a["k"], None)
+
+    assert call(k=320) == _lib.SVDQ_ERR_UNSUPPORTED          # K % 256
+    assert call(n=384, ldy=384) == _lib.SVDQ_ERR_UNSUPPORTED  # N % 256
+    assert call(r=16) == _lib.SVDQ_ERR_INVALID_ARG           # rank without D / up
+    assert call(r=24, d=p, up=p) == _lib.SVDQ_ERR_UNSUPPORTED
+    assert call(dt=2) == _lib.SVDQ_ERR_INVALID_ARG
+    assert call(ldy=100) == _lib.SVDQ_ERR_INVALID_ARG         # ldy < N
+    assert call(y=ctypes.c_void_p(FAKE + 8)) == _lib.SVDQ_ERR_MISALIGNED
+    assert call(sga=None) == _lib.SVDQ_ERR_INVALID_ARG
+
+
+def test_score_and_residual_reject_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(FAKE)
+    segs, n = _lib.seg_array([(0, 4)])
+    assert lib.svdq_score_lambda(p, p, 4, 64, 64, None, 0, p, p, p, p, 4096, None) == _lib.SVDQ_ERR_INVALID_ARG
+    bad, nb = _lib.seg_array([(2, 1)])
+    assert lib.svdq_score_lambda(p, p, 4, 64, 64, bad, nb, p, p, p, p, 4096, None) == _lib.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_score_lambda(p, p, 4, 64, 64, segs, n, p, p, p, None, 0, None) == _lib.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_residual(p, 16, 64, 64, None, None, None, 33, p, None) == _lib.SVDQ_ERR_UNSUPPORTED
+    assert lib.svdq_residual(p, 16, 64, 64, None, None, None, 4, p, None) == _lib.SVDQ_ERR_INVALID_ARG
+
+
+def test_device_error_requires_output_pointer():
+    lib = _lib.load()
+    assert lib.svdq_device_error(None, None) == _lib.SVDQ_ERR_INVALID_ARG
