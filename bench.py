@@ -1,0 +1,362 @@
+"""Benchmark of the SVDQuant-style NVFP4 W4A4 linear on B200.
+
+One step = one pass of the whole hot path over one batch: svdq_calib_lambda
+(absmax over the packed rows), svdq_quantize_act (smooth + NVFP4 + fused
+down-projection), svdq_linear (FP4 tcgen05 GEMM + low-rank + bias) and
+svdq_score_lambda (per-modality rel-L2 against the bf16 layer).  The workload
+is the DiT attention projection: 4096 packed rows (text 29 | video 4039 |
+audio 28), K = N = 5120, rank 32, synthetic seeded data.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl svdq|reference]
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU
+(independent batches, no collective on the data path: weak scaling); the
+reported time is the max over ranks.  ``--impl reference`` times the CPU
+oracle on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "W4A4 linear TFLOP/s and % of B200 dense-FP4 peak; quantize GB/s vs HBM peak"
+UNIT = "TFLOP/s"
+WORKLOAD = "dit_attention_projection_M4096_K5120_N5120_r32"
+CONFIG_INDEX = 1
+L2_FLUSH_BYTES = 256 << 20
+FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def workload_bytes(m, k, n, r, m_cal):
+    """Algorithmic bytes of the HBM-bound kernels (one launch each)."""
+    quant = m * k * 2 + m * k // 2 + m * k // 16 + m * r * 4
+    calib = m_cal * k * 2 + n * k * 2
+    score = 2 * m * n * 2
+    return dict(quantize=quant, calib=calib, score=score)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    def __init__(self, index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.index = index
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm (also the cpu_baseline of the GPU arm)
+# ---------------------------------------------------------------------------
+
+class OracleArm:
+    """The CPU oracle's hot path (calib, quantize, W4A4 linear, score) on a row sample."""
+
+    def __init__(self, layer):
+        from oracle import svdq_oracle as O
+
+        import synthetic as S
+
+        self.O = O
+        self.layer = layer
+        segs = layer.seg_ranges(layer.calib_sets["all"])
+        self.c = O.calib(layer.x, segs, layer.w)
+        self.conv = O.convert_weight(layer.w, self.c["lam"], layer.rank,
+                                     sketch=S.power_iteration_sketch(layer.n, layer.rank))
+
+    def run(self, rows: int):
+        """Returns (TFLOP/s, seconds, rows) of one timed pass over `rows` evenly spaced rows."""
+        O, layer = self.O, self.layer
+        idx = np.linspace(0, layer.m - 1, rows).astype(np.int64)
+        x = layer.x[idx]
+        yref = O.f64_to_bf16(O.reference_linear(x, layer.w, layer.bias))
+        t0 = time.perf_counter()
+        c2 = O.calib(x, None, layer.w)
+        y64, _ = O.layer_forward(x, c2["inv_lam"], self.c["s_g"], self.conv["down"], self.conv, layer.bias)
+        O.score(O.f64_to_bf16(y64), yref, [(0, rows)])
+        dt = time.perf_counter() - t0
+        return 2.0 * rows * layer.n * layer.k / dt / 1e12, dt, rows
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synthetic as S
+
+    layer = S.make_layer(CONFIG_INDEX)
+    arm = OracleArm(layer)
+    rows = 64
+    for _ in range(min(args.warmup, 1)):
+        arm.run(8)
+    times, vals = [], []
+    for _ in range(args.steps):
+        v, dt, rows = arm.run(rows)
+        times.append(dt)
+        vals.append(v)
+    value = statistics.median(vals)
+    cores = _oracle_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "rows_per_step": rows, "note": "CPU oracle on a row sample"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} of 4096 rows per step, full K and N"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    import bit_w4a4_quantized_svdq_b200 as P
+    import synthetic as S
+
+    layer = S.make_layer(CONFIG_INDEX)
+    m, k, n, r = layer.m, layer.k, layer.n, layer.rank
+    segs_all = layer.seg_ranges(layer.calib_sets["all"])
+    segs_mod = [(s.begin, s.end) for s in layer.segments]
+
+    def dev_bits(b):
+        return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev)
+
+    x = dev_bits(layer.x)
+    w = dev_bits(layer.w)
+    bias = dev_bits(layer.bias)
+    # offline: calibration and weight conversion, the bf16 reference output
+    calib = P.svdq_calib_lambda(x, segs_all, w)
+    lin = P.SVDQW4A4Linear.convert(w, bias, calib, r)
+    yref = torch.matmul(x.view(torch.bfloat16), w.view(torch.bfloat16).t()) + bias.view(torch.bfloat16)
+    q_out = dict(codes=torch.empty((m, k // 2), dtype=torch.uint8, device=dev),
+                 sf=torch.empty(P.sf_bytes(m, k), dtype=torch.uint8, device=dev),
+                 d=torch.empty((m, r), dtype=torch.float32, device=dev))
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(P.score_workspace_bytes(segs_mod, n), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(xx, ev=None):
+        if ev is not None:
+            ev[0].record()
+        cal = P.svdq_calib_lambda(xx, segs_all, w)
+        if ev is not None:
+            ev[1].record()
+        q = P.svdq_quantize_act(xx, cal["inv_lam"], lin.s_g_act, lin.down, out=q_out)
+        if ev is not None:
+            ev[2].record()
+        P.svdq_linear(q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf, lin.s_g_w, lin.up,
+                      lin.bias, out=y)
+        if ev is not None:
+            ev[3].record()
+        res = P.svdq_score_lambda(y, yref, segs_mod, workspace=ws)
+        if ev is not None:
+            ev[4].record()
+        return res
+
+    launches_per_step = 3 + 1 + 1 + 2   # calib (2 absmax + lambda), quantize, linear, score (2)
+    for _ in range(args.warmup):
+        step(x)
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: inputs resident in HBM, L2 flushed between steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        step(x, evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
+    step_ms = float(per.sum(axis=1).mean())
+    kern_ms = per.mean(axis=0)       # calib, quantize, linear, score
+    t_local = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    step_ms_max = float(t_local.item())
+
+    flops = 2.0 * m * n * k
+    value = flops * world / (step_ms_max * 1e-3) / 1e12
+    peaks = read_peaks()
+    fp4_peak = peaks["bf16"] * FP4_PER_BF16
+    lin_tflops = flops / (kern_ms[2] * 1e-3) / 1e12
+    by = workload_bytes(m, k, n, r, m)
+    quant_gbs = by["quantize"] / (kern_ms[1] * 1e-3) / 1e9
+    calib_gbs = by["calib"] / (kern_ms[0] * 1e-3) / 1e9
+    score_gbs = by["score"] / (kern_ms[3] * 1e-3) / 1e9
+
+    # ---- end to end through the public layer API with host buffers
+    x_host = torch.from_numpy(np.ascontiguousarray(layer.x).view(np.int16)).pin_memory()
+    x_dev = torch.empty_like(x)
+    rel_host = torch.empty(len(segs_mod), dtype=torch.float64).pin_memory()
+    for _ in range(max(1, args.warmup)):
+        x_dev.copy_(x_host, non_blocking=True)
+        rel_host.copy_(step(x_dev)[2], non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        rel_host.copy_(step(x_dev)[2], non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = flops * world / (float(e2e_ms.item()) * 1e-3) / 1e12
+    rel = rel_host.tolist()
+
+    err = P.svdq_device_error()
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, dt, rows = OracleArm(layer).run(256)
+            cpu = {"value": v, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+                   "sample": f"{rows} of {m} rows, full K={k} and N={n}, {dt:.1f} s"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) -> fp32 accum, bf16 out", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": m, "K": k, "N": n, "rank": r, "rows_per_gpu": m,
+                       "segments": {s.name: [s.begin, s.end] for s in layer.segments},
+                       "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write)"},
+            "kernels_ms": {"calib": kern_ms[0], "quantize": kern_ms[1], "linear": kern_ms[2],
+                           "score": kern_ms[3]},
+            "linear_tflops": lin_tflops, "quantize_gbs": quant_gbs, "calib_gbs": calib_gbs, "score_gbs": score_gbs,
+            "roofline": {"bound": "tensor", "kernel": "svdq_linear", "achieved": lin_tflops, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": lin_tflops / fp4_peak, "traffic": None,
+                         "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} x {FP4_PER_BF16:g} "
+                                        "(nominal dense FP4/BF16 ratio)"},
+            "roofline_hbm": {"kernel": "svdq_quantize_act", "achieved": quant_gbs, "peak": peaks["hbm"],
+                             "unit": "GB/s", "frac": quant_gbs / peaks["hbm"]},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": m * k * 2,
+                    "d2h_bytes_per_step": 8 * len(segs_mod)},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "rel_l2_vs_bf16": dict(zip([s.name for s in layer.segments], rel)),
+            "device_error": err,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "svdq":
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -20,27 +20,48 @@ namespace {
 constexpr int kColsPerThread = 8;             // one 16-byte load
 constexpr int kThreadsX = 32;                 // 256 channels per block
 constexpr int kThreadsY = 8;
-constexpr int kRowsPerBlock = 64;
+constexpr int kRowsPerThread = 16;            // independent loads in flight per thread
+constexpr int kRowsPerBlock = kThreadsY * kRowsPerThread;
 
+struct AbsmaxJob {
+    const uint16_t* base;
+    int64_t ld;
+    SegTable segs;
+    int64_t total_rows;
+    uint32_t* out_bits;
+};
+
+// blockIdx.z selects the job (0: activations over the selected rows, 1: the weight).
 __global__ void __launch_bounds__(kThreadsX * kThreadsY)
-col_absmax_kernel(const uint16_t* __restrict__ X, int64_t K, int64_t ldx, SegTable segs,
-                  int64_t total_rows, uint32_t* __restrict__ out_bits) {
+col_absmax_kernel(AbsmaxJob job0, AbsmaxJob job1, int64_t K) {
     __shared__ uint32_t red[kThreadsY][kThreadsX][kColsPerThread / 2];
+    const AbsmaxJob& job = blockIdx.z == 0 ? job0 : job1;
+    const int64_t v0 = static_cast<int64_t>(blockIdx.y) * kRowsPerBlock;
+    if (v0 >= job.total_rows) return;                       // uniform per block
+    const int64_t v1 = min(v0 + kRowsPerBlock, job.total_rows);
     const int64_t col0 = (static_cast<int64_t>(blockIdx.x) * kThreadsX + threadIdx.x) * kColsPerThread;
     const bool col_ok = col0 < K;
     uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
-    const int64_t v0 = static_cast<int64_t>(blockIdx.y) * kRowsPerBlock;
-    const int64_t v1 = min(v0 + kRowsPerBlock, total_rows);
     if (col_ok) {
+        uint4 q[kRowsPerThread];
         int s = 0;
-        for (int64_t v = v0 + threadIdx.y; v < v1; v += kThreadsY) {
-            while (s + 1 < segs.n && v >= segs.prefix[s + 1]) ++s;   // v increases monotonically
-            const int64_t row = segs.begin[s] + (v - segs.prefix[s]);
-            const uint4 q = *reinterpret_cast<const uint4*>(X + row * ldx + col0);
-            m0 = __vmaxu2(m0, q.x & 0x7FFF7FFFu);
-            m1 = __vmaxu2(m1, q.y & 0x7FFF7FFFu);
-            m2 = __vmaxu2(m2, q.z & 0x7FFF7FFFu);
-            m3 = __vmaxu2(m3, q.w & 0x7FFF7FFFu);
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+            const int64_t v = v0 + threadIdx.y + static_cast<int64_t>(i) * kThreadsY;
+            if (v < v1) {
+                while (s + 1 < job.segs.n && v >= job.segs.prefix[s + 1]) ++s;   // v increases with i
+                const int64_t row = job.segs.begin[s] + (v - job.segs.prefix[s]);
+                q[i] = __ldg(reinterpret_cast<const uint4*>(job.base + row * job.ld + col0));
+            } else {
+                q[i] = make_uint4(0, 0, 0, 0);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+            m0 = __vmaxu2(m0, q[i].x & 0x7FFF7FFFu);
+            m1 = __vmaxu2(m1, q[i].y & 0x7FFF7FFFu);
+            m2 = __vmaxu2(m2, q[i].z & 0x7FFF7FFFu);
+            m3 = __vmaxu2(m3, q[i].w & 0x7FFF7FFFu);
         }
     }
     red[threadIdx.y][threadIdx.x][0] = m0;
@@ -61,8 +82,8 @@ col_absmax_kernel(const uint16_t* __restrict__ X, int64_t K, int64_t ldx, SegTab
             // bf16 -> fp32 bit pattern is a 16-bit left shift.
             const uint32_t lo = (w[i] & 0xFFFFu) << 16;
             const uint32_t hi = w[i] & 0xFFFF0000u;
-            if (lo) atomicMax(out_bits + col0 + 2 * i, lo);
-            if (hi) atomicMax(out_bits + col0 + 2 * i + 1, hi);
+            if (lo) atomicMax(job.out_bits + col0 + 2 * i, lo);
+            if (hi) atomicMax(job.out_bits + col0 + 2 * i + 1, hi);
         }
     }
 }
@@ -94,18 +115,26 @@ lambda_kernel(const float* __restrict__ ax, const float* __restrict__ aw, int64_
     }
 }
 
-int launch_col_absmax(const void* X, int64_t K, int64_t ldx, const SegTable& segs, float* out,
-                      cudaStream_t st) {
-    const int64_t total = segs.prefix[segs.n];
-    if (cudaMemsetAsync(out, 0, sizeof(float) * K, st) != cudaSuccess) return SVDQ_ERR_CUDA;
-    if (total == 0) return SVDQ_OK;
+// Column absmax of X over `segs` (and of W over all of its rows, if given) in one launch.
+int launch_col_absmax(const void* X, int64_t K, int64_t ldx, const SegTable& segs, float* out_x,
+                      const void* W, int64_t N, int64_t ldw, float* out_w, cudaStream_t st) {
+    AbsmaxJob jx{static_cast<const uint16_t*>(X), ldx, segs, segs.prefix[segs.n], reinterpret_cast<uint32_t*>(out_x)};
+    AbsmaxJob jw = jx;
+    if (W != nullptr) {
+        SegTable all;
+        make_seg_table(nullptr, 0, N, &all);
+        jw = AbsmaxJob{static_cast<const uint16_t*>(W), ldw, all, N, reinterpret_cast<uint32_t*>(out_w)};
+    }
+    if (cudaMemsetAsync(out_x, 0, sizeof(float) * K, st) != cudaSuccess) return SVDQ_ERR_CUDA;
+    if (W != nullptr && cudaMemsetAsync(out_w, 0, sizeof(float) * K, st) != cudaSuccess) return SVDQ_ERR_CUDA;
+    const int64_t rows = max(jx.total_rows, W != nullptr ? jw.total_rows : int64_t(0));
+    if (rows == 0) return SVDQ_OK;
     const int64_t gx = (K + kThreadsX * kColsPerThread - 1) / (kThreadsX * kColsPerThread);
-    const int64_t gy = (total + kRowsPerBlock - 1) / kRowsPerBlock;
-    // 65535 blocks of 64 rows in y: about 4.2 million calibration rows per call.
+    const int64_t gy = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
+    // 65535 blocks of 128 rows in y: about 8.4 million rows per call.
     if (gy > 65535) return SVDQ_ERR_UNSUPPORTED;
-    dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
-    col_absmax_kernel<<<grid, dim3(kThreadsX, kThreadsY), 0, st>>>(
-        static_cast<const uint16_t*>(X), K, ldx, segs, total, reinterpret_cast<uint32_t*>(out));
+    dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy), W != nullptr ? 2u : 1u);
+    col_absmax_kernel<<<grid, dim3(kThreadsX, kThreadsY), 0, st>>>(jx, jw, K);
     return launch_status(cudaGetLastError());
 }
 
@@ -128,14 +157,8 @@ extern "C" int svdq_calib_lambda(const void* X, int64_t M, int64_t K, int64_t ld
     if (st != SVDQ_OK) return st;
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    st = launch_col_absmax(X, K, ldx, table, amax_x, cs);
+    st = launch_col_absmax(X, K, ldx, table, amax_x, W, N, ldw, amax_w, cs);
     if (st != SVDQ_OK) return st;
-    if (W != nullptr) {
-        SegTable all;
-        make_seg_table(nullptr, 0, N, &all);
-        st = launch_col_absmax(W, K, ldw, all, amax_w, cs);
-        if (st != SVDQ_OK) return st;
-    }
     lambda_kernel<<<1, 1024, 0, cs>>>(amax_x, W != nullptr ? amax_w : nullptr, K, lambda, inv_lambda, s_g);
     return launch_status(cudaGetLastError());
 }

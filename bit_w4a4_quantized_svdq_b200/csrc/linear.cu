@@ -21,8 +21,8 @@
 //         4 kind::mxf4nvf4 block16 MMAs (K = 64 each) into one fp32 accumulator
 //   2     low-rank operand builder: D' hi/lo and the duplicated up tile written
 //         into the swizzled operand layout in shared memory
-//   3..6  epilogue: tensor memory -> registers, alpha and bias, bf16 (or fp32)
-//         rows to global memory; the accumulator is released as soon as it has
+//   3..10 epilogue (two warps per tensor-memory lane quarter): tensor memory ->
+//         registers, alpha and bias, bf16 (or fp32) rows to global memory; the accumulator is released as soon as it has
 //         been read, so the stores overlap the next tile's main loop.
 #include "common.cuh"
 #include "sm100.cuh"
@@ -35,9 +35,9 @@ constexpr int kBN = 256;
 constexpr int kBKBytes = 128;                 // packed FP4 bytes per row per stage (256 channels)
 constexpr int kBK = 256;                      // channels per stage
 constexpr int kStages = 3;
-constexpr int kThreads = 224;
+constexpr int kThreads = 352;                 // 11 warps
 constexpr int kEpiWarp0 = 3;
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;
 
 constexpr uint32_t kATile = kBM * kBKBytes;          // 16 KB
 constexpr uint32_t kBTile = kBN * kBKBytes;          // 32 KB
@@ -51,7 +51,8 @@ constexpr uint32_t kOffStages = 0;
 constexpr uint32_t kOffLrA = kStages * kStageBytes;  // multiple of 1024
 constexpr uint32_t kOffLrB = kOffLrA + kLrA;
 constexpr uint32_t kOffBar = kOffLrB + kLrB;
-constexpr uint32_t kSmemBytes = kOffBar + 256;
+constexpr uint32_t kOffBias = kOffBar + 256;          // 2 x 256 bf16 bias staging
+constexpr uint32_t kSmemBytes = kOffBias + 2 * kBN * 2;
 
 // Tensor-memory columns: accumulator [0, 256), block scales after it.
 constexpr uint32_t kTmemCols = 512;
@@ -277,46 +278,49 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int quarter = warp & 3;                       // tensor-memory lane quarter of this warp
-        const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        // Two warps per tensor-memory lane quarter, each owning 128 of the 256
+        // columns.  The tile's bias is staged in shared memory before the
+        // accumulator wait, so nothing but tensor-memory reads sits between
+        // "accumulator full" and "accumulator free".
+        const int ew = warp - kEpiWarp0;                    // 0..7
+        const int quarter = warp & 3;                       // lane quarter this warp may access
+        const int half = ew >> 2;                           // column half of the tile
+        const int etid = ew * 32 + lane;                    // 0..255
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * (kBN / 2);
+        uint16_t* bias_s = reinterpret_cast<uint16_t*>(smem + kOffBias);
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             const int m_blk = tile % args.m_tiles;
             const int n_blk = tile / args.m_tiles;
+            const int64_t col0 = static_cast<int64_t>(n_blk) * kBN;
+            uint16_t* bt = bias_s + (local & 1) * kBN;
+            bt[etid] = args.bias ? args.bias[col0 + etid] : static_cast<uint16_t>(0);
+            asm volatile("bar.sync 1, %0;" :: "n"(kEpiWarps * 32) : "memory");
             if (!mbar_wait(acc_full, local & 1, abort_flag, args.err, kErrWaitMma)) break;
             tc_fence_after();
             const int64_t row = static_cast<int64_t>(m_blk) * kBM + quarter * 32 + lane;
-            const int64_t col0 = static_cast<int64_t>(n_blk) * kBN;
+            const int64_t ccol = col0 + half * (kBN / 2);   // first output column of this warp
+            const uint16_t* bw = bt + half * (kBN / 2);
             const bool row_ok = row < args.M;
             if constexpr (!kOutF32) {
-                uint32_t packed[kBN / 2];
+                uint32_t packed[kBN / 4];
 #pragma unroll
-                for (int c = 0; c < kBN / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tbase + c * 32, v);
+                for (int c = 0; c < kBN / 2 / 64; ++c) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld_32x32b_x32(tbase + c * 64, v0);
+                    tmem_ld_32x32b_x32(tbase + c * 64 + 32, v1);
                     tmem_ld_wait();
-                    float b[32];
-                    if (args.bias) {
-                        const uint4* bp = reinterpret_cast<const uint4*>(args.bias + col0 + c * 32);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint4 w = __ldg(bp + q);
-                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                b[8 * q + 2 * e] = bf16_lo(ws[e]);
-                                b[8 * q + 2 * e + 1] = bf16_hi(ws[e]);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) b[j] = 0.0f;
+                    for (int j = 0; j < 16; ++j) {
+                        const uint32_t bb = *reinterpret_cast<const uint32_t*>(bw + c * 64 + 2 * j);
+                        packed[c * 32 + j] = pack_bf16x2(fmaf(alpha, __uint_as_float(v0[2 * j]), bf16_lo(bb)),
+                                                         fmaf(alpha, __uint_as_float(v0[2 * j + 1]), bf16_hi(bb)));
                     }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const float y0 = fmaf(alpha, __uint_as_float(v[2 * j]), b[2 * j]);
-                        const float y1 = fmaf(alpha, __uint_as_float(v[2 * j + 1]), b[2 * j + 1]);
-                        packed[c * 16 + j] = pack_bf16x2(y0, y1);
+                        const uint32_t bb = *reinterpret_cast<const uint32_t*>(bw + c * 64 + 32 + 2 * j);
+                        packed[c * 32 + 16 + j] = pack_bf16x2(fmaf(alpha, __uint_as_float(v1[2 * j]), bf16_lo(bb)),
+                                                              fmaf(alpha, __uint_as_float(v1[2 * j + 1]), bf16_hi(bb)));
                     }
                 }
                 // The accumulator has been read: let the next tile's MMAs start.
@@ -324,27 +328,26 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 __syncwarp();
                 if (lane == 0) mbar_arrive(acc_empty);
                 if (row_ok) {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(args.Y) + row * args.ldy + col0);
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(args.Y) + row * args.ldy + ccol);
 #pragma unroll
-                    for (int q = 0; q < kBN / 8; ++q)
+                    for (int q = 0; q < kBN / 16; ++q)
                         dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < kBN / 32; ++c) {
+                for (int c = 0; c < kBN / 2 / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, v);
                     tmem_ld_wait();
                     if (row_ok) {
-                        float* dst = static_cast<float*>(args.Y) + row * args.ldy + col0 + c * 32;
+                        float* dst = static_cast<float*>(args.Y) + row * args.ldy + ccol + c * 32;
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             float y[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int j = 4 * q + e;
-                                const float bj = args.bias
-                                    ? __uint_as_float(static_cast<uint32_t>(args.bias[col0 + c * 32 + j]) << 16) : 0.0f;
+                                const float bj = __uint_as_float(static_cast<uint32_t>(bw[c * 32 + j]) << 16);
                                 y[e] = fmaf(alpha, __uint_as_float(v[j]), bj);
                             }
                             reinterpret_cast<float4*>(dst)[q] = make_float4(y[0], y[1], y[2], y[3]);

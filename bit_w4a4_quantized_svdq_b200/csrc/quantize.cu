@@ -9,15 +9,17 @@
 // "DeltaQuant on MiniMax-H3", section "The activation scale bound held": the
 // tensor scale is static and saturated groups are counted at run time.
 //
-// Layout of one CTA (6 warps) over a 128-row tile and a slice of K:
-//   warp 4      TMA producer: 128 x 64 bf16 tiles of X (128-byte swizzle) and
-//               the matching r x 64 tile of the down weight into a 4-stage ring
-//   warp 5      tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
-//   warps 0..3  quantisers: read the swizzled tile from shared memory, 2 lanes
+// Layout of one CTA (10 warps, one CTA per SM) over a 128-row tile and a
+// slice of K:
+//   warp 8      TMA producer: 128 x 64 bf16 tiles of X (128-byte swizzle) and
+//               the matching r x 64 tile of the down weight into an 8-stage ring
+//   warp 9      tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
+//   warps 0..7  quantisers: read the swizzled tile from shared memory, 2 lanes
 //               per 16-element group (amax by one shuffle), E4M3 scale and E2M1
 //               codes through the hardware RNE conversions, coalesced stores;
-//               finally read D_partial from tensor memory.
-// K is split across the CTAs of a thread-block cluster (up to 8); the partial
+//               warps 0..3 (one per tensor-memory lane quarter) finally read
+//               D_partial from tensor memory.
+// K is split across the CTAs of a thread-block cluster (up to 4); the partial
 // D tiles are summed in a fixed order through distributed shared memory, so D
 // is deterministic.  Memory traffic per element: 2 bytes in, 0.5625 out.
 #include "common.cuh"
@@ -28,12 +30,12 @@ namespace {
 
 constexpr int kBM = 128;               // rows per CTA tile
 constexpr int kBK = 64;                // channels per stage (128 bytes of bf16)
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
-constexpr int kQuantWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kMaxSplit = 8;
+constexpr int kStages = 8;
+constexpr int kThreads = 320;
+constexpr int kQuantWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kMaxSplit = 4;          // CTAs of a cluster along K
 constexpr uint32_t kXTileBytes = kBM * kBK * 2;  // 16 KB
 
 template <int R>
@@ -181,8 +183,8 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             }
             const uint8_t* tile = smem + L::kXOff + s * kXTileBytes;
 #pragma unroll 2
-            for (int it = 0; it < 8; ++it) {
-                const int row = warp * 32 + it * 4 + rsub;                // row inside the tile
+            for (int it = 0; it < kBM / (4 * kQuantWarps); ++it) {
+                const int row = warp * (kBM / kQuantWarps) + it * 4 + rsub;   // row inside the tile
                 const uint4 v = *reinterpret_cast<const uint4*>(tile + row * 128 + ((c8 ^ (row & 7)) << 4));
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
                 float xs[8];
@@ -229,7 +231,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         for (int o = 16; o > 0; o >>= 1) sat += __shfl_xor_sync(0xffffffffu, sat, o);
         if (lane == 0 && sat && args.sat_count) atomicAdd(args.sat_count, sat);
 
-        if (R > 0) {
+        if (R > 0 && warp < 4) {   // one warp per tensor-memory lane quarter
             float* part = reinterpret_cast<float*>(smem + L::kPartOff);   // [R][128]
             const int row = warp * 32 + lane;
             if (mbar_wait(dfull, 0, abort_flag, args.err, kErrWaitMma)) {
@@ -260,7 +262,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     if constexpr (R > 0) {
         // Sum the split-K partials in cluster-rank order (deterministic) on rank 0.
         cluster_sync_all();
-        if (cluster_ctarank() == 0 && warp < kQuantWarps) {
+        if (cluster_ctarank() == 0 && warp < 4) {
             const int row = warp * 32 + lane;
             const int64_t grow = static_cast<int64_t>(m_blk) * kBM + row;
             const uint32_t base = smem_u32(smem + L::kPartOff);
@@ -302,9 +304,9 @@ int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const Quan
     QuantArgs a = base;
     a.n_chunks = static_cast<int>(K / kBK);
     const int64_t m_tiles = (M + kBM - 1) / kBM;
-    // Split K so the grid covers the GPU about twice over, up to a cluster of 8.
+    // Split K so the grid covers every SM about once (one CTA fits per SM), up to a cluster of 4.
     const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
-    int split = static_cast<int>((2 * sms + m_tiles - 1) / m_tiles);
+    int split = static_cast<int>((sms + m_tiles - 1) / m_tiles);
     split = split < 1 ? 1 : (split > kMaxSplit ? kMaxSplit : split);
     if (split > a.n_chunks) split = a.n_chunks;
     a.split = split;

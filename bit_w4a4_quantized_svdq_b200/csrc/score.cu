@@ -6,7 +6,8 @@
 //
 // Bandwidth-bound two-pass reduction with a fixed order, so results are
 // bitwise reproducible: pass 1 gives every (segment, row chunk) one block that
-// writes fp64 partial sums to the caller's workspace; pass 2 sums each
+// writes fp64 partial sums to the caller's workspace (16 independent 16-byte
+// loads per thread and input in flight); pass 2 sums each
 // segment's partials in index order and forms num, den and rel.
 #include "common.cuh"
 #include "sm100.cuh"
@@ -15,30 +16,25 @@ namespace svdq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int64_t kElemsPerChunk = 1 << 17;        // elements a partial-sum block covers
+constexpr int kVecPerThread = 16;                   // 16-byte vectors of each input per thread
+constexpr int64_t kElemsPerChunk = int64_t(kThreads) * kVecPerThread * 8;   // 32768 elements per block
 
+// Segment s covers the flat element range [0, rows_s * N) of its rows; block
+// `chunk` sums elements [c * kElemsPerChunk, (c + 1) * kElemsPerChunk) of one segment.
 struct ChunkPlan {
     int n;                                           // segments
     int64_t begin[kMaxSegments];                     // first row of segment s
-    int64_t end[kMaxSegments];
-    int64_t rows_per_chunk;                          // rows one block sums
+    int64_t elems[kMaxSegments];                     // rows_s * N
     int64_t chunk_prefix[kMaxSegments + 1];          // first chunk index of segment s
 };
 
-inline int64_t rows_per_chunk_for(int64_t N) {
-    const int64_t r = kElemsPerChunk / (N > 0 ? N : 1);
-    return r < 1 ? 1 : r;
-}
-
 inline void make_plan(const svdq_seg* segs, int n_seg, int64_t N, ChunkPlan* p) {
     p->n = n_seg;
-    p->rows_per_chunk = rows_per_chunk_for(N);
     p->chunk_prefix[0] = 0;
     for (int s = 0; s < n_seg; ++s) {
         p->begin[s] = segs[s].begin;
-        p->end[s] = segs[s].end;
-        const int64_t rows = segs[s].end - segs[s].begin;
-        const int64_t chunks = rows > 0 ? (rows + p->rows_per_chunk - 1) / p->rows_per_chunk : 1;
+        p->elems[s] = (segs[s].end - segs[s].begin) * N;
+        const int64_t chunks = p->elems[s] > 0 ? (p->elems[s] + kElemsPerChunk - 1) / kElemsPerChunk : 1;
         p->chunk_prefix[s + 1] = p->chunk_prefix[s] + chunks;
     }
 }
@@ -55,6 +51,21 @@ __device__ __forceinline__ double block_sum(double v, double* sh) {
     return v;   // valid in thread 0
 }
 
+__device__ __forceinline__ void accum8(const uint4& qa, const uint4& qb, double& num, double& den) {
+    const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
+    const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const double r_lo = bf16_lo(wb[i]), r_hi = bf16_hi(wb[i]);
+        const double d_lo = static_cast<double>(bf16_lo(wa[i])) - r_lo;
+        const double d_hi = static_cast<double>(bf16_hi(wa[i])) - r_hi;
+        num = fma(d_lo, d_lo, num);
+        num = fma(d_hi, d_hi, num);
+        den = fma(r_lo, r_lo, den);
+        den = fma(r_hi, r_hi, den);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads)
 score_partial_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict__ yr, int64_t N, int64_t ld,
                      ChunkPlan plan, double* __restrict__ partial) {
@@ -62,37 +73,35 @@ score_partial_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict
     const int64_t chunk = blockIdx.x;
     int s = 0;
     while (s + 1 < plan.n && chunk >= plan.chunk_prefix[s + 1]) ++s;
-    const int64_t r0 = plan.begin[s] + (chunk - plan.chunk_prefix[s]) * plan.rows_per_chunk;
-    const int64_t r1 = min(r0 + plan.rows_per_chunk, plan.end[s]);
+    const int64_t e0 = (chunk - plan.chunk_prefix[s]) * kElemsPerChunk;
+    const int64_t e1 = min(e0 + kElemsPerChunk, plan.elems[s]);
+    const uint16_t* qa = yq + plan.begin[s] * ld;
+    const uint16_t* qb = yr + plan.begin[s] * ld;
     double num = 0.0, den = 0.0;
-    const bool vec = (N % 8 == 0);
-    for (int64_t row = r0; row < r1; ++row) {
-        const uint16_t* a = yq + row * ld;
-        const uint16_t* b = yr + row * ld;
-        if (vec) {
-            for (int64_t c = static_cast<int64_t>(threadIdx.x) * 8; c < N; c += kThreads * 8) {
-                const uint4 qa = *reinterpret_cast<const uint4*>(a + c);
-                const uint4 qb = *reinterpret_cast<const uint4*>(b + c);
-                const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
-                const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+    if (N % 8 == 0) {
+        // 16-byte vectors; a vector never straddles a row because N % 8 == 0.
+        uint4 va[kVecPerThread], vb[kVecPerThread];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const double r_lo = bf16_lo(wb[i]), r_hi = bf16_hi(wb[i]);
-                    const double d_lo = static_cast<double>(bf16_lo(wa[i])) - r_lo;
-                    const double d_hi = static_cast<double>(bf16_hi(wa[i])) - r_hi;
-                    num = fma(d_lo, d_lo, num);
-                    num = fma(d_hi, d_hi, num);
-                    den = fma(r_lo, r_lo, den);
-                    den = fma(r_hi, r_hi, den);
-                }
+        for (int i = 0; i < kVecPerThread; ++i) {
+            const int64_t e = e0 + (static_cast<int64_t>(i) * kThreads + threadIdx.x) * 8;
+            if (e < e1) {
+                const int64_t off = (ld == N) ? e : (e / N) * ld + (e % N);   // contiguous rows: no division
+                va[i] = __ldg(reinterpret_cast<const uint4*>(qa + off));
+                vb[i] = __ldg(reinterpret_cast<const uint4*>(qb + off));
+            } else {
+                va[i] = make_uint4(0, 0, 0, 0);
+                vb[i] = make_uint4(0, 0, 0, 0);
             }
-        } else {
-            for (int64_t c = threadIdx.x; c < N; c += kThreads) {
-                const double r = __uint_as_float(static_cast<uint32_t>(b[c]) << 16);
-                const double d = static_cast<double>(__uint_as_float(static_cast<uint32_t>(a[c]) << 16)) - r;
-                num = fma(d, d, num);
-                den = fma(r, r, den);
-            }
+        }
+#pragma unroll
+        for (int i = 0; i < kVecPerThread; ++i) accum8(va[i], vb[i], num, den);
+    } else {
+        for (int64_t e = e0 + threadIdx.x; e < e1; e += kThreads) {
+            const int64_t off = (ld == N) ? e : (e / N) * ld + (e % N);
+            const double r = __uint_as_float(static_cast<uint32_t>(qb[off]) << 16);
+            const double d = static_cast<double>(__uint_as_float(static_cast<uint32_t>(qa[off]) << 16)) - r;
+            num = fma(d, d, num);
+            den = fma(r, r, den);
         }
     }
     num = block_sum(num, sh);
@@ -157,12 +166,11 @@ int score_lambda_check(const void* Yq, const void* Yref, int64_t M, int64_t N, i
 }
 
 size_t score_partial_bytes(const svdq_seg* segs, int n_seg, int64_t N) {
-    if (segs == nullptr || n_seg < 1 || n_seg > kMaxSegments) return 0;
-    const int64_t rpc = rows_per_chunk_for(N);
+    if (segs == nullptr || n_seg < 1 || n_seg > kMaxSegments || N < 1) return 0;
     int64_t chunks = 0;
     for (int s = 0; s < n_seg; ++s) {
-        const int64_t rows = segs[s].end - segs[s].begin;
-        chunks += rows > 0 ? (rows + rpc - 1) / rpc : 1;
+        const int64_t elems = (segs[s].end - segs[s].begin) * N;
+        chunks += elems > 0 ? (elems + kElemsPerChunk - 1) / kElemsPerChunk : 1;
     }
     return static_cast<size_t>(chunks) * 2 * sizeof(double);
 }

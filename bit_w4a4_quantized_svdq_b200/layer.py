@@ -34,6 +34,8 @@ def lowrank_factors_device(w: torch.Tensor, lam: torch.Tensor, rank: int, oversa
         n, k = w.shape
         return (torch.zeros((0, k), dtype=torch.bfloat16, device=w.device),
                 torch.zeros((n, 0), dtype=torch.bfloat16, device=w.device))
+    if w.dtype in (torch.int16, torch.uint16):
+        w = w.view(torch.bfloat16)                               # raw bf16 bit patterns
     lam64 = lam.to(torch.float64)
     a = (w.to(torch.float64) * lam64[None, :]).t()              # [K, N]
     gen = torch.Generator(device=w.device)

@@ -283,3 +283,37 @@ def test_config1_residual_and_linear_sampled(lib, cfg1):
 
 def test_no_device_wait_timed_out(lib):
     assert lib.svdq_device_error() == 0
+
+
+# ---------------------------------------------------------------------------
+# The product's own offline conversion (device factorisation + library kernels)
+# ---------------------------------------------------------------------------
+
+def test_product_conversion_quality(lib, cfg0):
+    """The layer built by SVDQW4A4Linear.convert is as good as the oracle's pipeline.
+
+    Its low-rank factors come from a randomized range finder on the device, so
+    they are not bit-identical to the oracle's exact SVD; what must hold is
+    that the rank-r residual is near-optimal and the layer's error against the
+    unquantised fp64 output is no worse than the oracle pipeline's.
+    """
+    L, segs, c, conv = cfg0
+    x, w, b = dev_bits(L.x), dev_bits(L.w), dev_bits(L.bias)
+    cal = lib.SVDQW4A4Linear.calibrate(x, w, segs)
+    assert np.array_equal(cal["lam"].cpu().numpy(), c["lam"])
+    layer = lib.SVDQW4A4Linear.convert(w, b, cal, L.rank)
+    y = layer(x, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
+    y_ref = O.reference_linear(L.x, L.w, L.bias)
+    y_orc, _ = O.layer_forward(L.x, c["inv_lam"], c["s_g"], conv["down"], conv, L.bias)
+    rel_gpu, rel_orc = rel_l2(y, y_ref), rel_l2(y_orc, y_ref)
+    assert rel_gpu <= 1.10 * rel_orc, (rel_gpu, rel_orc)
+    # near-optimal rank-r split: ||W lambda - (lambda down^T up^T)^T||_F vs the SVD tail
+    lam = c["lam"].astype(np.float64)
+    w_hat = O.bf16_to_f64(L.w) * lam[None, :]
+    down = O.bf16_to_f64(host_bits(layer.down))
+    up = O.bf16_to_f64(host_bits(layer.up))
+    resid = np.linalg.norm(w_hat - up @ (down * lam[None, :]))
+    sv = np.linalg.svd(w_hat, compute_uv=False)
+    tail = np.sqrt(np.sum(sv[L.rank:] ** 2))
+    assert resid <= 1.02 * tail, (resid, tail)
+    assert lib.svdq_device_error() == 0
