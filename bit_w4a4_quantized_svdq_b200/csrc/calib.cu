@@ -20,8 +20,9 @@ namespace {
 constexpr int kColsPerThread = 8;             // one 16-byte load
 constexpr int kThreadsX = 32;                 // 256 channels per block
 constexpr int kThreadsY = 8;
-constexpr int kRowsPerThread = 16;            // independent loads in flight per thread
-constexpr int kRowsPerBlock = kThreadsY * kRowsPerThread;
+constexpr int kRowsPerThread = 16;            // independent loads in flight per thread (one round)
+constexpr int kRounds = 4;                    // rounds per block: 512 rows, so few atomics per column
+constexpr int kRowsPerBlock = kThreadsY * kRowsPerThread * kRounds;
 
 struct AbsmaxJob {
     const uint16_t* base;
@@ -43,11 +44,12 @@ col_absmax_kernel(AbsmaxJob job0, AbsmaxJob job1, int64_t K) {
     const bool col_ok = col0 < K;
     uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
     if (col_ok) {
+      int s = 0;
+      for (int round = 0; round < kRounds; ++round) {
         uint4 q[kRowsPerThread];
-        int s = 0;
 #pragma unroll
         for (int i = 0; i < kRowsPerThread; ++i) {
-            const int64_t v = v0 + threadIdx.y + static_cast<int64_t>(i) * kThreadsY;
+            const int64_t v = v0 + threadIdx.y + static_cast<int64_t>(round * kRowsPerThread + i) * kThreadsY;
             if (v < v1) {
                 while (s + 1 < job.segs.n && v >= job.segs.prefix[s + 1]) ++s;   // v increases with i
                 const int64_t row = job.segs.begin[s] + (v - job.segs.prefix[s]);
@@ -63,6 +65,7 @@ col_absmax_kernel(AbsmaxJob job0, AbsmaxJob job1, int64_t K) {
             m2 = __vmaxu2(m2, q[i].z & 0x7FFF7FFFu);
             m3 = __vmaxu2(m3, q[i].w & 0x7FFF7FFFu);
         }
+      }
     }
     red[threadIdx.y][threadIdx.x][0] = m0;
     red[threadIdx.y][threadIdx.x][1] = m1;
@@ -131,7 +134,7 @@ int launch_col_absmax(const void* X, int64_t K, int64_t ldx, const SegTable& seg
     if (rows == 0) return SVDQ_OK;
     const int64_t gx = (K + kThreadsX * kColsPerThread - 1) / (kThreadsX * kColsPerThread);
     const int64_t gy = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
-    // 65535 blocks of 128 rows in y: about 8.4 million rows per call.
+    // 65535 blocks of 512 rows in y: about 33 million rows per call.
     if (gy > 65535) return SVDQ_ERR_UNSUPPORTED;
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy), W != nullptr ? 2u : 1u);
     col_absmax_kernel<<<grid, dim3(kThreadsX, kThreadsY), 0, st>>>(jx, jw, K);

@@ -17,11 +17,14 @@
 //         256 x 128 B (128-byte swizzle) plus 2 + 4 KB of scale atoms (bulk copies)
 //   1     tcgen05 issuer and tensor-memory owner: per tile 4 kind::f16 MMAs for
 //         the low-rank term (K = 64: 32 ranks of D'_hi then 32 of D'_lo against
-//         up twice), then per stage: scale atoms -> tensor memory (tcgen05.cp),
-//         4 kind::mxf4nvf4 block16 MMAs (K = 64 each) into one fp32 accumulator
+//         up twice), then per stage 4 kind::mxf4nvf4 block16 MMAs (K = 64 each)
+//         into one fp32 accumulator
 //   2     low-rank operand builder: D' hi/lo and the duplicated up tile written
 //         into the swizzled operand layout in shared memory
-//   3..10 epilogue (two warps per tensor-memory lane quarter): tensor memory ->
+//   3..6  block-scale writers: each stage's scale atoms, shared memory ->
+//         registers -> tensor memory (tcgen05.st, one warp per lane quarter),
+//         into a per-stage buffer; this keeps the tensor pipe free for MMAs
+//   7..14 epilogue (two warps per tensor-memory lane quarter): tensor memory ->
 //         registers, alpha and bias, bf16 (or fp32) rows to global memory; the accumulator is released as soon as it has
 //         been read, so the stores overlap the next tile's main loop.
 #include "common.cuh"
@@ -35,8 +38,10 @@ constexpr int kBN = 256;
 constexpr int kBKBytes = 128;                 // packed FP4 bytes per row per stage (256 channels)
 constexpr int kBK = 256;                      // channels per stage
 constexpr int kStages = 3;
-constexpr int kThreads = 352;                 // 11 warps
-constexpr int kEpiWarp0 = 3;
+constexpr int kThreads = 480;                 // 15 warps
+constexpr int kSfWarp0 = 3;                   // warps 3..6 write block scales into tensor memory
+constexpr int kSfWarps = 4;
+constexpr int kEpiWarp0 = 7;                  // warps 7..14: epilogue
 constexpr int kEpiWarps = 8;
 
 constexpr uint32_t kATile = kBM * kBKBytes;          // 16 KB
@@ -54,10 +59,12 @@ constexpr uint32_t kOffBar = kOffLrB + kLrB;
 constexpr uint32_t kOffBias = kOffBar + 256;          // 2 x 256 bf16 bias staging
 constexpr uint32_t kSmemBytes = kOffBias + 2 * kBN * 2;
 
-// Tensor-memory columns: accumulator [0, 256), block scales after it.
+// Tensor-memory columns: accumulator [0, 256), then one block-scale buffer per
+// pipeline stage (48 columns each: A scales 4 per MMA, B scales 8 per MMA).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemSfa = 256;                   // 4 columns per MMA, 4 MMAs per stage
-constexpr uint32_t kTmemSfb = 272;                   // 8 columns per MMA
+constexpr uint32_t kTmemSf0 = 256;
+constexpr uint32_t kTmemSfStride = 48;
+constexpr uint32_t kTmemSfbOff = 16;
 
 struct LinearArgs {
     const uint8_t* a_sf;
@@ -93,7 +100,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* lr_full = acc_empty + 1;
     uint64_t* lr_empty = lr_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lr_empty + 1);
+    uint64_t* sf_full = lr_empty + 1;                       // kStages
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + kStages);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5;
@@ -108,6 +116,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sf_full[s], kSfWarps);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kEpiWarps);
@@ -186,22 +195,16 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
                     if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) { ok = false; break; }
+                    if (!mbar_wait(&sf_full[s], ph, abort_flag, args.err, kErrWaitFull)) { ok = false; break; }
                     tc_fence_after();
                     uint8_t* st = smem + kOffStages + s * kStageBytes;
-                    const uint32_t sfa = smem_u32(st + kATile + kBTile);
-                    const uint32_t sfb = sfa + kSfaTile;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        tc_cp_32x128b_x4(tmem + kTmemSfa + 4 * j, desc_sf_block(sfa + 512 * j));
-                        tc_cp_32x128b_x4(tmem + kTmemSfb + 8 * j, desc_sf_block(sfb + 512 * j));
-                        tc_cp_32x128b_x4(tmem + kTmemSfb + 8 * j + 4, desc_sf_block(sfb + kSfbTile / 2 + 512 * j));
-                    }
+                    const uint32_t sf = tmem + kTmemSf0 + s * kTmemSfStride;
                     const uint32_t a0 = smem_u32(st);
                     const uint32_t b0 = smem_u32(st + kATile);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         mma_nvf4(tmem, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc_f4,
-                                 tmem + kTmemSfa + 4 * kk, tmem + kTmemSfb + 8 * kk, (first && kk == 0) ? 0u : 1u);
+                                 sf + 4 * kk, sf + kTmemSfbOff + 8 * kk, (first && kk == 0) ? 0u : 1u);
                     }
                     first = false;
                     tc_commit(&empty[s]);
@@ -276,6 +279,47 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 if (lane == 0) mbar_arrive(lr_full);
             }
         }
+    } else if (warp < kEpiWarp0) {
+        // ------------------------------------------------------------ block-scale writers
+        // Each warp copies the stage's scale atoms from shared memory into its
+        // own tensor-memory lane quarter with tcgen05.st (every quarter holds
+        // the full set, the layout the block-scaled MMA reads).  Unlike a
+        // shared->tensor copy issued by the MMA thread, these stores run
+        // alongside the MMAs instead of in front of them.  Buffer s is free
+        // again once stage s has been refilled: the refill waited for the MMAs
+        // that read it.
+        const uint32_t tq = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const int local_tiles = (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                                static_cast<int>(gridDim.x);
+        const int total = local_tiles * k_stages;
+        for (int it = 0; it < total; ++it) {
+            const int s = it % kStages;
+            const uint32_t ph = (it / kStages) & 1;
+            if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
+            tc_fence_after();
+            const uint8_t* sfa = smem + kOffStages + s * kStageBytes + kATile + kBTile;
+            const uint8_t* sfb = sfa + kSfaTile;
+            // Column layout of one buffer: A scales of MMA kk at 4 kk + (row / 32);
+            // B scales of MMA kk at 16 + 8 kk + (row / 32), rows 128..255 at + 4.
+            // Lane i reads row i of each 512-byte atom: its 4 words are the 4 columns.
+            uint32_t ra[16], rb[32];
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+                const uint4 a = *reinterpret_cast<const uint4*>(sfa + kb * 512 + lane * 16);
+                const uint4 x = *reinterpret_cast<const uint4*>(sfb + kb * 512 + lane * 16);
+                const uint4 y = *reinterpret_cast<const uint4*>(sfb + kSfbTile / 2 + kb * 512 + lane * 16);
+                ra[4 * kb] = a.x; ra[4 * kb + 1] = a.y; ra[4 * kb + 2] = a.z; ra[4 * kb + 3] = a.w;
+                rb[8 * kb] = x.x; rb[8 * kb + 1] = x.y; rb[8 * kb + 2] = x.z; rb[8 * kb + 3] = x.w;
+                rb[8 * kb + 4] = y.x; rb[8 * kb + 5] = y.y; rb[8 * kb + 6] = y.z; rb[8 * kb + 7] = y.w;
+            }
+            const uint32_t base = tq + kTmemSf0 + s * kTmemSfStride;
+            tmem_st_32x32b_x16(base, ra);
+            tmem_st_32x32b_x32(base + kTmemSfbOff, rb);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sf_full[s]);
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         // Two warps per tensor-memory lane quarter, each owning 128 of the 256
@@ -305,22 +349,15 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             if constexpr (!kOutF32) {
                 uint32_t packed[kBN / 4];
 #pragma unroll
-                for (int c = 0; c < kBN / 2 / 64; ++c) {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld_32x32b_x32(tbase + c * 64, v0);
-                    tmem_ld_32x32b_x32(tbase + c * 64 + 32, v1);
+                for (int c = 0; c < kBN / 2 / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase + c * 32, v);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const uint32_t bb = *reinterpret_cast<const uint32_t*>(bw + c * 64 + 2 * j);
-                        packed[c * 32 + j] = pack_bf16x2(fmaf(alpha, __uint_as_float(v0[2 * j]), bf16_lo(bb)),
-                                                         fmaf(alpha, __uint_as_float(v0[2 * j + 1]), bf16_hi(bb)));
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const uint32_t bb = *reinterpret_cast<const uint32_t*>(bw + c * 64 + 32 + 2 * j);
-                        packed[c * 32 + 16 + j] = pack_bf16x2(fmaf(alpha, __uint_as_float(v1[2 * j]), bf16_lo(bb)),
-                                                              fmaf(alpha, __uint_as_float(v1[2 * j + 1]), bf16_hi(bb)));
+                        const uint32_t bb = *reinterpret_cast<const uint32_t*>(bw + c * 32 + 2 * j);
+                        packed[c * 16 + j] = pack_bf16x2(fmaf(alpha, __uint_as_float(v[2 * j]), bf16_lo(bb)),
+                                                         fmaf(alpha, __uint_as_float(v[2 * j + 1]), bf16_hi(bb)));
                     }
                 }
                 // The accumulator has been read: let the next tile's MMAs start.

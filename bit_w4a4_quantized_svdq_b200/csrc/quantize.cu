@@ -9,14 +9,16 @@
 // "DeltaQuant on MiniMax-H3", section "The activation scale bound held": the
 // tensor scale is static and saturated groups are counted at run time.
 //
-// Layout of one CTA (10 warps, one CTA per SM) over a 128-row tile and a
+// Layout of one CTA (18 warps, one CTA per SM) over a 128-row tile and a
 // slice of K:
-//   warp 8      TMA producer: 128 x 64 bf16 tiles of X (128-byte swizzle) and
-//               the matching r x 64 tile of the down weight into an 8-stage ring
-//   warp 9      tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
-//   warps 0..7  quantisers: read the swizzled tile from shared memory, 2 lanes
-//               per 16-element group (amax by one shuffle), E4M3 scale and E2M1
-//               codes through the hardware RNE conversions, coalesced stores;
+//   warp 16     TMA producer: 128 x 64 bf16 tiles of X (128-byte swizzle), the
+//               matching r x 64 tile of the down weight and 64 values of
+//               1/lambda into an 8-stage ring
+//   warp 17     tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
+//   warps 0..15 quantisers: one lane per 16-element group (8 rows x 4 groups
+//               per warp and stage) read from the swizzled tile, E4M3 scale and
+//               E2M1 codes through the hardware RNE conversions, 8-byte code
+//               stores and one 4-byte scale word per row;
 //               warps 0..3 (one per tensor-memory lane quarter) finally read
 //               D_partial from tensor memory.
 // K is split across the CTAs of a thread-block cluster (up to 4); the partial
@@ -31,10 +33,10 @@ namespace {
 constexpr int kBM = 128;               // rows per CTA tile
 constexpr int kBK = 64;                // channels per stage (128 bytes of bf16)
 constexpr int kStages = 8;
-constexpr int kThreads = 320;
-constexpr int kQuantWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kThreads = 576;
+constexpr int kQuantWarps = 16;       // 8 rows x 4 groups of 16 channels per warp and stage
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
 constexpr int kMaxSplit = 4;          // CTAs of a cluster along K
 constexpr uint32_t kXTileBytes = kBM * kBK * 2;  // 16 KB
 
@@ -44,7 +46,8 @@ struct QSmem {
     static constexpr uint32_t kXOff = 0;
     static constexpr uint32_t kDownOff = kStages * kXTileBytes;
     static constexpr uint32_t kPartOff = kDownOff + kStages * kDownTileBytes;     // D partial [R][128] fp32
-    static constexpr uint32_t kBarOff = kPartOff + R * kBM * 4;
+    static constexpr uint32_t kIlamOff = kPartOff + R * kBM * 4;                   // 1/lambda, 64 fp32 per stage
+    static constexpr uint32_t kBarOff = kIlamOff + kStages * kBK * 4;
     static constexpr uint32_t kBytes = kBarOff + 256;
 };
 
@@ -127,8 +130,10 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
                 if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) break;
-                mbar_arrive_expect_tx(&full[s], kXTileBytes + L::kDownTileBytes);
                 const int col = (c_begin + i) * kBK;
+                mbar_arrive_expect_tx(&full[s], kXTileBytes + L::kDownTileBytes + (args.inv_lambda ? kBK * 4 : 0));
+                if (args.inv_lambda)
+                    bulk_load(smem + L::kIlamOff + s * kBK * 4, args.inv_lambda + col, kBK * 4, &full[s]);
                 tma_load_2d(smem + L::kXOff + s * kXTileBytes, &tmap_x, &full[s], col, m_blk * kBM);
                 if (R > 0)
                     tma_load_2d(smem + L::kDownOff + s * L::kDownTileBytes, &tmap_down, &full[s], col, 0);
@@ -166,66 +171,69 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         const int64_t half_k = K >> 1;
         const int64_t atoms_k = K >> 6;
         uint32_t sat = 0;
-        const int c8 = lane & 7;           // 16-byte chunk of the 128-byte row this lane reads
-        const int rsub = lane >> 3;        // which of 4 rows this iteration
+        // Lane -> (row of the warp's 8, group of 16 channels); the group's two
+        // 16-byte halves are chunks 2b and 2b+1 of the row's 128-byte line.
+        const int rw = lane >> 2;
+        const int b = lane & 3;
+        const int row = warp * (kBM / kQuantWarps) + rw;                  // row inside the tile
+        const int64_t grow = static_cast<int64_t>(m_blk) * kBM + row;
+        const int ph0 = ((2 * b) ^ (row & 7)) << 4;
+        const int ph1 = ((2 * b + 1) ^ (row & 7)) << 4;
         for (int i = 0; i < n_local; ++i) {
             const int s = i % kStages;
             const uint32_t ph = (i / kStages) & 1;
             if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
             const int chunk = c_begin + i;
-            const int64_t k0 = static_cast<int64_t>(chunk) * kBK + c8 * 8;
-            float il[8];
+            const uint8_t* tile = smem + L::kXOff + s * kXTileBytes + row * 128;
+            const uint4 v0 = *reinterpret_cast<const uint4*>(tile + ph0);
+            const uint4 v1 = *reinterpret_cast<const uint4*>(tile + ph1);
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            float xs[16];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                xs[2 * j] = bf16_lo(w[j]);
+                xs[2 * j + 1] = bf16_hi(w[j]);
+            }
             if (args.inv_lambda) {
-                const float4 a = __ldg(reinterpret_cast<const float4*>(args.inv_lambda + k0));
-                const float4 b = __ldg(reinterpret_cast<const float4*>(args.inv_lambda + k0 + 4));
-                il[0] = a.x; il[1] = a.y; il[2] = a.z; il[3] = a.w;
-                il[4] = b.x; il[5] = b.y; il[6] = b.z; il[7] = b.w;
-            }
-            const uint8_t* tile = smem + L::kXOff + s * kXTileBytes;
-#pragma unroll 2
-            for (int it = 0; it < kBM / (4 * kQuantWarps); ++it) {
-                const int row = warp * (kBM / kQuantWarps) + it * 4 + rsub;   // row inside the tile
-                const uint4 v = *reinterpret_cast<const uint4*>(tile + row * 128 + ((c8 ^ (row & 7)) << 4));
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                float xs[8];
+                const float4* il = reinterpret_cast<const float4*>(smem + L::kIlamOff + s * kBK * 4 + b * 64);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    xs[2 * j] = bf16_lo(w[j]);
-                    xs[2 * j + 1] = bf16_hi(w[j]);
-                }
-                if (args.inv_lambda) {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) xs[j] = __fmul_rn(xs[j], il[j]);
-                }
-                float a = 0.0f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(xs[j]));
-                a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));            // the other half of the group
-                const float t = __fdiv_rn(a, d);
-                const uint32_t sfb = cvt_e4m3(t);
-                const float S = __fmul_rn(e4m3_to_f32(sfb), s_g);
-                const float rS = (S == 0.0f) ? 0.0f : __frcp_rn(S);
-                float q[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) q[j] = __fmul_rn(xs[j], rS);
-                const uint32_t packed = cvt_e2m1x8(q);
-                if ((c8 & 1) == 0 && t > 448.0f) ++sat;
-                // 4 scale bytes of this row and chunk -> one 32-bit word (lane c8 == 0 of the row)
-                uint32_t sfw = sfb;
-                sfw |= __shfl_down_sync(0xffffffffu, sfb, 2) << 8;
-                sfw |= __shfl_down_sync(0xffffffffu, sfb, 4) << 16;
-                sfw |= __shfl_down_sync(0xffffffffu, sfb, 6) << 24;
-                const int64_t grow = static_cast<int64_t>(m_blk) * kBM + row;
-                if (grow < M)
-                    *reinterpret_cast<uint32_t*>(args.codes + grow * half_k + chunk * (kBK / 2) + c8 * 4) = packed;
-                if (c8 == 0) {
-                    const int64_t off = (static_cast<int64_t>(m_blk) * atoms_k + chunk) * 512 + (row & 31) * 16 +
-                                        ((row >> 5) & 3) * 4;
-                    *reinterpret_cast<uint32_t*>(args.sf + off) = sfw;
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 l = il[q4];
+                    xs[4 * q4] = __fmul_rn(xs[4 * q4], l.x);
+                    xs[4 * q4 + 1] = __fmul_rn(xs[4 * q4 + 1], l.y);
+                    xs[4 * q4 + 2] = __fmul_rn(xs[4 * q4 + 2], l.z);
+                    xs[4 * q4 + 3] = __fmul_rn(xs[4 * q4 + 3], l.w);
                 }
             }
+            float a = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(xs[j]));
+            const float t = __fdiv_rn(a, d);
+            const uint32_t sfb = cvt_e4m3(t);
+            const float S = __fmul_rn(e4m3_to_f32(sfb), s_g);
+            const float rS = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+            float q0[8], q1[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                q0[j] = __fmul_rn(xs[j], rS);
+                q1[j] = __fmul_rn(xs[8 + j], rS);
+            }
+            const uint2 packed = make_uint2(cvt_e2m1x8(q0), cvt_e2m1x8(q1));
+            if (t > 448.0f) ++sat;
+            // the row's 4 scale bytes (groups b = 0..3 in lanes 4 rw .. 4 rw + 3) -> one 32-bit word
+            uint32_t sfw = sfb;
+            sfw |= __shfl_down_sync(0xffffffffu, sfb, 1) << 8;
+            sfw |= __shfl_down_sync(0xffffffffu, sfb, 2) << 16;
+            sfw |= __shfl_down_sync(0xffffffffu, sfb, 3) << 24;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            if (lane == 0) mbar_arrive(&empty[s]);        // shared memory of this stage no longer read
+            if (grow < M)
+                *reinterpret_cast<uint2*>(args.codes + grow * half_k + chunk * (kBK / 2) + b * 8) = packed;
+            if (b == 0) {
+                const int64_t off = (static_cast<int64_t>(m_blk) * atoms_k + chunk) * 512 + (row & 31) * 16 +
+                                    ((row >> 5) & 3) * 4;
+                *reinterpret_cast<uint32_t*>(args.sf + off) = sfw;
+            }
         }
         // saturation count: one atomic per warp
         for (int o = 16; o > 0; o >>= 1) sat += __shfl_xor_sync(0xffffffffu, sat, o);

@@ -6,7 +6,7 @@
 //
 // Bandwidth-bound two-pass reduction with a fixed order, so results are
 // bitwise reproducible: pass 1 gives every (segment, row chunk) one block that
-// writes fp64 partial sums to the caller's workspace (16 independent 16-byte
+// writes fp64 partial sums to the caller's workspace (8 independent 16-byte
 // loads per thread and input in flight); pass 2 sums each
 // segment's partials in index order and forms num, den and rel.
 #include "common.cuh"
@@ -16,8 +16,8 @@ namespace svdq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kVecPerThread = 16;                   // 16-byte vectors of each input per thread
-constexpr int64_t kElemsPerChunk = int64_t(kThreads) * kVecPerThread * 8;   // 32768 elements per block
+constexpr int kVecPerThread = 8;                    // 16-byte vectors of each input per thread
+constexpr int64_t kElemsPerChunk = int64_t(kThreads) * kVecPerThread * 8;   // 16384 elements per block
 
 // Segment s covers the flat element range [0, rows_s * N) of its rows; block
 // `chunk` sums elements [c * kElemsPerChunk, (c + 1) * kElemsPerChunk) of one segment.
@@ -51,19 +51,25 @@ __device__ __forceinline__ double block_sum(double v, double* sh) {
     return v;   // valid in thread 0
 }
 
+// Eight element pairs: differences and squares in fp32 (the difference of two
+// bf16 values and its square carry at most a 2^-24 relative rounding each), the
+// 8-term partial sums are added to the fp64 accumulators.
 __device__ __forceinline__ void accum8(const uint4& qa, const uint4& qb, double& num, double& den) {
     const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
     const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+    float n8 = 0.0f, d8 = 0.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const double r_lo = bf16_lo(wb[i]), r_hi = bf16_hi(wb[i]);
-        const double d_lo = static_cast<double>(bf16_lo(wa[i])) - r_lo;
-        const double d_hi = static_cast<double>(bf16_hi(wa[i])) - r_hi;
-        num = fma(d_lo, d_lo, num);
-        num = fma(d_hi, d_hi, num);
-        den = fma(r_lo, r_lo, den);
-        den = fma(r_hi, r_hi, den);
+        const float r_lo = bf16_lo(wb[i]), r_hi = bf16_hi(wb[i]);
+        const float e_lo = __fsub_rn(bf16_lo(wa[i]), r_lo);
+        const float e_hi = __fsub_rn(bf16_hi(wa[i]), r_hi);
+        n8 = __fmaf_rn(e_lo, e_lo, n8);
+        n8 = __fmaf_rn(e_hi, e_hi, n8);
+        d8 = __fmaf_rn(r_lo, r_lo, d8);
+        d8 = __fmaf_rn(r_hi, r_hi, d8);
     }
+    num += static_cast<double>(n8);
+    den += static_cast<double>(d8);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -98,10 +104,10 @@ score_partial_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict
     } else {
         for (int64_t e = e0 + threadIdx.x; e < e1; e += kThreads) {
             const int64_t off = (ld == N) ? e : (e / N) * ld + (e % N);
-            const double r = __uint_as_float(static_cast<uint32_t>(qb[off]) << 16);
-            const double d = static_cast<double>(__uint_as_float(static_cast<uint32_t>(qa[off]) << 16)) - r;
-            num = fma(d, d, num);
-            den = fma(r, r, den);
+            const float r = __uint_as_float(static_cast<uint32_t>(qb[off]) << 16);
+            const float d = __fsub_rn(__uint_as_float(static_cast<uint32_t>(qa[off]) << 16), r);
+            num += static_cast<double>(__fmul_rn(d, d));
+            den += static_cast<double>(__fmul_rn(r, r));
         }
     }
     num = block_sum(num, sh);

@@ -213,8 +213,10 @@ def test_score_matches_oracle(lib, m, n):
     segs = [(0, m // 3), (m // 3, m // 3), (m // 3, m), (0, m)]
     num, den, rel = O.score(yq, yref, segs)
     g = lib.svdq_score_lambda(dev_bits(yq), dev_bits(yref), segs)
+    # fp32 differences/squares summed in groups of 8, fp64 beyond: relative error
+    # of each sum well under 1e-6 (2^-24 per operation, 8-term fp32 partials)
     for a, b in zip(g, (num, den, rel)):
-        np.testing.assert_allclose(a.cpu().numpy(), b, rtol=1e-12, atol=0)
+        np.testing.assert_allclose(a.cpu().numpy(), b, rtol=1e-6, atol=0)
     g2 = lib.svdq_score_lambda(dev_bits(yq), dev_bits(yref), segs)
     for a, b in zip(g, g2):
         assert torch.equal(a, b)      # fixed reduction order: bitwise reproducible
