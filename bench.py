@@ -223,6 +223,7 @@ def run_gpu(args):
     y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(P.score_workspace_bytes(segs_mod, n), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_read = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(xx, ev=None):
@@ -257,7 +258,11 @@ def run_gpu(args):
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
+        # L2 flush between steps, outside the events: write a buffer larger than
+        # L2, then read another one so the write-back of the dirty lines happens
+        # here and every step starts from a cold, clean L2.
         flush.fill_(i & 0xFF)
+        flush_read.sum()
         step(x, evs[i])
     torch.cuda.synchronize()
     if world > 1:
@@ -318,7 +323,8 @@ def run_gpu(args):
             "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) -> fp32 accum, bf16 out", "data": "synthetic",
             "config": {"workload": WORKLOAD, "M": m, "K": k, "N": n, "rank": r, "rows_per_gpu": m,
                        "segments": {s.name: [s.begin, s.end] for s in layer.segments},
-                       "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write)"},
+                       "parallelism": f"replicas x{world}",
+                       "l2": "flushed between steps: 256 MiB write, then 256 MiB read (cold, clean L2)"},
             "kernels_ms": {"calib": kern_ms[0], "quantize": kern_ms[1], "linear": kern_ms[2],
                            "score": kern_ms[3]},
             "linear_tflops": lin_tflops, "quantize_gbs": quant_gbs, "calib_gbs": calib_gbs, "score_gbs": score_gbs,

@@ -25,8 +25,12 @@
 //         registers -> tensor memory (tcgen05.st, one warp per lane quarter),
 //         into a per-stage buffer; this keeps the tensor pipe free for MMAs
 //   7..14 epilogue (two warps per tensor-memory lane quarter): tensor memory ->
-//         registers, alpha and bias, bf16 (or fp32) rows to global memory; the accumulator is released as soon as it has
-//         been read, so the stores overlap the next tile's main loop.
+//         registers, alpha and bias, bf16 rows staged in shared memory and
+//         written by TMA bulk stores (fp32 rows: plain stores); the accumulator
+//         is released as soon as it has been read, so the stores overlap the
+//         next tile's main loop.
+// The low-rank MMAs close each tile, so their operand area doubles as the
+// epilogue's output staging: builder -> MMA -> epilogue -> builder.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -91,7 +95,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <bool kOutF32>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-              LinearArgs args) {
+              const __grid_constant__ CUtensorMap tmap_y, LinearArgs args) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -99,8 +103,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     uint64_t* acc_full = empty + kStages;
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* lr_full = acc_empty + 1;
-    uint64_t* lr_empty = lr_full + 1;
-    uint64_t* sf_full = lr_empty + 1;                       // kStages
+    uint64_t* stage_free = lr_full + 1;                     // epilogue done with the staging area
+    uint64_t* sf_full = stage_free + 1;                     // kStages
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + kStages);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -121,7 +125,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kEpiWarps);
         mbar_init(lr_full, 1);
-        mbar_init(lr_empty, 1);
+        mbar_init(stage_free, kEpiWarps);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -179,18 +183,6 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 if (!mbar_wait(acc_empty, (local & 1) ^ 1, abort_flag, args.err, kErrWaitAccum)) break;
                 tc_fence_after();
                 bool first = true;
-                if (has_lr) {
-                    if (!mbar_wait(lr_full, local & 1, abort_flag, args.err, kErrWaitLowRank)) break;
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(smem + kOffLrA);
-                    const uint32_t b0 = smem_u32(smem + kOffLrB);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc_lr,
-                                 kk > 0 ? 1u : 0u);
-                    tc_commit(lr_empty);
-                    first = false;
-                }
                 for (int kb = 0; kb < k_stages; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
@@ -209,6 +201,19 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     first = false;
                     tc_commit(&empty[s]);
                 }
+                if (!ok) break;
+                if (has_lr) {
+                    // Low-rank term last: its operands share shared memory with the
+                    // epilogue's output staging, which is free again once this
+                    // tile's accumulator has been drained.
+                    if (!mbar_wait(lr_full, local & 1, abort_flag, args.err, kErrWaitLowRank)) break;
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + kOffLrA);
+                    const uint32_t b0 = smem_u32(smem + kOffLrB);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc_lr, 1u);
+                }
                 tc_commit(acc_full);
             }
         }
@@ -220,7 +225,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
                 const int m_blk = tile % args.m_tiles;
                 const int n_blk = tile / args.m_tiles;
-                if (!mbar_wait(lr_empty, (local & 1) ^ 1, abort_flag, args.err, kErrWaitLowRank)) break;
+                if (!mbar_wait(stage_free, (local & 1) ^ 1, abort_flag, args.err, kErrWaitLowRank)) break;
                 uint8_t* la = smem + kOffLrA;
                 uint8_t* lb = smem + kOffLrB;
                 // A: row = D'[m] as bf16 hi (channels 0..31) and lo (32..63)
@@ -364,12 +369,35 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(acc_empty);
-                if (row_ok) {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(args.Y) + row * args.ldy + ccol);
+                // Output through shared memory and the TMA: the low-rank operand
+                // area is free (this tile's low-rank MMAs completed before the
+                // accumulator was signalled full).  Each warp stages its 32 rows x
+                // 64 columns (128-byte swizzle) twice.  Bulk stores keep the
+                // scattered per-row writes off the load/store path the tensor
+                // core reads its operands through.
+                uint8_t* stg = smem + kOffLrA + ew * 4096;
+                const int32_t grow0 = static_cast<int32_t>(m_blk * kBM + quarter * 32);
 #pragma unroll
-                    for (int q = 0; q < kBN / 16; ++q)
-                        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                for (int h = 0; h < 2; ++h) {
+                    if (h == 1) {
+                        if (lane == 0) bulk_wait_read_all();
+                        __syncwarp();
+                    }
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                            make_uint4(packed[h * 32 + 4 * c], packed[h * 32 + 4 * c + 1],
+                                       packed[h * 32 + 4 * c + 2], packed[h * 32 + 4 * c + 3]);
+                    fence_async_shared();
+                    __syncwarp();
+                    if (lane == 0 && grow0 < args.M) {          // boxes wholly below row M are skipped
+                        tma_store_2d(&tmap_y, stg, static_cast<int32_t>(ccol) + h * 64, grow0);
+                        bulk_commit_group();
+                    }
                 }
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(stage_free);
             } else {
 #pragma unroll 1
                 for (int c = 0; c < kBN / 2 / 32; ++c) {
@@ -393,8 +421,15 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
+                if (lane == 0) {
+                    mbar_arrive(acc_empty);
+                    mbar_arrive(stage_free);
+                }
             }
+        }
+        if constexpr (!kOutF32) {
+            if (lane == 0) bulk_wait_all();          // bulk stores complete before the CTA exits
+            __syncwarp();
         }
     }
 
@@ -408,7 +443,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
 }
 
 template <bool kOutF32>
-int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const LinearArgs& a, cudaStream_t st) {
+int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, const LinearArgs& a,
+                  cudaStream_t st) {
     const uint32_t smem = kSmemBytes + 1024;
     auto kern = linear_kernel<kOutF32>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -416,7 +452,7 @@ int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const LinearArgs
     const int tiles = a.m_tiles * a.n_tiles;
     const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
     const int grid = tiles < sms ? tiles : sms;
-    kern<<<grid, kThreads, smem, st>>>(ta, tb, a);
+    kern<<<grid, kThreads, smem, st>>>(ta, tb, ty, a);
     return launch_status(cudaGetLastError());
 }
 
@@ -459,6 +495,10 @@ extern "C" int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const fl
         !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_codes, K / 2, N, K / 2, 128, 256,
                         CU_TENSOR_MAP_SWIZZLE_128B))
         return SVDQ_ERR_CUDA;
+    CUtensorMap ty = ta;
+    if (out_dtype == 0 &&
+        !encode_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, N, M, ldy * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+        return SVDQ_ERR_CUDA;
     LinearArgs a{};
     a.a_sf = a_sf;
     a.w_sf = w_sf;
@@ -477,5 +517,5 @@ extern "C" int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const fl
     a.n_tiles = static_cast<int>(n_tiles);
     a.err = err;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return out_dtype ? launch_linear<true>(ta, tb, a, st) : launch_linear<false>(ta, tb, a, st);
+    return out_dtype ? launch_linear<true>(ta, tb, ty, a, st) : launch_linear<false>(ta, tb, ty, a, st);
 }
