@@ -7,7 +7,7 @@
 #include <cstddef>
 #include <cstdint>
 
-#include "../../include/svdq.h"
+#include "svdq.h"   // include/ is on the include path (see build.py)
 
 namespace svdq {
 
