@@ -1,17 +1,23 @@
 """B200 (sm_100a) SVDQuant-style NVFP4 W4A4 linear layer.
 
 The computation runs in ``libsvdq.so`` (C ABI in ``include/svdq.h``); this
-package is its Python binding.  Importing it loads the library and fails if it
-has not been built (``python -m bit_w4a4_quantized_svdq_b200.build``).
+package is its Python binding.  The library is loaded on first use, and any
+call fails with ImportError if it has not been built
+(``python -m bit_w4a4_quantized_svdq_b200.build``): there is no fallback.
 """
 from . import _lib
 from .ops import (score_workspace_bytes, sf_bytes, svdq_calib_lambda, svdq_device_error, svdq_linear,
                   svdq_quantize_act, svdq_residual, svdq_score_lambda)
 from .layer import SVDQW4A4Linear, lowrank_factors_device
 
-lib = _lib.load()
+
+def load():
+    """Load libsvdq.so (raises ImportError if it is missing) and return the ctypes handle."""
+    return _lib.load()
+
 
 __all__ = [
     "svdq_calib_lambda", "svdq_quantize_act", "svdq_linear", "svdq_score_lambda", "svdq_residual",
-    "svdq_device_error", "sf_bytes", "score_workspace_bytes", "SVDQW4A4Linear", "lowrank_factors_device", "lib",
+    "svdq_device_error", "sf_bytes", "score_workspace_bytes", "SVDQW4A4Linear",
+    "lowrank_factors_device", "load",
 ]
