@@ -17,6 +17,7 @@ SVDQ_ERR_MISALIGNED = 3
 SVDQ_ERR_CUDA = 4
 SVDQ_ERR_TIMEOUT = 5
 SVDQ_ERR_NO_DEVICE = 6
+SVDQ_ERR_SCRATCH_TOO_SMALL = 7
 
 
 class SvdqSeg(Structure):
@@ -45,6 +46,9 @@ SIGNATURES = {
     "svdq_score_workspace_bytes": (c_size_t, [POINTER(SvdqSeg), c_int, c_int64]),
     "svdq_score_lambda": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int64, POINTER(SvdqSeg), c_int,
                                   c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "svdq_score_static_max_bytes": (c_size_t, []),
+    "svdq_score_lambda_static": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int64, POINTER(SvdqSeg), c_int,
+                                         c_void_p, c_void_p, c_void_p, c_void_p]),
     "svdq_residual": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_int,
                               c_void_p, c_void_p]),
     "svdq_device_error": (c_int, [c_void_p, POINTER(c_uint32)]),

@@ -102,6 +102,7 @@ const char* svdq_status_string(int status) {
         case SVDQ_ERR_CUDA: return "CUDA error";
         case SVDQ_ERR_TIMEOUT: return "device wait timed out";
         case SVDQ_ERR_NO_DEVICE: return "no sm_100 device";
+        case SVDQ_ERR_SCRATCH_TOO_SMALL: return "problem exceeds the library's static scratch array";
         default: return "unknown status";
     }
 }

@@ -9,6 +9,8 @@
 // writes fp64 partial sums to the caller's workspace (8 independent 16-byte
 // loads per thread and input in flight); pass 2 sums each
 // segment's partials in index order and forms num, den and rel.
+#include <mutex>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -200,5 +202,64 @@ extern "C" int svdq_score_lambda(const void* Yq, const void* Yref, int64_t M, in
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
     return score_lambda_launch(Yq, Yref, M, N, ld, segs, n_seg, num, den, rel,
                                static_cast<double*>(workspace), workspace_bytes,
+                               static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// Scoring without a caller workspace.
+//
+// Some callers cannot allocate device memory while they score: code running
+// inside a framework's memory pool that forbids side allocations, a
+// pre-recorded launch sequence whose buffers were fixed in advance, or a
+// plugin host that hands out only input and output tensors.  For them the
+// per-block partial sums live in a fixed array inside this library instead of
+// a workspace argument.  The array is a __device__ variable, so every GPU that
+// loads the library holds it (kStaticScoreBytes) until the process exits.
+// ---------------------------------------------------------------------------
+namespace svdq {
+namespace {
+
+constexpr size_t kStaticScoreBytes = size_t(1) << 20;   // 65536 partial-sum pairs
+
+static __device__ __align__(256) double g_score_scratch[kStaticScoreBytes / sizeof(double)];
+
+constexpr int kMaxDevicesStatic = 64;
+double* g_score_scratch_ptr[kMaxDevicesStatic] = {};
+std::mutex g_score_scratch_mutex;
+
+// Host code may not hand the array's name to a kernel: on the host it is only a
+// stand-in for the device variable.  Its device address is looked up once per
+// device, with that device current.
+double* static_scratch_for_current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesStatic) return nullptr;
+    std::lock_guard<std::mutex> lock(g_score_scratch_mutex);
+    if (g_score_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_score_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        g_score_scratch_ptr[dev] = static_cast<double*>(p);
+    }
+    return g_score_scratch_ptr[dev];
+}
+
+}  // namespace
+}  // namespace svdq
+
+extern "C" size_t svdq_score_static_max_bytes(void) { return svdq::kStaticScoreBytes; }
+
+extern "C" int svdq_score_lambda_static(const void* Yq, const void* Yref, int64_t M, int64_t N, int64_t ld,
+                                        const svdq_seg* segs, int n_seg,
+                                        double* num, double* den, double* rel, void* stream) {
+    using namespace svdq;
+    int st = score_lambda_check(Yq, Yref, M, N, ld, segs, n_seg, num, den, rel);
+    if (st != SVDQ_OK) return st;
+    const size_t need = score_partial_bytes(segs, n_seg, N);
+    if (need > kStaticScoreBytes) return SVDQ_ERR_SCRATCH_TOO_SMALL;
+    if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    double* scratch = static_scratch_for_current_device();
+    if (scratch == nullptr) return SVDQ_ERR_CUDA;
+    // Every partial-sum slot a call reads is written by the same call first, so
+    // the previous call's contents need no clearing.
+    return score_lambda_launch(Yq, Yref, M, N, ld, segs, n_seg, num, den, rel, scratch, kStaticScoreBytes,
                                static_cast<cudaStream_t>(stream));
 }

@@ -136,6 +136,25 @@ def svdq_score_lambda(yq: torch.Tensor, yref: torch.Tensor, segs: Sequence[Tuple
     return num, den, rel
 
 
+def svdq_score_lambda_static(yq: torch.Tensor, yref: torch.Tensor, segs: Sequence[Tuple[int, int]], stream=None):
+    """svdq_score_lambda without a workspace: partial sums in the library's static array."""
+    lib = _lib.load()
+    _check_bf16(yq, "yq")
+    _check_bf16(yref, "yref")
+    m, n = yq.shape
+    ld = _row_stride(yq, "yq")
+    if _row_stride(yref, "yref") != ld:
+        raise ValueError("yq and yref must share a row stride")
+    arr, n_seg = _lib.seg_array(segs)
+    dev = yq.device
+    num = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    den = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    rel = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    _lib.check("svdq_score_lambda_static", lib.svdq_score_lambda_static(
+        _ptr(yq), _ptr(yref), m, n, ld, arr, n_seg, _ptr(num), _ptr(den), _ptr(rel), _stream(stream)))
+    return num, den, rel
+
+
 def svdq_residual(w: torch.Tensor, lam: Optional[torch.Tensor], down: Optional[torch.Tensor],
                   up: Optional[torch.Tensor], stream=None) -> torch.Tensor:
     """R = bf16(W diag(lambda) - (diag(lambda) down^T up^T)^T), computed in fp64."""

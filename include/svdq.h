@@ -65,7 +65,8 @@ typedef enum {
     SVDQ_ERR_MISALIGNED = 3,    /* pointer or row stride not 16-byte aligned */
     SVDQ_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, attribute) */
     SVDQ_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out */
-    SVDQ_ERR_NO_DEVICE = 6      /* no sm_100 device is current */
+    SVDQ_ERR_NO_DEVICE = 6,     /* no sm_100 device is current */
+    SVDQ_ERR_SCRATCH_TOO_SMALL = 7  /* problem needs more than the library's static scratch array */
 } svdq_status;
 
 /* Half-open row range [begin, end) of X; a host array of these selects rows. */
@@ -194,6 +195,35 @@ int svdq_score_lambda(const void* Yq, const void* Yref, int64_t M, int64_t N, in
                       const svdq_seg* segs, int n_seg,
                       double* num, double* den, double* rel,
                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * svdq_score_lambda_static -- svdq_score_lambda for callers that cannot
+ * allocate device memory (no counterpart in the paper: an interface addition).
+ *
+ * Some callers cannot call cudaMalloc while they score -- a host framework
+ * whose memory pool forbids side allocations, a launch sequence whose buffers
+ * were fixed beforehand, a plugin that is handed only its input and output
+ * tensors.  This entry point computes exactly what svdq_score_lambda computes,
+ * but keeps the per-block partial sums in a fixed array inside the library
+ * (svdq_score_static_max_bytes() bytes, 1 MiB, held on every GPU that loads the
+ * library until the process exits) instead of a workspace argument.  It
+ * allocates nothing.
+ *
+ * Limit: the problem must need at most svdq_score_static_max_bytes() of
+ * partial sums, i.e. svdq_score_workspace_bytes(segs, n_seg, N) <= 1 MiB
+ * (about 65536 blocks of 16384 elements); larger problems return
+ * SVDQ_ERR_SCRATCH_TOO_SMALL and launch nothing.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before capturing
+ * any stream.  All calls share the one array: calls whose kernels overlap on
+ * the GPU (different streams, no ordering between them) race and give wrong
+ * sums; calls ordered on one stream are safe.  Arguments and results are as
+ * for svdq_score_lambda.
+ */
+size_t svdq_score_static_max_bytes(void);
+int svdq_score_lambda_static(const void* Yq, const void* Yref, int64_t M, int64_t N, int64_t ld,
+                             const svdq_seg* segs, int n_seg,
+                             double* num, double* den, double* rel, void* stream);
 
 /*
  * svdq_residual -- offline weight conversion: the residual the 4-bit weight
