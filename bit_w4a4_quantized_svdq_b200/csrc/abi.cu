@@ -29,6 +29,8 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 EncodeTiledFn g_encode = nullptr;
 }  // namespace
 
+int current_device_index() { return current_device(); }
+
 uint32_t* device_error_word() {
     const int dev = current_device();
     if (dev < 0) return nullptr;

@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
@@ -56,6 +57,24 @@ int device_sm_count();
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t elem_bytes,
                     const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
                     uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
+// Current device ordinal, or -1.
+int current_device_index();
+
+// Raise a kernel's dynamic shared memory limit to `bytes`, once per device
+// (`done` is a per-kernel bit set over device ordinals 0..63).
+template <typename Kernel>
+inline bool set_dynamic_smem_once(Kernel kern, uint32_t bytes, std::atomic<uint64_t>& done) {
+    const int dev = current_device_index();
+    if (dev < 0) return false;
+    const uint64_t bit = uint64_t(1) << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return true;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+        cudaSuccess)
+        return false;
+    done.fetch_or(bit, std::memory_order_release);
+    return true;
+}
 
 inline int launch_status(cudaError_t e) {
     if (e == cudaSuccess) return SVDQ_OK;

@@ -447,8 +447,8 @@ int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMa
                   cudaStream_t st) {
     const uint32_t smem = kSmemBytes + 1024;
     auto kern = linear_kernel<kOutF32>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return SVDQ_ERR_CUDA;
+    static std::atomic<uint64_t> smem_set{0};
+    if (!set_dynamic_smem_once(kern, smem, smem_set)) return SVDQ_ERR_CUDA;
     const int tiles = a.m_tiles * a.n_tiles;
     const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
     const int grid = tiles < sms ? tiles : sms;

@@ -15,10 +15,16 @@
 //               matching r x 64 tile of the down weight and 64 values of
 //               1/lambda into an 8-stage ring
 //   warp 17     tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
-//   warps 0..15 quantisers: one lane per 16-element group (8 rows x 4 groups
-//               per warp and stage) read from the swizzled tile, E4M3 scale and
-//               E2M1 codes through the hardware RNE conversions, 8-byte code
-//               stores and one 4-byte scale word per row;
+//   warps 0..15 quantisers, in two teams of 8 that take alternate stages; a
+//               lane owns one 16-channel group in each of two rows (two
+//               independent dependency chains), reads them from the swizzled
+//               tile, multiplies by 1/lambda and later by 1/S with packed
+//               f32x2 multiplies, forms the E4M3 scales of both rows with one
+//               conversion and the E2M1 codes with the hardware RNE
+//               conversions, and stores 8-byte code words and 4-byte scale
+//               words; 1/S comes from a per-CTA table over the 127 finite
+//               non-negative E4M3 bytes (S = RN(dec(byte) * s_g), 1/S = RN(1/S)),
+//               built once at CTA start;
 //               warps 0..3 (one per tensor-memory lane quarter) finally read
 //               D_partial from tensor memory.
 // K is split across the CTAs of a thread-block cluster (up to 4); the partial
@@ -34,7 +40,9 @@ constexpr int kBM = 128;               // rows per CTA tile
 constexpr int kBK = 64;                // channels per stage (128 bytes of bf16)
 constexpr int kStages = 8;
 constexpr int kThreads = 576;
-constexpr int kQuantWarps = 16;       // 8 rows x 4 groups of 16 channels per warp and stage
+constexpr int kQuantWarps = 16;       // two teams of 8, alternate stages
+constexpr int kTeamWarps = 8;        // per stage: 16 rows x 4 groups of 16 channels per warp
+static_assert(kQuantWarps == 2 * kTeamWarps, "two teams of quantiser warps");
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kMaxSplit = 4;          // CTAs of a cluster along K
@@ -47,7 +55,8 @@ struct QSmem {
     static constexpr uint32_t kDownOff = kStages * kXTileBytes;
     static constexpr uint32_t kPartOff = kDownOff + kStages * kDownTileBytes;     // D partial [R][128] fp32
     static constexpr uint32_t kIlamOff = kPartOff + R * kBM * 4;                   // 1/lambda, 64 fp32 per stage
-    static constexpr uint32_t kBarOff = kIlamOff + kStages * kBK * 4;
+    static constexpr uint32_t kTabOff = kIlamOff + kStages * kBK * 4;              // 1/S per E4M3 byte, 128 fp32
+    static constexpr uint32_t kBarOff = kTabOff + 128 * 4;
     static constexpr uint32_t kBytes = kBarOff + 256;
 };
 
@@ -106,7 +115,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kQuantWarps + (R > 0 ? 1 : 0));
+            mbar_init(&empty[s], kTeamWarps + (R > 0 ? 1 : 0));
         }
         mbar_init(dfull, 1);
         *abort_flag = 0;
@@ -115,6 +124,13 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     if (R > 0 && warp == kMmaWarp) {
         tmem_alloc(tmem_slot, 32);
         tmem_relinquish();
+    }
+    if (threadIdx.x < 128) {
+        // 1/S for every scale byte the RNE-satfinite conversion can produce (0x00..0x7E).
+        const float s_g = __ldg(args.s_g);
+        const float S = __fmul_rn(e4m3_to_f32(threadIdx.x), s_g);
+        reinterpret_cast<float*>(smem + L::kTabOff)[threadIdx.x] =
+            (threadIdx.x == 0x7F || S == 0.0f) ? 0.0f : __frcp_rn(S);
     }
     tc_fence_before();
     __syncthreads();
@@ -167,72 +183,89 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         // ------------------------------------------------------------ quantisers
         const float s_g = __ldg(args.s_g);
         const float d = __fmul_rn(6.0f, s_g);
-        const int64_t M = args.M, K = args.K;
-        const int64_t half_k = K >> 1;
-        const int64_t atoms_k = K >> 6;
+        const int64_t M = args.M;
+        const int64_t half_k = args.K >> 1;
+        const int64_t atoms_k = args.K >> 6;
+        const bool has_il = args.inv_lambda != nullptr;
+        const float* rs_tab = reinterpret_cast<const float*>(smem + L::kTabOff);
         uint32_t sat = 0;
-        // Lane -> (row of the warp's 8, group of 16 channels); the group's two
-        // 16-byte halves are chunks 2b and 2b+1 of the row's 128-byte line.
+        // Team (stage parity), rows and group of this lane: rows r0 and r0 + 8
+        // of the tile, channels 16 b .. 16 b + 15 of the stage; the group's two
+        // 16-byte halves are chunks 2b and 2b+1 of the row's 128-byte line
+        // (both rows have the same swizzle phase, r0 % 8 == (r0 + 8) % 8).
+        const int team = warp / kTeamWarps;
         const int rw = lane >> 2;
         const int b = lane & 3;
-        const int row = warp * (kBM / kQuantWarps) + rw;                  // row inside the tile
-        const int64_t grow = static_cast<int64_t>(m_blk) * kBM + row;
-        const int ph0 = ((2 * b) ^ (row & 7)) << 4;
-        const int ph1 = ((2 * b + 1) ^ (row & 7)) << 4;
-        for (int i = 0; i < n_local; ++i) {
+        const int r0 = (warp % kTeamWarps) * 16 + rw;
+        const int64_t grow0 = static_cast<int64_t>(m_blk) * kBM + r0;
+        const int64_t grow1 = grow0 + 8;
+        const int ph0 = ((2 * b) ^ (r0 & 7)) << 4;
+        const int ph1 = ((2 * b + 1) ^ (r0 & 7)) << 4;
+        const uint64_t one2 = pack_f32x2(1.0f, 1.0f);
+        for (int i = team; i < n_local; i += 2) {
             const int s = i % kStages;
             const uint32_t ph = (i / kStages) & 1;
             if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
             const int chunk = c_begin + i;
-            const uint8_t* tile = smem + L::kXOff + s * kXTileBytes + row * 128;
-            const uint4 v0 = *reinterpret_cast<const uint4*>(tile + ph0);
-            const uint4 v1 = *reinterpret_cast<const uint4*>(tile + ph1);
-            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            float xs[16];
+            const uint8_t* tile = smem + L::kXOff + s * kXTileBytes;
+            const uint4 u0 = *reinterpret_cast<const uint4*>(tile + r0 * 128 + ph0);
+            const uint4 u1 = *reinterpret_cast<const uint4*>(tile + r0 * 128 + ph1);
+            const uint4 v0 = *reinterpret_cast<const uint4*>(tile + (r0 + 8) * 128 + ph0);
+            const uint4 v1 = *reinterpret_cast<const uint4*>(tile + (r0 + 8) * 128 + ph1);
+            uint64_t il[8];
+            if (has_il) {
+                const ulonglong2* ilp = reinterpret_cast<const ulonglong2*>(smem + L::kIlamOff + s * kBK * 4 + b * 64);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                xs[2 * j] = bf16_lo(w[j]);
-                xs[2 * j + 1] = bf16_hi(w[j]);
-            }
-            if (args.inv_lambda) {
-                const float4* il = reinterpret_cast<const float4*>(smem + L::kIlamOff + s * kBK * 4 + b * 64);
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 l = il[q4];
-                    xs[4 * q4] = __fmul_rn(xs[4 * q4], l.x);
-                    xs[4 * q4 + 1] = __fmul_rn(xs[4 * q4 + 1], l.y);
-                    xs[4 * q4 + 2] = __fmul_rn(xs[4 * q4 + 2], l.z);
-                    xs[4 * q4 + 3] = __fmul_rn(xs[4 * q4 + 3], l.w);
+                for (int q = 0; q < 4; ++q) {
+                    const ulonglong2 t = ilp[q];
+                    il[2 * q] = t.x;
+                    il[2 * q + 1] = t.y;
                 }
-            }
-            float a = 0.0f;
+            } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(xs[j]));
-            const float t = __fdiv_rn(a, d);
-            const uint32_t sfb = cvt_e4m3(t);
-            const float S = __fmul_rn(e4m3_to_f32(sfb), s_g);
-            const float rS = (S == 0.0f) ? 0.0f : __frcp_rn(S);
-            float q0[8], q1[8];
+                for (int q = 0; q < 8; ++q) il[q] = one2;
+            }
+            const uint32_t wa[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            const uint32_t wb[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            // xs = RN(x * (1/lambda)), element pairs (2j, 2j+1) of each row
+            uint64_t xa[8], xb[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                q0[j] = __fmul_rn(xs[j], rS);
-                q1[j] = __fmul_rn(xs[8 + j], rS);
+                xa[j] = mul_f32x2(bf16x2_to_f32x2(wa[j]), il[j]);
+                xb[j] = mul_f32x2(bf16x2_to_f32x2(wb[j]), il[j]);
             }
-            const uint2 packed = make_uint2(cvt_e2m1x8(q0), cvt_e2m1x8(q1));
-            if (t > 448.0f) ++sat;
-            // the row's 4 scale bytes (groups b = 0..3 in lanes 4 rw .. 4 rw + 3) -> one 32-bit word
-            uint32_t sfw = sfb;
-            sfw |= __shfl_down_sync(0xffffffffu, sfb, 1) << 8;
-            sfw |= __shfl_down_sync(0xffffffffu, sfb, 2) << 16;
-            sfw |= __shfl_down_sync(0xffffffffu, sfb, 3) << 24;
+            const float aa = absmax16(xa), ab = absmax16(xb);
+            const float ta = __fdiv_rn(aa, d), tb = __fdiv_rn(ab, d);
+            const uint32_t sf2 = cvt_e4m3x2(ta, tb);          // byte 0: row r0, byte 1: row r0 + 8
+            const float rsa = rs_tab[sf2 & 0xFFu], rsb = rs_tab[sf2 >> 8];
+            const uint64_t ra = pack_f32x2(rsa, rsa), rb = pack_f32x2(rsb, rsb);
+            uint64_t qa[8], qb[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                qa[j] = mul_f32x2(xa[j], ra);
+                qb[j] = mul_f32x2(xb[j], rb);
+            }
+            const uint2 ca = make_uint2(cvt_e2m1x8_pairs(qa[0], qa[1], qa[2], qa[3]),
+                                        cvt_e2m1x8_pairs(qa[4], qa[5], qa[6], qa[7]));
+            const uint2 cb = make_uint2(cvt_e2m1x8_pairs(qb[0], qb[1], qb[2], qb[3]),
+                                        cvt_e2m1x8_pairs(qb[4], qb[5], qb[6], qb[7]));
+            sat += (ta > 448.0f ? 1u : 0u) + (tb > 448.0f ? 1u : 0u);
+            // scale words of both rows: bytes of lanes 4 rw .. 4 rw + 3 (groups b = 0..3)
+            const uint32_t n1 = __shfl_down_sync(0xffffffffu, sf2, 1);
+            const uint32_t n2 = __shfl_down_sync(0xffffffffu, sf2, 2);
+            const uint32_t n3 = __shfl_down_sync(0xffffffffu, sf2, 3);
+            const uint32_t x01 = __byte_perm(sf2, n1, 0x5140);   // a0 b0 a1 b1
+            const uint32_t x23 = __byte_perm(n2, n3, 0x5140);    // c0 d0 c1 d1
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);        // shared memory of this stage no longer read
-            if (grow < M)
-                *reinterpret_cast<uint2*>(args.codes + grow * half_k + chunk * (kBK / 2) + b * 8) = packed;
+            uint8_t* cbase = args.codes + chunk * (kBK / 2) + b * 8;
+            if (grow0 < M) *reinterpret_cast<uint2*>(cbase + grow0 * half_k) = ca;
+            if (grow1 < M) *reinterpret_cast<uint2*>(cbase + grow1 * half_k) = cb;
             if (b == 0) {
-                const int64_t off = (static_cast<int64_t>(m_blk) * atoms_k + chunk) * 512 + (row & 31) * 16 +
-                                    ((row >> 5) & 3) * 4;
-                *reinterpret_cast<uint32_t*>(args.sf + off) = sfw;
+                uint8_t* atom = args.sf + (static_cast<int64_t>(m_blk) * atoms_k + chunk) * 512;
+                const int r1 = r0 + 8;
+                *reinterpret_cast<uint32_t*>(atom + (r0 & 31) * 16 + ((r0 >> 5) & 3) * 4) = __byte_perm(x01, x23, 0x5410);
+                *reinterpret_cast<uint32_t*>(atom + (r1 & 31) * 16 + ((r1 >> 5) & 3) * 4) = __byte_perm(x01, x23, 0x7632);
             }
         }
         // saturation count: one atomic per warp
@@ -322,8 +355,8 @@ int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const Quan
 
     const uint32_t smem = QSmem<R>::kBytes + 1024;
     auto kern = quantize_act_kernel<R>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return SVDQ_ERR_CUDA;
+    static std::atomic<uint64_t> smem_set{0};
+    if (!set_dynamic_smem_once(kern, smem, smem_set)) return SVDQ_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(m_tiles), static_cast<unsigned>(split), 1);
     cfg.blockDim = dim3(kThreads, 1, 1);

@@ -36,6 +36,15 @@ __device__ __forceinline__ uint32_t lane_id() {
     return l;
 }
 
+// Streaming 16-byte global load: read-only path, no L1 allocation (the data
+// is used once).
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
@@ -336,6 +345,71 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
     float f;
     asm volatile("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
     return f;
+}
+
+
+// ---------------------------------------------------------------------------
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: two IEEE round-to-nearest
+// operations per instruction, identical results to two scalar ones)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Two bf16 (low half = element 0) -> their exact fp32 values as a pair.
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+    return pack_f32x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// max_j |x_j| over 16 values held as 8 pairs (balanced tree).
+__device__ __forceinline__ float absmax16(const uint64_t (&x)[8]) {
+    float m[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float lo, hi;
+        unpack_f32x2(x[j], lo, hi);
+        m[j] = fmaxf(fabsf(lo), fabsf(hi));
+    }
+    const float a = fmaxf(m[0], m[1]), b = fmaxf(m[2], m[3]), c = fmaxf(m[4], m[5]), e = fmaxf(m[6], m[7]);
+    return fmaxf(fmaxf(a, b), fmaxf(c, e));
+}
+
+// Two non-negative fp32 -> two E4M3 bytes (RNE, saturating at 448): `lo` in
+// bits 0..7, `hi` in bits 8..15.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
+    return out;
+}
+
+// Four fp32 pairs -> eight E2M1 codes, pair j in byte j, element 2j in its low nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x8_pairs(uint64_t p0, uint64_t p1, uint64_t p2, uint64_t p3) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        ".reg .f32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
+        "mov.b64 {l0, h0}, %1;\n\t"
+        "mov.b64 {l1, h1}, %2;\n\t"
+        "mov.b64 {l2, h2}, %3;\n\t"
+        "mov.b64 {l3, h3}, %4;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, h0, l0;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, h1, l1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, h2, l2;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, h3, l3;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out) : "l"(p0), "l"(p1), "l"(p2), "l"(p3));
+    return out;
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }

@@ -64,6 +64,31 @@ def test_calib_ragged_and_without_weight(lib, m, k):
     assert g["s_g"].item() == float(c["s_g"])
 
 
+def test_calib_all_zero_rows_give_unit_scales(lib):
+    x = np.zeros((300, 1024), dtype=np.uint16)
+    x[:, 7] = 0x8000                                   # negative zeros only
+    w = S.random_bf16((64, 1024), 5, 0.02)
+    c = O.calib(x, None, w)
+    g = lib.svdq_calib_lambda(dev_bits(x), None, dev_bits(w))
+    assert np.all(g["lam"].cpu().numpy() == 1.0) and np.all(c["lam"] == 1.0)
+    assert g["s_g"].item() == 1.0 == float(c["s_g"])
+
+
+def test_calib_wide_k_many_strips_and_repeated_calls(lib):
+    """K = 20480 (the FFN down-projection width): 80 channel strips; two calls
+    into recycled output memory must agree with the oracle both times."""
+    x = S.random_bf16((300, 20480), 41, 2.0)
+    w = S.random_bf16((96, 20480), 42, 0.02)
+    segs = [(0, 7), (50, 299)]
+    c = O.calib(x, segs, w)
+    for _ in range(2):
+        g = lib.svdq_calib_lambda(dev_bits(x), segs, dev_bits(w))
+        for key, gk in (("ax", "amax_x"), ("aw", "amax_w"), ("lam", "lam"), ("inv_lam", "inv_lam")):
+            assert np.array_equal(g[gk].cpu().numpy(), c[key]), key
+        assert g["s_g"].item() == float(c["s_g"])
+        del g
+
+
 def _d_tolerance(x_bits, down_bits):
     """|D_gpu - D64| bound: fp32 accumulation of exact bf16 products."""
     ax = np.abs(O.bf16_to_f64(x_bits))
