@@ -265,8 +265,17 @@ def run_gpu(args):
                           lin.up, lin.bias, out=y)
         with torch.cuda.graph(graphs[3], stream=side, pool=graphs[0].pool()):
             g_res = P.svdq_score_lambda(y, yref, segs_mod, workspace=ws)
+        # the whole step (calib -> quantize -> linear -> score) as one graph
+        g_step = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step, stream=side, pool=graphs[0].pool()):
+            s_cal = P.svdq_calib_lambda(x, segs_all, w)
+            P.svdq_quantize_act(x, s_cal["inv_lam"], lin.s_g_act, lin.down, out=q_out)
+            P.svdq_linear(q_out["codes"], q_out["sf"], lin.s_g_act, q_out["d"], lin.w_codes, lin.w_sf, lin.s_g_w,
+                          lin.up, lin.bias, out=y)
+            s_res = P.svdq_score_lambda(y, yref, segs_mod, workspace=ws)
     torch.cuda.current_stream().wait_stream(side)
     for _ in range(args.warmup):
+        g_step.replay()
         for g in graphs:
             g.replay()
     torch.cuda.synchronize()
@@ -279,10 +288,18 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    step_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     for i in range(args.steps):
         # L2 flush between steps, outside the events: write a buffer larger than
         # L2, then read another one so the write-back of the dirty lines happens
         # here and every step starts from a cold, clean L2.
+        flush.fill_(i & 0xFF)
+        flush_read.sum()
+        step_evs[i][0].record()
+        g_step.replay()
+        step_evs[i][1].record()
+    # per-call breakdown: the same calls, one graph each, events between them
+    for i in range(args.steps):
         flush.fill_(i & 0xFF)
         flush_read.sum()
         evs[i][0].record()
@@ -294,7 +311,7 @@ def run_gpu(args):
         dist.barrier()
     clocks = sampler.stop()
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
-    step_ms = float(per.sum(axis=1).mean())
+    step_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in step_evs]))
     kern_ms = per.mean(axis=0)       # calib, quantize, linear, score
     t_local = torch.tensor([step_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -334,7 +351,7 @@ def run_gpu(args):
     e2e_value = flops * world / (float(e2e_ms.item()) * 1e-3) / 1e12
     rel = rel_host.tolist()
     # the graphs replay the same calls on the same data: same scores, bit for bit
-    graph_matches_eager = bool(torch.equal(g_res[2].cpu(), rel_host))
+    graph_matches_eager = bool(torch.equal(g_res[2].cpu(), rel_host) and torch.equal(s_res[2].cpu(), rel_host))
 
     err = P.svdq_device_error()
     line = None
@@ -352,7 +369,7 @@ def run_gpu(args):
                        "segments": {s.name: [s.begin, s.end] for s in layer.segments},
                        "parallelism": f"replicas x{world}",
                        "l2": "flushed between steps: 256 MiB write, then 256 MiB read (cold, clean L2)",
-                       "timing": "one CUDA graph per call, replayed back to back; CUDA events between them"},
+                       "timing": "the step as one CUDA graph, CUDA events around it; kernels_ms from one graph per call"},
             "kernels_ms": {"calib": kern_ms[0], "quantize": kern_ms[1], "linear": kern_ms[2],
                            "score": kern_ms[3]},
             "linear_tflops": lin_tflops, "quantize_gbs": quant_gbs, "calib_gbs": calib_gbs, "score_gbs": score_gbs,

@@ -39,12 +39,12 @@ namespace {
 constexpr int kBM = 128;               // rows per CTA tile
 constexpr int kBK = 64;                // channels per stage (128 bytes of bf16)
 constexpr int kStages = 8;
-constexpr int kThreads = 576;
-constexpr int kQuantWarps = 16;       // two teams of 8, alternate stages
-constexpr int kTeamWarps = 8;        // per stage: 16 rows x 4 groups of 16 channels per warp
-static_assert(kQuantWarps == 2 * kTeamWarps, "two teams of quantiser warps");
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
+constexpr int kTeams = 3;             // teams of quantiser warps take stages in turn
+constexpr int kTeamWarps = 8;         // per stage: 16 rows x 4 groups of 16 channels per warp
+constexpr int kQuantWarps = kTeams * kTeamWarps;
+constexpr int kProducerWarp = kQuantWarps;
+constexpr int kMmaWarp = kQuantWarps + 1;
+constexpr int kThreads = (kQuantWarps + 2) * 32;
 constexpr int kMaxSplit = 4;          // CTAs of a cluster along K
 constexpr uint32_t kXTileBytes = kBM * kBK * 2;  // 16 KB
 
@@ -79,6 +79,33 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
     return v;
+}
+
+// E4M3 scale byte and saturation (t > 448) of t = RN(a / d), a >= 0, d > 0,
+// for two groups.  With y = RN(1 / d): |a y - a / d| <= 2^-24 a / d < 1 ulp,
+// rounding a y to q adds at most 1/2 ulp and t is within 1/2 ulp of a / d, so
+// |q - t| < 2 ulp (a power-of-two boundary between them only widens the
+// bit-pattern steps used below).  E4M3 rounding and the test t > 448 are
+// monotonic in t: when the floats 3 steps below and above q give the same byte
+// and the same test, t gives them too.  Otherwise -- near a rounding boundary
+// of the byte, at 448, or for a = 0 -- the exact quotient decides.
+__device__ __forceinline__ uint32_t scale_byte_checked(float a, float d, float rd, uint32_t& sat) {
+    const float q = __fmul_rn(a, rd);
+    const uint32_t qb = __float_as_uint(q);
+    const float lo = __uint_as_float(qb - 3u), hi = __uint_as_float(qb + 3u);
+    const uint32_t b2 = cvt_e4m3x2(lo, hi);
+    const bool sat_lo = lo > 448.0f, sat_hi = hi > 448.0f;
+    if (a != 0.0f && qb >= 3u && (b2 & 0xFFu) == (b2 >> 8) && sat_lo == sat_hi) {
+        sat += sat_lo ? 1u : 0u;
+        return b2 & 0xFFu;
+    }
+    const float t = __fdiv_rn(a, d);
+    sat += t > 448.0f ? 1u : 0u;
+    return cvt_e4m3x2(t, 0.0f) & 0xFFu;
+}
+
+__device__ __forceinline__ uint32_t scale_bytes2(float a0, float a1, float d, float rd, uint32_t& sat) {
+    return scale_byte_checked(a0, d, rd, sat) | (scale_byte_checked(a1, d, rd, sat) << 8);
 }
 
 template <int R>
@@ -173,6 +200,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         // ------------------------------------------------------------ quantisers
         const float s_g = __ldg(args.s_g);
         const float d = __fmul_rn(6.0f, s_g);
+        const float rd = __frcp_rn(d);
         const int64_t M = args.M;
         const int64_t half_k = args.K >> 1;
         const int64_t atoms_k = args.K >> 6;
@@ -192,7 +220,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         const int ph0 = ((2 * b) ^ (r0 & 7)) << 4;
         const int ph1 = ((2 * b + 1) ^ (r0 & 7)) << 4;
         const uint64_t one2 = pack_f32x2(1.0f, 1.0f);
-        for (int i = team; i < n_local; i += 2) {
+        for (int i = team; i < n_local; i += kTeams) {
             const int s = i % kStages;
             const uint32_t ph = (i / kStages) & 1;
             if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
@@ -225,8 +253,10 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 xb[j] = mul_f32x2(bf16x2_to_f32x2(wb[j]), il[j]);
             }
             const float aa = absmax16(xa), ab = absmax16(xb);
-            const float ta = __fdiv_rn(aa, d), tb = __fdiv_rn(ab, d);
-            const uint32_t sf2 = cvt_e4m3x2(ta, tb);          // byte 0: row r0, byte 1: row r0 + 8
+            // Scale bytes and saturation of both rows from t = RN(a / d), through
+            // the product with 1/d where that is provably the same (see scale_from_amax).
+            uint32_t sat2 = 0;
+            const uint32_t sf2 = scale_bytes2(aa, ab, d, rd, sat2);   // byte 0: row r0, byte 1: row r0 + 8
             const float rsa = rs_tab[sf2 & 0xFFu], rsb = rs_tab[sf2 >> 8];
             const uint64_t ra = pack_f32x2(rsa, rsa), rb = pack_f32x2(rsb, rsb);
             uint64_t qa[8], qb[8];
@@ -239,7 +269,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                                         cvt_e2m1x8_pairs(qa[4], qa[5], qa[6], qa[7]));
             const uint2 cb = make_uint2(cvt_e2m1x8_pairs(qb[0], qb[1], qb[2], qb[3]),
                                         cvt_e2m1x8_pairs(qb[4], qb[5], qb[6], qb[7]));
-            sat += (ta > 448.0f ? 1u : 0u) + (tb > 448.0f ? 1u : 0u);
+            sat += sat2;
             // scale words of both rows: bytes of lanes 4 rw .. 4 rw + 3 (groups b = 0..3)
             const uint32_t n1 = __shfl_down_sync(0xffffffffu, sf2, 1);
             const uint32_t n2 = __shfl_down_sync(0xffffffffu, sf2, 2);

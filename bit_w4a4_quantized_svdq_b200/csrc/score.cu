@@ -142,6 +142,121 @@ score_finalize_kernel(ChunkPlan plan, const double* __restrict__ partial, double
     }
 }
 
+// ---------------------------------------------------------------------------
+// Streaming version for rows stored back to back (ld == N, N % 8 == 0): every
+// chunk is one contiguous run of 2 x 32 KB, so a producer warp copies whole
+// chunks with bulk copies into a 3-slot shared-memory ring (192 KB in flight
+// per SM) while 8 consumer warps reduce earlier chunks.  One persistent CTA
+// per SM takes chunks c = blockIdx.x, blockIdx.x + gridDim.x, ... so the CTAs
+// together stream through memory in order.  Each chunk is reduced by the same
+// thread mapping and the same reduction tree as score_partial_kernel: the
+// partial sums are bitwise the same.
+// ---------------------------------------------------------------------------
+constexpr int kStreamSlots = 3;
+constexpr int kStreamConsumerWarps = kThreads / 32;            // 8
+constexpr int kStreamThreads = kThreads + 32;                  // + producer warp
+constexpr uint32_t kChunkBytes = kElemsPerChunk * 2;           // 32 KB per input
+constexpr uint32_t kStreamSmem = kStreamSlots * 2 * kChunkBytes + 256;
+
+__device__ __forceinline__ double consumer_sum(double v, double* sh) {
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    asm volatile("bar.sync 1, %0;" :: "n"(kThreads) : "memory");
+    if (l == 0) sh[w] = v;
+    asm volatile("bar.sync 1, %0;" :: "n"(kThreads) : "memory");
+    v = (threadIdx.x < (kThreads >> 5)) ? sh[threadIdx.x] : 0.0;
+    if (w == 0)
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;   // valid in thread 0
+}
+
+__global__ void __launch_bounds__(kStreamThreads, 1)
+score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict__ yr, int64_t N,
+                    const __grid_constant__ ChunkPlan plan, int64_t n_chunks, double* __restrict__ partial,
+                    uint32_t* err) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStreamSlots * 2 * kChunkBytes);
+    uint64_t* empty = full + kStreamSlots;
+    uint32_t* n_elems = reinterpret_cast<uint32_t*>(empty + kStreamSlots);    // per slot
+    volatile uint32_t* abort_flag = n_elems + kStreamSlots;
+    __shared__ double sh[kThreads / 32];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStreamSlots; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kStreamConsumerWarps);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kStreamConsumerWarps) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int i = 0;
+            int seg = 0;
+            for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++i) {
+                const int s = i % kStreamSlots;
+                const uint32_t ph = (i / kStreamSlots) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, err, kErrWaitEmpty)) break;
+                while (seg + 1 < plan.n && c >= plan.chunk_prefix[seg + 1]) ++seg;   // c increases
+                const int64_t e0 = (c - plan.chunk_prefix[seg]) * kElemsPerChunk;
+                const int64_t e1 = min(e0 + kElemsPerChunk, plan.elems[seg]);
+                const uint32_t n = e1 > e0 ? static_cast<uint32_t>(e1 - e0) : 0u;
+                n_elems[s] = n;
+                mbar_arrive_expect_tx(&full[s], 4u * n);
+                if (n) {
+                    const int64_t off = plan.begin[seg] * N + e0;
+                    uint8_t* dst = smem + s * 2 * kChunkBytes;
+                    bulk_load(dst, yq + off, 2u * n, &full[s]);
+                    bulk_load(dst + kChunkBytes, yr + off, 2u * n, &full[s]);
+                }
+            }
+            for (int j = (i > kStreamSlots ? i - kStreamSlots : 0); j < i; ++j) {   // bounded drain
+                const long long t0 = clock64();
+                while (!mbar_try_wait(&full[j % kStreamSlots], (j / kStreamSlots) & 1) &&
+                       clock64() - t0 < kWaitLimitCycles) {}
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ consumers
+        int i = 0;
+        for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++i) {
+            const int s = i % kStreamSlots;
+            const uint32_t ph = (i / kStreamSlots) & 1;
+            if (!mbar_wait(&full[s], ph, abort_flag, err, kErrWaitFull)) break;
+            const uint32_t n = n_elems[s];
+            const uint8_t* qa = smem + s * 2 * kChunkBytes;
+            const uint8_t* qb = qa + kChunkBytes;
+            uint4 va[kVecPerThread], vb[kVecPerThread];
+#pragma unroll
+            for (int v = 0; v < kVecPerThread; ++v) {
+                const uint32_t e = (static_cast<uint32_t>(v) * kThreads + threadIdx.x) * 8;
+                if (e < n) {
+                    va[v] = *reinterpret_cast<const uint4*>(qa + 2 * e);
+                    vb[v] = *reinterpret_cast<const uint4*>(qb + 2 * e);
+                } else {
+                    va[v] = make_uint4(0, 0, 0, 0);
+                    vb[v] = make_uint4(0, 0, 0, 0);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);           // slot read: the producer may refill it
+            double num = 0.0, den = 0.0;
+#pragma unroll
+            for (int v = 0; v < kVecPerThread; ++v) accum8(va[v], vb[v], num, den);
+            num = consumer_sum(num, sh);
+            den = consumer_sum(den, sh);
+            if (threadIdx.x == 0) {
+                partial[2 * c] = num;
+                partial[2 * c + 1] = den;
+            }
+        }
+    }
+}
+
 }  // namespace
 
 // Shared by the entry point below; `partial` must hold 2 doubles per chunk.
@@ -153,8 +268,19 @@ int score_lambda_launch(const void* Yq, const void* Yref, int64_t M, int64_t N, 
     const int64_t chunks = plan.chunk_prefix[n_seg];
     if (partial_bytes < static_cast<size_t>(chunks) * 2 * sizeof(double)) return SVDQ_ERR_INVALID_ARG;
     if (chunks > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
-    score_partial_kernel<<<static_cast<unsigned>(chunks), kThreads, 0, cs>>>(
-        static_cast<const uint16_t*>(Yq), static_cast<const uint16_t*>(Yref), N, ld, plan, partial);
+    if (ld == N && N % 8 == 0) {
+        static std::atomic<uint64_t> smem_set{0};
+        if (!set_dynamic_smem_once(score_stream_kernel, kStreamSmem, smem_set)) return SVDQ_ERR_CUDA;
+        uint32_t* err = device_error_word();
+        if (err == nullptr) return SVDQ_ERR_CUDA;
+        const int64_t sms = device_sm_count() > 0 ? device_sm_count() : 148;
+        const int64_t grid = chunks < sms ? chunks : sms;
+        score_stream_kernel<<<static_cast<unsigned>(grid), kStreamThreads, kStreamSmem, cs>>>(
+            static_cast<const uint16_t*>(Yq), static_cast<const uint16_t*>(Yref), N, plan, chunks, partial, err);
+    } else {
+        score_partial_kernel<<<static_cast<unsigned>(chunks), kThreads, 0, cs>>>(
+            static_cast<const uint16_t*>(Yq), static_cast<const uint16_t*>(Yref), N, ld, plan, partial);
+    }
     if (cudaGetLastError() != cudaSuccess) return SVDQ_ERR_CUDA;
     score_finalize_kernel<<<n_seg, kThreads, 0, cs>>>(plan, partial, num, den, rel);
     return launch_status(cudaGetLastError());

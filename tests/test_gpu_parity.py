@@ -157,6 +157,42 @@ def test_quantize_ties_saturation_and_signed_zero(lib):
         assert int(sat.item()) == n_sat
 
 
+def _e4m3_boundaries():
+    """The finite positive E4M3 values' rounding midpoints, and 448 (saturation)."""
+    vals = sorted({float(O.e4m3_decode(np.array([b], np.uint8))[0]) for b in range(0x7F)})
+    mids = [(a + b) / 2 for a, b in zip(vals[:-1], vals[1:])]
+    return mids + [448.0]
+
+
+def test_quantize_scale_near_every_e4m3_boundary(lib):
+    """Group absmax a with a / (6 s_g) within +-4 fp32 ulps of each E4M3
+    rounding midpoint and of 448: the scale byte, the codes and the saturation
+    count must match the oracle's exact quotient bit for bit."""
+    for s_g in (np.float32(1.0), np.float32(0.0123), np.float32(3.7e-5)):
+        d = np.float64(np.float32(np.float32(6.0) * s_g))
+        targets = []
+        for m in _e4m3_boundaries():
+            a0 = np.float32(m * d)
+            bits = int(a0.view(np.uint32))
+            targets += [np.uint32(bits + j).view(np.float32) for j in range(-4, 5)]   # +-4 fp32 steps
+        g = len(targets)
+        k = (g * 16 + 63) // 64 * 64
+        inv = np.ones(k, np.float32)
+        x = np.zeros((2, k), np.float32)
+        for i, t in enumerate(targets):
+            inv[16 * i] = t                      # xs = RN(1 * t) = t: the group's absmax
+            x[0, 16 * i] = 1.0
+            x[1, 16 * i] = -1.0
+            x[:, 16 * i + 1] = 0.5               # a second, smaller element in every group
+        xb = S.f32_to_bf16_bits(x)
+        codes, sf, n_sat = O.quantize_blocks(xb, inv, s_g)
+        sat = torch.zeros(1, dtype=torch.int32, device="cuda")
+        q = lib.svdq_quantize_act(dev_bits(xb), dev_f32(inv), dev_f32(np.array([s_g])), None, sat_count=sat)
+        check_codes(q["codes"], codes)
+        check_sf(q["sf"], sf, 2, k)
+        assert int(sat.item()) == n_sat
+
+
 def test_quantize_zero_rows(lib):
     x = np.zeros((130, 128), np.uint16)
     q = lib.svdq_quantize_act(dev_bits(x), None, dev_f32(np.array([1.0])), dev_bits(S.random_bf16((16, 128), 1)))
@@ -245,6 +281,28 @@ def test_score_matches_oracle(lib, m, n):
     g2 = lib.svdq_score_lambda(dev_bits(yq), dev_bits(yref), segs)
     for a, b in zip(g, g2):
         assert torch.equal(a, b)      # fixed reduction order: bitwise reproducible
+
+
+def test_score_row_strided_and_odd_width(lib):
+    """Rows with a stride wider than N take the per-chunk kernel, back-to-back
+    rows the streaming one; both reduce each chunk in the same order, so the
+    results agree bit for bit.  N % 8 != 0 (scalar path, rows strided) against the oracle."""
+    m, n, ld = 1000, 512, 576
+    yref = S.random_bf16((m, ld), 17, 1.0)
+    yq = S.f32_to_bf16_bits(S.bf16_bits_to_f32(yref) + S.bf16_bits_to_f32(S.random_bf16((m, ld), 18, 0.05)))
+    segs = [(0, 13), (13, 990), (990, 1000)]
+    wide_q, wide_r = dev_bits(yq), dev_bits(yref)
+    strided = lib.svdq_score_lambda(wide_q[:, :n], wide_r[:, :n], segs)
+    packed = lib.svdq_score_lambda(wide_q[:, :n].contiguous(), wide_r[:, :n].contiguous(), segs)
+    for a, b in zip(strided, packed):
+        assert torch.equal(a, b)
+    num, den, rel = O.score(np.ascontiguousarray(yq[:, :n]), np.ascontiguousarray(yref[:, :n]), segs)
+    np.testing.assert_allclose(packed[2].cpu().numpy(), rel, rtol=1e-6, atol=0)
+    odd = 100                                 # rows stay 16-byte aligned through the stride
+    g = lib.svdq_score_lambda(wide_q[:, :odd], wide_r[:, :odd], segs)
+    q2, r2 = np.ascontiguousarray(yq[:, :odd]), np.ascontiguousarray(yref[:, :odd])
+    for a, b in zip(g, O.score(q2, r2, segs)):
+        np.testing.assert_allclose(a.cpu().numpy(), b, rtol=1e-6, atol=0)
 
 
 def test_score_identities(lib):
