@@ -53,8 +53,9 @@ struct QSmem {
     static constexpr uint32_t kDownTileBytes = R * kBK * 2;
     static constexpr uint32_t kXOff = 0;
     static constexpr uint32_t kDownOff = kStages * kXTileBytes;
-    static constexpr uint32_t kPartOff = kDownOff + kStages * kDownTileBytes;     // D partial [R][128] fp32
-    static constexpr uint32_t kIlamOff = kPartOff + R * kBM * 4;                   // 1/lambda, 64 fp32 per stage
+    static constexpr uint32_t kPartStride = R + 4;                                 // floats per row (padded)
+    static constexpr uint32_t kPartOff = kDownOff + kStages * kDownTileBytes;     // D partial [128][R + 4] fp32
+    static constexpr uint32_t kIlamOff = kPartOff + (R > 0 ? kBM * kPartStride * 4 : 0);   // 1/lambda, 64 fp32 per stage
     static constexpr uint32_t kTabOff = kIlamOff + kStages * kBK * 4;              // 1/S per E4M3 byte, 128 fp32
     static constexpr uint32_t kBarOff = kTabOff + 128 * 4;
     static constexpr uint32_t kBytes = kBarOff + 256;
@@ -73,11 +74,12 @@ struct QuantArgs {
     int split;         // CTAs along K (cluster size when R > 0)
 };
 
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t local_addr, uint32_t rank) {
     uint32_t remote;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(remote) : "memory");
     return v;
 }
 
@@ -293,8 +295,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         if (lane == 0 && sat && args.sat_count) atomicAdd(args.sat_count, sat);
 
         if (R > 0 && warp < 4) {   // one warp per tensor-memory lane quarter
-            float* part = reinterpret_cast<float*>(smem + L::kPartOff);   // [R][128]
-            const int row = warp * 32 + lane;
+            float* part = reinterpret_cast<float*>(smem + L::kPartOff) + (warp * 32 + lane) * L::kPartStride;
             if (mbar_wait(dfull, 0, abort_flag, args.err, kErrWaitMma)) {
                 tc_fence_after();
                 const uint32_t taddr = tmem_d + (static_cast<uint32_t>(warp * 32) << 16);
@@ -303,17 +304,23 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                     tmem_ld_32x32b_x32(taddr, v);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) part[j * kBM + row] = __uint_as_float(v[j]);
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(part + j) = make_float4(
+                            __uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                            __uint_as_float(v[j + 3]));
                 } else {
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(taddr, v);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) part[j * kBM + row] = __uint_as_float(v[j]);
+                    for (int j = 0; j < 16; j += 4)
+                        *reinterpret_cast<float4*>(part + j) = make_float4(
+                            __uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                            __uint_as_float(v[j + 3]));
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < R; ++j) part[j * kBM + row] = 0.0f;
+                for (int j = 0; j < R; ++j) part[j] = 0.0f;
             }
             tc_fence_before();
         }
@@ -321,22 +328,54 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
 
     __syncwarp();   // reconverge each warp before the warp-aligned cluster barrier
     if constexpr (R > 0) {
-        // Sum the split-K partials in cluster-rank order (deterministic) on rank 0.
+        // Sum the split-K partials in cluster-rank order (deterministic).  Every
+        // CTA of the cluster takes a share of the ranks (in groups of 4): it
+        // issues all its 16-byte loads from the peers' shared memory first and
+        // then adds them, so the loads' latencies overlap.
         cluster_sync_all();
-        if (cluster_ctarank() == 0 && warp < 4) {
+        if (warp < 4) {
+            constexpr int kNq = R / 4;                           // float4 groups per row
+            constexpr int kMaxQ = (kNq + 1) / 2 + 1;             // groups one CTA takes (split >= 2), or all
+            const int split = args.split;
+            const int cr = static_cast<int>(cluster_ctarank());
+            const int q0 = cr * kNq / split, q1 = (cr + 1) * kNq / split;
             const int row = warp * 32 + lane;
             const int64_t grow = static_cast<int64_t>(m_blk) * kBM + row;
-            const uint32_t base = smem_u32(smem + L::kPartOff);
-            if (grow < args.M) {
-                float* dst = args.D + grow * R;
-#pragma unroll 4
-                for (int j = 0; j < R; j += 4) {
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int c = 0; c < args.split; ++c)
+            const uint32_t base = smem_u32(smem + L::kPartOff) + row * L::kPartStride * 4;
+            if (split == 1) {
+                if (grow < args.M) {
+                    const float4* src = reinterpret_cast<const float4*>(smem + L::kPartOff) + row * (L::kPartStride / 4);
+                    float4* dst = reinterpret_cast<float4*>(args.D + grow * R);
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            acc[u] += ld_dsmem_f32(base + ((j + u) * kBM + row) * 4, c);
-                    *reinterpret_cast<float4*>(dst + j) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                    for (int q = 0; q < kNq; ++q) dst[q] = src[q];
+                }
+            } else {
+                // two groups at a time: at most 8 remote 16-byte loads in flight per thread
+                for (int t0 = 0; t0 < kMaxQ; t0 += 2) {
+                    float4 got[2][kMaxSplit];
+#pragma unroll
+                    for (int t = 0; t < 2; ++t)
+#pragma unroll
+                        for (int c = 0; c < kMaxSplit; ++c)
+                            if (q0 + t0 + t < q1 && c < split)
+                                got[t][c] = ld_dsmem_f32x4(base + (q0 + t0 + t) * 16, c);
+                    if (grow < args.M) {
+                        float4* dst = reinterpret_cast<float4*>(args.D + grow * R);
+#pragma unroll
+                        for (int t = 0; t < 2; ++t) {
+                            if (q0 + t0 + t < q1) {
+                                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                                for (int c = 0; c < kMaxSplit; ++c) {
+                                    if (c < split) {
+                                        acc.x += got[t][c].x; acc.y += got[t][c].y;
+                                        acc.z += got[t][c].z; acc.w += got[t][c].w;
+                                    }
+                                }
+                                dst[q0 + t0 + t] = acc;
+                            }
+                        }
+                    }
                 }
             }
         }
