@@ -352,42 +352,47 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             const uint16_t* bw = bt + half * (kBN / 2);
             const bool row_ok = row < args.M;
             if constexpr (!kOutF32) {
-                uint32_t packed[kBN / 4];
-#pragma unroll
-                for (int c = 0; c < kBN / 2 / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tbase + c * 32, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const uint32_t bb = *reinterpret_cast<const uint32_t*>(bw + c * 32 + 2 * j);
-                        packed[c * 16 + j] = pack_bf16x2(fmaf(alpha, __uint_as_float(v[2 * j]), bf16_lo(bb)),
-                                                         fmaf(alpha, __uint_as_float(v[2 * j + 1]), bf16_hi(bb)));
-                    }
-                }
-                // The accumulator has been read: let the next tile's MMAs start.
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
-                // Output through shared memory and the TMA: the low-rank operand
-                // area is free (this tile's low-rank MMAs completed before the
-                // accumulator was signalled full).  Each warp stages its 32 rows x
-                // 64 columns (128-byte swizzle) twice.  Bulk stores keep the
-                // scattered per-row writes off the load/store path the tensor
-                // core reads its operands through.
+                // Per 64-column half: two 32-column tensor-memory loads in flight per
+                // wait, alpha and bias, bf16 rows staged in shared memory (the
+                // low-rank operand area, free since this tile's low-rank MMAs
+                // completed before the accumulator was signalled full; 32 rows x 64
+                // columns per warp, 128-byte swizzle) and written by a TMA bulk
+                // store.  The accumulator is released as soon as the second half
+                // has been read, before its conversion.  Bulk stores keep the
+                // scattered per-row writes off the load/store path the tensor core
+                // reads its operands through.
                 uint8_t* stg = smem + kOffLrA + ew * 4096;
                 const int32_t grow0 = static_cast<int32_t>(m_blk * kBM + quarter * 32);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    if (h == 1) {
+                    uint32_t v[2][32];
+                    tmem_ld_32x32b_x32(tbase + (2 * h) * 32, v[0]);
+                    tmem_ld_32x32b_x32(tbase + (2 * h + 1) * 32, v[1]);
+                    tmem_ld_wait();
+                    if (h == 1) {                   // the accumulator has been read: next tile's MMAs may start
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(acc_empty);
+                    }
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int c = 2 * h + hh;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const uint32_t bb = *reinterpret_cast<const uint32_t*>(bw + c * 32 + 2 * j);
+                            pk[hh * 16 + j] = pack_bf16x2(fmaf(alpha, __uint_as_float(v[hh][2 * j]), bf16_lo(bb)),
+                                                          fmaf(alpha, __uint_as_float(v[hh][2 * j + 1]), bf16_hi(bb)));
+                        }
+                    }
+                    if (h == 1) {                   // the first half's store has finished reading the buffer
                         if (lane == 0) bulk_wait_read_all();
                         __syncwarp();
                     }
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
                         *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                            make_uint4(packed[h * 32 + 4 * c], packed[h * 32 + 4 * c + 1],
-                                       packed[h * 32 + 4 * c + 2], packed[h * 32 + 4 * c + 3]);
+                            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                     fence_async_shared();
                     __syncwarp();
                     if (lane == 0 && grow0 < args.M) {          // boxes wholly below row M are skipped
