@@ -12,7 +12,8 @@
 //   Y[m, n] = alpha * (sum_k A[m,k] B[n,k] + sum_j D'[m,j] up[n,j]) + bias[n]
 //   alpha   = s_g_act * s_g_w,   D' = D / alpha (split into bf16 hi + lo)
 //
-// One persistent CTA per SM walks 128 x 256 output tiles (M fastest).  Warps:
+// One persistent CTA per SM walks 128 x 256 output tiles (the smaller
+// operand's blocks fastest, so it stays in L2).  Warps:
 //   0     TMA producer: per 256-channel stage, A codes 128 x 128 B and B codes
 //         256 x 128 B (128-byte swizzle) plus 2 + 4 KB of scale atoms (bulk copies)
 //   1     tcgen05 issuer and tensor-memory owner: per tile 4 kind::f16 MMAs for
@@ -83,8 +84,22 @@ struct LinearArgs {
     const float* s_g_w;
     int r;
     int m_tiles, n_tiles;
+    int n_fastest;            // tile order: 1 = N fastest (the weight stays in L2), 0 = M fastest
     uint32_t* err;
 };
+
+// Output tile -> (M block, N block).  The order decides what the CTAs working
+// at the same time share: walking the smaller operand's blocks fastest keeps
+// that operand resident in L2 while the other streams through once.
+__device__ __forceinline__ void tile_coords(const LinearArgs& a, int tile, int& m_blk, int& n_blk) {
+    if (a.n_fastest) {
+        n_blk = tile % a.n_tiles;
+        m_blk = tile / a.n_tiles;
+    } else {
+        m_blk = tile % a.m_tiles;
+        n_blk = tile / a.m_tiles;
+    }
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
@@ -147,8 +162,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             int it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int m_blk = tile % args.m_tiles;
-                const int n_blk = tile / args.m_tiles;
+                int m_blk, n_blk;
+                tile_coords(args, tile, m_blk, n_blk);
                 for (int kb = 0; kb < k_stages; ++kb, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
@@ -223,8 +238,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             int local = 0;
             const int r = args.r;
             for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-                const int m_blk = tile % args.m_tiles;
-                const int n_blk = tile / args.m_tiles;
+                int m_blk, n_blk;
+                tile_coords(args, tile, m_blk, n_blk);
                 if (!mbar_wait(stage_free, (local & 1) ^ 1, abort_flag, args.err, kErrWaitLowRank)) break;
                 uint8_t* la = smem + kOffLrA;
                 uint8_t* lb = smem + kOffLrB;
@@ -339,8 +354,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         uint16_t* bias_s = reinterpret_cast<uint16_t*>(smem + kOffBias);
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-            const int m_blk = tile % args.m_tiles;
-            const int n_blk = tile / args.m_tiles;
+            int m_blk, n_blk;
+            tile_coords(args, tile, m_blk, n_blk);
             const int64_t col0 = static_cast<int64_t>(n_blk) * kBN;
             uint16_t* bt = bias_s + (local & 1) * kBN;
             bt[etid] = args.bias ? args.bias[col0 + etid] : static_cast<uint16_t>(0);
@@ -520,6 +535,8 @@ extern "C" int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const fl
     a.r = r;
     a.m_tiles = static_cast<int>(m_tiles);
     a.n_tiles = static_cast<int>(n_tiles);
+    a.n_fastest = N <= M ? 1 : 0;                        // the weight is the smaller operand
+
     a.err = err;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return out_dtype ? launch_linear<true>(ta, tb, ty, a, st) : launch_linear<false>(ta, tb, ty, a, st);
