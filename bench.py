@@ -37,6 +37,11 @@ WORKLOAD = "dit_attention_projection_M4096_K5120_N5120_r32"
 CONFIG_INDEX = 1
 L2_FLUSH_BYTES = 256 << 20
 FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+# DRAM bytes (read + write) per launch from one ncu capture of the current kernels on this
+# workload (profiles/linear_kernel_*.md, profiles/quantize_act_kernel_*.md); set to None
+# whenever the kernel changes until it is captured again.
+LINEAR_TRAFFIC_BYTES = 27.45e6 + 3.16e6
+QUANTIZE_TRAFFIC_BYTES = 42.32e6 + 0.13e6
 
 
 def read_peaks():
@@ -186,6 +191,62 @@ def _oracle_threads():
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+
+LARGE_SHAPES = ((2, "ffn_up_projection_M16384_K5120_N20480_r32"), (3, "ffn_down_projection_M16384_K20480_N5120_r32"))
+
+
+def largest_shapes(P, S, dev, fp4_peak, flush, flush_read, steps=10, warmup=3):
+    """The fused W4A4 linear on the two largest configured shapes, inputs
+    prepared by the same path (calibration, weight conversion, quantisation);
+    each call is one CUDA graph, timed with CUDA events, L2 flushed before each."""
+    import torch
+    out = {}
+    for cfg, name in LARGE_SHAPES:
+        L = S.make_layer(cfg)
+        x = torch.from_numpy(np.ascontiguousarray(L.x).view(np.int16)).to(dev)
+        w = torch.from_numpy(np.ascontiguousarray(L.w).view(np.int16)).to(dev)
+        bias = torch.from_numpy(np.ascontiguousarray(L.bias).view(np.int16)).to(dev)
+        segs = L.seg_ranges(L.calib_sets["all"])
+        cal = P.svdq_calib_lambda(x, segs, w)
+        lin = P.SVDQW4A4Linear.convert(w, bias, cal, L.rank)
+        q = P.svdq_quantize_act(x, cal["inv_lam"], lin.s_g_act, lin.down)
+        y = torch.empty((L.m, L.n), dtype=torch.bfloat16, device=dev)
+        def call():
+            P.svdq_linear(q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf, lin.s_g_w, lin.up,
+                          lin.bias, out=y)
+        call()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                call()
+        torch.cuda.current_stream().wait_stream(side)
+        for _ in range(warmup):
+            g.replay()
+        times = []
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            flush_read.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = float(np.median(times))
+        flops = 2.0 * L.m * L.n * L.k
+        # accuracy against the bf16 layer (sanity: the same quantity the step scores)
+        yref = torch.matmul(x.view(torch.bfloat16), w.view(torch.bfloat16).t()) + bias.view(torch.bfloat16)
+        rel = float(torch.linalg.vector_norm(y.float() - yref.float()) / torch.linalg.vector_norm(yref.float()))
+        out[name] = {"M": L.m, "K": L.k, "N": L.n, "rank": L.rank, "linear_ms": ms,
+                     "linear_tflops": flops / (ms * 1e-3) / 1e12,
+                     "frac_of_fp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak, "rel_l2_vs_bf16": rel}
+        del x, w, bias, cal, lin, q, y, yref, g
+        torch.cuda.empty_cache()
+    return out
+
 
 def run_gpu(args):
     import torch
@@ -354,6 +415,9 @@ def run_gpu(args):
     graph_matches_eager = bool(torch.equal(g_res[2].cpu(), rel_host) and torch.equal(s_res[2].cpu(), rel_host))
 
     err = P.svdq_device_error()
+    large = None
+    if world == 1 and not args.no_large:
+        large = largest_shapes(P, S, dev, fp4_peak, flush, flush_read)
     line = None
     if rank == 0:
         cpu = None
@@ -374,11 +438,12 @@ def run_gpu(args):
                            "score": kern_ms[3]},
             "linear_tflops": lin_tflops, "quantize_gbs": quant_gbs, "calib_gbs": calib_gbs, "score_gbs": score_gbs,
             "roofline": {"bound": "tensor", "kernel": "svdq_linear", "achieved": lin_tflops, "peak": fp4_peak,
-                         "unit": "TFLOP/s", "frac": lin_tflops / fp4_peak, "traffic": None,
+                         "unit": "TFLOP/s", "frac": lin_tflops / fp4_peak, "traffic": LINEAR_TRAFFIC_BYTES,
                          "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} x {FP4_PER_BF16:g} "
                                         "(nominal dense FP4/BF16 ratio)"},
             "roofline_hbm": {"kernel": "svdq_quantize_act", "achieved": quant_gbs, "peak": peaks["hbm"],
-                             "unit": "GB/s", "frac": quant_gbs / peaks["hbm"]},
+                             "unit": "GB/s", "frac": quant_gbs / peaks["hbm"], "traffic": QUANTIZE_TRAFFIC_BYTES,
+                             "bound": "hbm"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": m * k * 2,
                     "d2h_bytes_per_step": 8 * len(segs_mod)},
             "gpu_launches": launches_per_step * args.steps,
@@ -386,6 +451,7 @@ def run_gpu(args):
             "rel_l2_vs_bf16": dict(zip([s.name for s in layer.segments], rel)),
             "device_error": err,
             "graph_replay_matches_eager": graph_matches_eager,
+            "largest_shapes": large,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line))
@@ -402,6 +468,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-large", action="store_true", help="skip the two largest-shape GEMM measurements")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "svdq":
         args.warmup = 3
