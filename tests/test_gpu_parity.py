@@ -252,7 +252,8 @@ def test_linear_cfg0(lib, cfg0):
 
 @pytest.mark.parametrize("m,n,k,r,bias", [
     (128, 256, 256, 0, True), (1, 256, 512, 16, True), (200, 512, 768, 32, False), (384, 256, 1024, 32, True),
-    (300, 768, 512, 16, True), (129, 512, 2048, 0, False)])
+    (300, 768, 512, 16, True), (129, 512, 2048, 0, False),
+    (3200, 1024, 256, 32, True)])     # 100 whole tiles: a last wave too full to split into half tiles
 def test_linear_shapes(lib, m, n, k, r, bias):
     x = _outlier_x(m, k, 3 * m + k)
     w = S.random_bf16((n, k), n + k, 0.02)
