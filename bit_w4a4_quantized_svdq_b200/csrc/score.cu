@@ -11,6 +11,8 @@
 // segment's partials in index order and forms num, den and rel.
 #include <mutex>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -170,9 +172,14 @@ __device__ __forceinline__ double consumer_sum(double v, double* sh) {
     return v;   // valid in thread 0
 }
 
+__device__ __forceinline__ void consumers_sync_all() {
+    asm volatile("bar.sync 1, %0;" :: "n"(kThreads) : "memory");
+}
+
 __global__ void __launch_bounds__(kStreamThreads, 1)
 score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict__ yr, int64_t N,
                     const __grid_constant__ ChunkPlan plan, int64_t n_chunks, double* __restrict__ partial,
+                    double* __restrict__ num_out, double* __restrict__ den_out, double* __restrict__ rel_out,
                     uint32_t* err) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStreamSlots * 2 * kChunkBytes);
@@ -255,6 +262,31 @@ score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict_
             }
         }
     }
+
+    // Every chunk's partial is written: CTA s sums segment s's partials in index
+    // order, with the same tree as score_finalize_kernel (the launch is
+    // cooperative, so all CTAs are resident and the grid barrier is safe).
+    cooperative_groups::this_grid().sync();
+    if (warp < kStreamConsumerWarps) {
+        for (int s = blockIdx.x; s < plan.n; s += gridDim.x) {
+            double num = 0.0, den = 0.0;
+            for (int64_t c = plan.chunk_prefix[s] + threadIdx.x; c < plan.chunk_prefix[s + 1]; c += kThreads) {
+                num += __ldcg(partial + 2 * c);
+                den += __ldcg(partial + 2 * c + 1);
+            }
+            num = consumer_sum(num, sh);
+            den = consumer_sum(den, sh);
+            if (threadIdx.x == 0) {
+                num_out[s] = num;
+                den_out[s] = den;
+                double rel;
+                if (den > 0.0) rel = sqrt(num / den);
+                else rel = (num == 0.0) ? 0.0 : __longlong_as_double(0x7FF0000000000000LL);
+                rel_out[s] = rel;
+            }
+            consumers_sync_all();
+        }
+    }
 }
 
 }  // namespace
@@ -275,8 +307,19 @@ int score_lambda_launch(const void* Yq, const void* Yref, int64_t M, int64_t N, 
         if (err == nullptr) return SVDQ_ERR_CUDA;
         const int64_t sms = device_sm_count() > 0 ? device_sm_count() : 148;
         const int64_t grid = chunks < sms ? chunks : sms;
-        score_stream_kernel<<<static_cast<unsigned>(grid), kStreamThreads, kStreamSmem, cs>>>(
-            static_cast<const uint16_t*>(Yq), static_cast<const uint16_t*>(Yref), N, plan, chunks, partial, err);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+        cfg.blockDim = dim3(kStreamThreads, 1, 1);
+        cfg.dynamicSmemBytes = kStreamSmem;
+        cfg.stream = cs;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return launch_status(cudaLaunchKernelEx(&cfg, score_stream_kernel, static_cast<const uint16_t*>(Yq),
+                                                static_cast<const uint16_t*>(Yref), N, plan, chunks, partial, num,
+                                                den, rel, err));
     } else {
         score_partial_kernel<<<static_cast<unsigned>(chunks), kThreads, 0, cs>>>(
             static_cast<const uint16_t*>(Yq), static_cast<const uint16_t*>(Yref), N, ld, plan, partial);
