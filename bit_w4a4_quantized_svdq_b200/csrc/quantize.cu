@@ -13,7 +13,7 @@
 // slice of K:
 //   warp 16     TMA producer: 128 x 64 bf16 tiles of X (128-byte swizzle), the
 //               matching r x 64 tile of the down weight and 64 values of
-//               1/lambda into an 8-stage ring
+//               1/lambda into a 9-stage ring (a multiple of the 3 quantiser teams)
 //   warp 17     tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
 //   warps 0..15 quantisers, in two teams of 8 that take alternate stages; a
 //               lane owns one 16-channel group in each of two rows (two
@@ -38,13 +38,18 @@ namespace {
 
 constexpr int kBM = 128;               // rows per CTA tile
 constexpr int kBK = 64;                // channels per stage (128 bytes of bf16)
-constexpr int kStages = 8;
+constexpr int kStages = 9;
 constexpr int kTeams = 3;             // teams of quantiser warps take stages in turn
 constexpr int kTeamWarps = 8;         // per stage: 16 rows x 4 groups of 16 channels per warp
 constexpr int kQuantWarps = kTeams * kTeamWarps;
 constexpr int kProducerWarp = kQuantWarps;
 constexpr int kMmaWarp = kQuantWarps + 1;
 constexpr int kThreads = (kQuantWarps + 2) * 32;
+// Stage i sits in slot i % kStages and is quantised by team i % kTeams.  A
+// parity wait only tells the current phase from the one before it, so a slot
+// must always be consumed by the same team: otherwise a team a whole ring lap
+// ahead could take the slot's unfinished phase for its own (completed) one.
+static_assert(kStages % kTeams == 0, "every slot is consumed by one team");
 constexpr int kMaxSplit = 4;          // CTAs of a cluster along K
 constexpr uint32_t kXTileBytes = kBM * kBK * 2;  // 16 KB
 

@@ -84,3 +84,15 @@ def check_linear_f32(y_gpu: np.ndarray, y64: np.ndarray, tight_rel: float = None
     if tight_rel is not None:
         assert rel <= tight_rel, f"rel-L2 {rel:.3e} above the expected {tight_rel:.1e}"
     return rel, mx
+
+
+def d_tolerance(x_bits: np.ndarray, down_bits: np.ndarray) -> np.ndarray:
+    """Bound on |D_gpu - D64|: D is accumulated in fp32 over K/16 MMA steps (16
+    exact bf16 products each) and a split-K sum of at most 4 partials, so the
+    recursive-summation bound (n additions, unit roundoff 2^-24) applies with
+    n = K/16 + 20: |error| <= n * 2^-24 * sum_k |x_k down_k|."""
+    k = x_bits.shape[1]
+    n = k // 16 + 20
+    ax = np.abs(O.bf16_to_f64(x_bits))
+    ad = np.abs(O.bf16_to_f64(down_bits))
+    return n * 2.0 ** -24 * (ax @ ad.T) + 1e-30
