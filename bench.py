@@ -40,8 +40,8 @@ FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (
 # DRAM bytes (read + write) per launch from one ncu capture of the current kernels on this
 # workload (profiles/linear_kernel_*.md, profiles/quantize_act_kernel_*.md); set to None
 # whenever the kernel changes until it is captured again.
-LINEAR_TRAFFIC_BYTES = 27.45e6 + 3.16e6
-QUANTIZE_TRAFFIC_BYTES = 42.32e6 + 0.13e6
+LINEAR_TRAFFIC_BYTES = 27.45e6 + 2.20e6
+QUANTIZE_TRAFFIC_BYTES = 42.32e6 + 0.11e6
 
 
 def read_peaks():
@@ -192,6 +192,34 @@ def _oracle_threads():
 # GPU arm
 # ---------------------------------------------------------------------------
 
+def _graph_ms(fn, flush, flush_read, reps=10, warmup=3):
+    """Median time of `fn` captured as one CUDA graph, L2 flushed before each replay."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(warmup):
+        g.replay()
+    times = []
+    for i in range(reps):
+        flush.fill_(i & 0xFF)
+        flush_read.sum()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    del g
+    return float(np.median(times))
+
+
 LARGE_SHAPES = ((2, "ffn_up_projection_M16384_K5120_N20480_r32"), (3, "ffn_down_projection_M16384_K20480_N5120_r32"))
 
 
@@ -211,31 +239,9 @@ def largest_shapes(P, S, dev, fp4_peak, flush, flush_read, steps=10, warmup=3):
         lin = P.SVDQW4A4Linear.convert(w, bias, cal, L.rank)
         q = P.svdq_quantize_act(x, cal["inv_lam"], lin.s_g_act, lin.down)
         y = torch.empty((L.m, L.n), dtype=torch.bfloat16, device=dev)
-        def call():
-            P.svdq_linear(q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf, lin.s_g_w, lin.up,
-                          lin.bias, out=y)
-        call()
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
-            with torch.cuda.graph(g, stream=side):
-                call()
-        torch.cuda.current_stream().wait_stream(side)
-        for _ in range(warmup):
-            g.replay()
-        times = []
-        for i in range(steps):
-            flush.fill_(i & 0xFF)
-            flush_read.sum()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            g.replay()
-            e1.record()
-            torch.cuda.synchronize()
-            times.append(e0.elapsed_time(e1))
-        ms = float(np.median(times))
+        ms = _graph_ms(lambda: P.svdq_linear(q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf,
+                                             lin.s_g_w, lin.up, lin.bias, out=y), flush, flush_read,
+                       reps=steps, warmup=warmup)
         flops = 2.0 * L.m * L.n * L.k
         # accuracy against the bf16 layer (sanity: the same quantity the step scores)
         yref = torch.matmul(x.view(torch.bfloat16), w.view(torch.bfloat16).t()) + bias.view(torch.bfloat16)
@@ -243,8 +249,65 @@ def largest_shapes(P, S, dev, fp4_peak, flush, flush_read, steps=10, warmup=3):
         out[name] = {"M": L.m, "K": L.k, "N": L.n, "rank": L.rank, "linear_ms": ms,
                      "linear_tflops": flops / (ms * 1e-3) / 1e12,
                      "frac_of_fp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak, "rel_l2_vs_bf16": rel}
-        del x, w, bias, cal, lin, q, y, yref, g
+        del x, w, bias, cal, lin, q, y, yref
         torch.cuda.empty_cache()
+    return out
+
+
+def all_configs(P, S, dev, fp4_peak, hbm_peak, flush, flush_read):
+    """Every call of the path on every configured workload (sweep: one layer per N,
+    every lambda candidate), each timed alone from a cold L2."""
+    import torch
+
+    def to_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
+
+    def layer_calls(L, calib_name):
+        x, w, bias = to_dev(L.x), to_dev(L.w), to_dev(L.bias)
+        segs_cal = L.seg_ranges(L.calib_sets[calib_name]) if calib_name != "1" else \
+            L.seg_ranges(L.calib_sets["all"])
+        w_cal = None if calib_name == "1" else w
+        segs_mod = [(sg.begin, sg.end) for sg in L.segments]
+        cal = P.svdq_calib_lambda(x, segs_cal, w_cal)
+        lin = P.SVDQW4A4Linear.convert(w, bias, cal, L.rank)
+        q = P.svdq_quantize_act(x, cal["inv_lam"], lin.s_g_act, lin.down)
+        y = torch.empty((L.m, L.n), dtype=torch.bfloat16, device=dev)
+        yref = torch.matmul(x.view(torch.bfloat16), w.view(torch.bfloat16).t()) + bias.view(torch.bfloat16)
+        ws = torch.empty(P.score_workspace_bytes(segs_mod, L.n), dtype=torch.uint8, device=dev)
+        m_sel = sum(e - b for b, e in segs_cal)
+        r = {}
+        t = _graph_ms(lambda: P.svdq_calib_lambda(x, segs_cal, w_cal), flush, flush_read)
+        by = 2.0 * m_sel * L.k + (2.0 * L.n * L.k if w_cal is not None else 0.0)
+        r["calib"] = {"ms": t, "GB/s": by / (t * 1e-3) / 1e9, "frac_hbm": by / (t * 1e-3) / 1e9 / hbm_peak}
+        t = _graph_ms(lambda: P.svdq_quantize_act(x, cal["inv_lam"], lin.s_g_act, lin.down, out=q), flush,
+                      flush_read)
+        by = (2 + 0.5 + 0.0625) * L.m * L.k + 4.0 * L.m * L.rank
+        r["quantize"] = {"ms": t, "GB/s": by / (t * 1e-3) / 1e9, "frac_hbm": by / (t * 1e-3) / 1e9 / hbm_peak}
+        t = _graph_ms(lambda: P.svdq_linear(q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf,
+                                            lin.s_g_w, lin.up, lin.bias, out=y), flush, flush_read)
+        fl = 2.0 * L.m * L.n * L.k
+        r["linear"] = {"ms": t, "TFLOP/s": fl / (t * 1e-3) / 1e12, "frac_fp4": fl / (t * 1e-3) / 1e12 / fp4_peak}
+        t = _graph_ms(lambda: P.svdq_score_lambda(y, yref, segs_mod, workspace=ws), flush, flush_read)
+        by = 4.0 * L.m * L.n
+        r["score"] = {"ms": t, "GB/s": by / (t * 1e-3) / 1e9, "frac_hbm": by / (t * 1e-3) / 1e9 / hbm_peak}
+        _, _, rel = P.svdq_score_lambda(y, yref, segs_mod, workspace=ws)
+        r["rel_l2_vs_bf16"] = dict(zip([sg.name for sg in L.segments], rel.cpu().tolist()))
+        del x, w, bias, cal, lin, q, y, yref, ws
+        torch.cuda.empty_cache()
+        return r
+
+    out = {}
+    for cfg in (0, 1, 2, 3):
+        L = S.make_layer(cfg)
+        names = ["all", "video"] if cfg == 3 else ["all"]
+        for name in names:
+            out[f"config{cfg}_M{L.m}_K{L.k}_N{L.n}_r{L.rank}_lambda_{name}"] = layer_calls(L, name)
+        del L
+    for layer in (0, 4, 5):                          # one sweep layer per N (5120, 15360, 20480)
+        L = S.make_layer(4, layer=layer)
+        for name in ("1", "all", "video", "text"):
+            out[f"config4_layer{layer}_M{L.m}_K{L.k}_N{L.n}_r{L.rank}_lambda_{name}"] = layer_calls(L, name)
+        del L
     return out
 
 
@@ -446,6 +509,9 @@ def run_gpu(args):
     large = None
     if world == 1 and not args.no_large:
         large = largest_shapes(P, S, dev, fp4_peak, flush, flush_read)
+    per_config = None
+    if world == 1 and args.all_configs:
+        per_config = all_configs(P, S, dev, fp4_peak, peaks["hbm"], flush, flush_read)
     line = None
     if rank == 0:
         cpu = None
@@ -486,6 +552,7 @@ def run_gpu(args):
             "device_error": err,
             "graph_replay_matches_eager": graph_matches_eager,
             "largest_shapes": large,
+            "all_configs": per_config,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line))
@@ -503,6 +570,8 @@ def main():
     ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-large", action="store_true", help="skip the two largest-shape GEMM measurements")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="also time every call on every configured workload (adds a few minutes)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "svdq":
         args.warmup = 3

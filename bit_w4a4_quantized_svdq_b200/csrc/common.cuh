@@ -58,6 +58,11 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t elem_b
                     const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
                     uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
+// Unswizzled 3-D map of bytes: dims {d0, d1, d2} (d0 innermost, contiguous),
+// byte strides s1 (dimension 1) and s2 (dimension 2), box {b0, b1, b2}.
+bool encode_tmap_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                       uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2);
+
 // Current device ordinal, or -1.
 int current_device_index();
 

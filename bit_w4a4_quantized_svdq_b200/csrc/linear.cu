@@ -15,16 +15,19 @@
 // One persistent CTA per SM walks 128 x 256 output tiles (the smaller
 // operand's blocks fastest, so it stays in L2).  Warps:
 //   0     TMA producer: per 256-channel stage, A codes 128 x 128 B and B codes
-//         256 x 128 B (128-byte swizzle) plus 2 + 4 KB of scale atoms (bulk copies)
-//   1     tcgen05 issuer and tensor-memory owner: per tile 4 kind::f16 MMAs for
-//         the low-rank term (K = 64: 32 ranks of D'_hi then 32 of D'_lo against
-//         up twice), then per stage 4 kind::mxf4nvf4 block16 MMAs (K = 64 each)
-//         into one fp32 accumulator
+//         256 x 128 B (128-byte swizzle); every second stage, the scale atoms of
+//         the next two stages (A 4 KB, W 8 KB) with two 3-D tensor loads into a
+//         2-slot ring
+//   1     tcgen05 issuer and tensor-memory owner: per stage one barrier wait and
+//         4 kind::mxf4nvf4 block16 MMAs (K = 64 each) into one fp32
+//         accumulator, then per tile 4 kind::f16 MMAs for the low-rank term
+//         (K = 64: 32 ranks of D'_hi then 32 of D'_lo against up twice)
 //   2     low-rank operand builder: D' hi/lo and the duplicated up tile written
 //         into the swizzled operand layout in shared memory
 //   3..6  block-scale writers: each stage's scale atoms, shared memory ->
 //         registers -> tensor memory (tcgen05.st, one warp per lane quarter),
-//         into a per-stage buffer; this keeps the tensor pipe free for MMAs
+//         into a per-stage buffer, then an arrival on the stage's barrier; this
+//         keeps the tensor pipe free for MMAs
 //   7..14 epilogue (two warps per tensor-memory lane quarter): tensor memory ->
 //         registers, alpha and bias, bf16 rows staged in shared memory and
 //         written by TMA bulk stores (fp32 rows: plain stores); the accumulator
@@ -32,6 +35,14 @@
 //         next tile's main loop.
 // The low-rank MMAs close each tile, so their operand area doubles as the
 // epilogue's output staging: builder -> MMA -> epilogue -> builder.
+//
+// What paces the main loop (measured on B200 with a stripped main-loop kernel):
+// the tensor pipe keeps only a short queue, so every instruction the issuing
+// thread runs between MMAs shows up as idle tensor cycles (hence one barrier
+// wait per stage, stage and phase kept as counters, descriptors precomputed);
+// and the TMA unit spends a roughly fixed time per copy, so the scale atoms
+// travel in as few copies as possible (two per two stages instead of three per
+// stage).
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -51,18 +62,22 @@ constexpr int kEpiWarps = 8;
 
 constexpr uint32_t kATile = kBM * kBKBytes;          // 16 KB
 constexpr uint32_t kBTile = kBN * kBKBytes;          // 32 KB
-constexpr uint32_t kSfaTile = kBM * (kBK / 16);      // 2 KB: 4 atoms of 512 B
-constexpr uint32_t kSfbTile = kBN * (kBK / 16);      // 4 KB: 2 row blocks x 4 atoms
-constexpr uint32_t kStageBytes = kATile + kBTile + kSfaTile + kSfbTile;
+constexpr uint32_t kStageBytes = kATile + kBTile;
+// Scale atoms (512 B per 128 rows x 64 channels) of two consecutive stages:
+// A: 8 atoms of the tile's row block; W: 8 atoms of each of its two row blocks.
+constexpr uint32_t kSfaPair = 4096;
+constexpr uint32_t kSfSlot = kSfaPair + 8192;        // 12 KB
 constexpr uint32_t kLrA = kBM * 128;                 // 128 rows x 64 bf16
 constexpr uint32_t kLrB = kBN * 128;                 // 256 rows x 64 bf16
 
 constexpr uint32_t kOffStages = 0;
-constexpr uint32_t kOffLrA = kStages * kStageBytes;  // multiple of 1024
+constexpr uint32_t kOffSf = kStages * kStageBytes;   // 2 slots, multiple of 1024
+constexpr uint32_t kOffLrA = kOffSf + 2 * kSfSlot;
 constexpr uint32_t kOffLrB = kOffLrA + kLrA;
 constexpr uint32_t kOffBar = kOffLrB + kLrB;
 constexpr uint32_t kOffBias = kOffBar + 256;          // 2 x 256 bf16 bias staging
 constexpr uint32_t kSmemBytes = kOffBias + 2 * kBN * 2;
+static_assert(kSmemBytes + 1024 <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
 
 // Tensor-memory columns: accumulator [0, 256), then one block-scale buffer per
 // pipeline stage (48 columns each: A scales 4 per MMA, B scales 8 per MMA).
@@ -110,7 +125,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <bool kOutF32>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-              const __grid_constant__ CUtensorMap tmap_y, LinearArgs args) {
+              const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_sfa,
+              const __grid_constant__ CUtensorMap tmap_sfb, LinearArgs args) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -119,8 +135,9 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* lr_full = acc_empty + 1;
     uint64_t* stage_free = lr_full + 1;                     // epilogue done with the staging area
-    uint64_t* sf_full = stage_free + 1;                     // kStages
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + kStages);
+    uint64_t* sf_data = stage_free + 1;                     // 2 slots: scale atoms landed
+    uint64_t* sf_free = sf_data + 2;                        // 2 slots: the writers have read them
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_free + 2);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5;
@@ -133,9 +150,12 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 1 + kSfWarps);              // operand bytes + the stage's scales in tensor memory
             mbar_init(&empty[s], 1);
-            mbar_init(&sf_full[s], kSfWarps);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sf_data[i], 1);
+            mbar_init(&sf_free[i], kSfWarps);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kEpiWarps);
@@ -158,26 +178,46 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         if (lane == 0) {
             prefetch_tmap(&tmap_a);
             prefetch_tmap(&tmap_b);
-            const int64_t atoms_k = args.K / 64;
-            int it = 0;
-            bool ok = true;
+            prefetch_tmap(&tmap_sfa);
+            prefetch_tmap(&tmap_sfb);
+            // Scale batches run one batch (two stages) ahead of the operands: the
+            // batch a stage needs has landed by the time its operands do.
+            int sf_tile = blockIdx.x, sf_kb = 0, issued = 0;
+            auto issue_scales = [&]() -> bool {
+                if (sf_tile >= num_tiles) return true;
+                const int slot = issued & 1;
+                if (issued >= 2 &&
+                    !mbar_wait(&sf_free[slot], ((issued >> 1) & 1) ^ 1, abort_flag, args.err, kErrWaitEmpty))
+                    return false;
+                int m_blk, n_blk;
+                tile_coords(args, sf_tile, m_blk, n_blk);
+                uint8_t* dst = smem + kOffSf + slot * kSfSlot;
+                mbar_arrive_expect_tx(&sf_data[slot], kSfSlot);
+                // scale atoms of stages sf_kb and sf_kb + 1 (a last odd stage reads zeros past K)
+                tma_load_3d(dst, &tmap_sfa, &sf_data[slot], 0, sf_kb * 8, m_blk);
+                tma_load_3d(dst + kSfaPair, &tmap_sfb, &sf_data[slot], 0, sf_kb * 8, 2 * n_blk);
+                ++issued;
+                sf_kb += 2;
+                if (sf_kb >= k_stages) {
+                    sf_kb = 0;
+                    sf_tile += gridDim.x;
+                }
+                return true;
+            };
+            int s = 0, it = 0;
+            uint32_t ph = 0;
+            bool ok = issue_scales();
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 int m_blk, n_blk;
                 tile_coords(args, tile, m_blk, n_blk);
                 for (int kb = 0; kb < k_stages; ++kb, ++it) {
-                    const int s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1;
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) { ok = false; break; }
                     uint8_t* st = smem + kOffStages + s * kStageBytes;
                     mbar_arrive_expect_tx(&full[s], kStageBytes);
                     tma_load_2d(st, &tmap_a, &full[s], kb * kBKBytes, m_blk * kBM);
                     tma_load_2d(st + kATile, &tmap_b, &full[s], kb * kBKBytes, n_blk * kBN);
-                    bulk_load(st + kATile + kBTile, args.a_sf + (static_cast<int64_t>(m_blk) * atoms_k + kb * 4) * 512,
-                              kSfaTile, &full[s]);
-                    const uint8_t* sfb0 = args.w_sf + (static_cast<int64_t>(2 * n_blk) * atoms_k + kb * 4) * 512;
-                    bulk_load(st + kATile + kBTile + kSfaTile, sfb0, kSfbTile / 2, &full[s]);
-                    bulk_load(st + kATile + kBTile + kSfaTile + kSfbTile / 2, sfb0 + atoms_k * 512, kSfbTile / 2,
-                              &full[s]);
+                    if ((kb & 1) == 0 && !issue_scales()) { ok = false; break; }
+                    if (++s == kStages) { s = 0; ph ^= 1u; }
                 }
             }
             // Bounded drain of the copies still in flight.
@@ -185,36 +225,43 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 const long long t0 = clock64();
                 while (!mbar_try_wait(&full[i % kStages], (i / kStages) & 1) && clock64() - t0 < kWaitLimitCycles) {}
             }
+            for (int q = (issued > 2 ? issued - 2 : 0); q < issued; ++q) {
+                const long long t0 = clock64();
+                while (!mbar_try_wait(&sf_data[q & 1], (q >> 1) & 1) && clock64() - t0 < kWaitLimitCycles) {}
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Kept to the minimum between MMAs: one wait per stage (the barrier counts
+        // the operand bytes and the four scale writers), counters instead of
+        // divisions, descriptors advanced by constant offsets.
         if (lane == 0) {
             const uint32_t idesc_f4 = idesc_nvf4(kBM, kBN);
             const uint32_t idesc_lr = idesc_bf16(kBM, kBN);
-            int it = 0;
-            int local = 0;
+            const uint64_t da0 = desc_kmajor_sw128(smem_u32(smem + kOffStages));
+            const uint64_t db0 = desc_kmajor_sw128(smem_u32(smem + kOffStages + kATile));
+            constexpr uint64_t kStageDesc = kStageBytes >> 4;     // descriptor address field counts 16 bytes
+            int s = 0, local = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
                 if (!mbar_wait(acc_empty, (local & 1) ^ 1, abort_flag, args.err, kErrWaitAccum)) break;
                 tc_fence_after();
-                bool first = true;
-                for (int kb = 0; kb < k_stages; ++kb, ++it) {
-                    const int s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1;
-                    if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) { ok = false; break; }
-                    if (!mbar_wait(&sf_full[s], ph, abort_flag, args.err, kErrWaitFull)) { ok = false; break; }
-                    tc_fence_after();
-                    uint8_t* st = smem + kOffStages + s * kStageBytes;
-                    const uint32_t sf = tmem + kTmemSf0 + s * kTmemSfStride;
-                    const uint32_t a0 = smem_u32(st);
-                    const uint32_t b0 = smem_u32(st + kATile);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        mma_nvf4(tmem, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc_f4,
-                                 sf + 4 * kk, sf + kTmemSfbOff + 8 * kk, (first && kk == 0) ? 0u : 1u);
+                for (int kb = 0; kb < k_stages; ++kb) {
+                    if (!mbar_try_wait(&full[s], ph) &&
+                        !mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) {
+                        ok = false;
+                        break;
                     }
-                    first = false;
+                    tc_fence_after();
+                    const uint64_t da = da0 + kStageDesc * s, db = db0 + kStageDesc * s;
+                    const uint32_t sf = tmem + kTmemSf0 + s * kTmemSfStride;
+                    mma_nvf4(tmem, da, db, idesc_f4, sf, sf + kTmemSfbOff, kb == 0 ? 0u : 1u);
+                    mma_nvf4(tmem, da + 2, db + 2, idesc_f4, sf + 4, sf + kTmemSfbOff + 8, 1u);
+                    mma_nvf4(tmem, da + 4, db + 4, idesc_f4, sf + 8, sf + kTmemSfbOff + 16, 1u);
+                    mma_nvf4(tmem, da + 6, db + 6, idesc_f4, sf + 12, sf + kTmemSfbOff + 24, 1u);
                     tc_commit(&empty[s]);
+                    if (++s == kStages) { s = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
                 if (has_lr) {
@@ -301,44 +348,62 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         }
     } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------------ block-scale writers
-        // Each warp copies the stage's scale atoms from shared memory into its
-        // own tensor-memory lane quarter with tcgen05.st (every quarter holds
-        // the full set, the layout the block-scaled MMA reads).  Unlike a
-        // shared->tensor copy issued by the MMA thread, these stores run
-        // alongside the MMAs instead of in front of them.  Buffer s is free
-        // again once stage s has been refilled: the refill waited for the MMAs
-        // that read it.
+        // Each warp copies the stage's scale atoms from the shared-memory ring
+        // into its own tensor-memory lane quarter with tcgen05.st (every quarter
+        // holds the full set, the layout the block-scaled MMA reads), then
+        // arrives on the stage's barrier.  Unlike a shared->tensor copy issued by
+        // the MMA thread, these stores run alongside the MMAs instead of in front
+        // of them.  Ring slot: released once both of its stages are in registers.
+        // Tensor-memory buffer s: written only after the MMAs of its previous
+        // use have completed (the stage's empty barrier).
         const uint32_t tq = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        const int local_tiles = (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
-                                static_cast<int>(gridDim.x);
-        const int total = local_tiles * k_stages;
-        for (int it = 0; it < total; ++it) {
-            const int s = it % kStages;
-            const uint32_t ph = (it / kStages) & 1;
-            if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
-            tc_fence_after();
-            const uint8_t* sfa = smem + kOffStages + s * kStageBytes + kATile + kBTile;
-            const uint8_t* sfb = sfa + kSfaTile;
-            // Column layout of one buffer: A scales of MMA kk at 4 kk + (row / 32);
-            // B scales of MMA kk at 16 + 8 kk + (row / 32), rows 128..255 at + 4.
-            // Lane i reads row i of each 512-byte atom: its 4 words are the 4 columns.
-            uint32_t ra[16], rb[32];
+        int s = 0, it = 0, pair = -1;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < k_stages; ++kb, ++it) {
+                if ((kb & 1) == 0) ++pair;
+                const int slot = pair & 1;
+                if (!mbar_try_wait(&sf_data[slot], (pair >> 1) & 1) &&
+                    !mbar_wait(&sf_data[slot], (pair >> 1) & 1, abort_flag, args.err, kErrWaitFull)) {
+                    ok = false;
+                    break;
+                }
+                // Slot layout: A atoms [8][512] of the two stages, then W row block
+                // 2n and 2n + 1, [8][512] each.  Column layout of one tensor-memory
+                // buffer: A scales of MMA kk at 4 kk + (row / 32); W scales of MMA
+                // kk at 16 + 8 kk + (row / 32), rows 128..255 at + 4.  Lane i reads
+                // row i of each 512-byte atom: its 4 words are the 4 columns.
+                const uint8_t* sfa = smem + kOffSf + slot * kSfSlot + (kb & 1) * 2048;
+                const uint8_t* sfb = smem + kOffSf + slot * kSfSlot + kSfaPair + (kb & 1) * 2048;
+                uint32_t ra[16], rb[32];
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-                const uint4 a = *reinterpret_cast<const uint4*>(sfa + kb * 512 + lane * 16);
-                const uint4 x = *reinterpret_cast<const uint4*>(sfb + kb * 512 + lane * 16);
-                const uint4 y = *reinterpret_cast<const uint4*>(sfb + kSfbTile / 2 + kb * 512 + lane * 16);
-                ra[4 * kb] = a.x; ra[4 * kb + 1] = a.y; ra[4 * kb + 2] = a.z; ra[4 * kb + 3] = a.w;
-                rb[8 * kb] = x.x; rb[8 * kb + 1] = x.y; rb[8 * kb + 2] = x.z; rb[8 * kb + 3] = x.w;
-                rb[8 * kb + 4] = y.x; rb[8 * kb + 5] = y.y; rb[8 * kb + 6] = y.z; rb[8 * kb + 7] = y.w;
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(sfa + q * 512 + lane * 16);
+                    const uint4 x = *reinterpret_cast<const uint4*>(sfb + q * 512 + lane * 16);
+                    const uint4 y = *reinterpret_cast<const uint4*>(sfb + 4096 + q * 512 + lane * 16);
+                    ra[4 * q] = a.x; ra[4 * q + 1] = a.y; ra[4 * q + 2] = a.z; ra[4 * q + 3] = a.w;
+                    rb[8 * q] = x.x; rb[8 * q + 1] = x.y; rb[8 * q + 2] = x.z; rb[8 * q + 3] = x.w;
+                    rb[8 * q + 4] = y.x; rb[8 * q + 5] = y.y; rb[8 * q + 6] = y.z; rb[8 * q + 7] = y.w;
+                }
+                if ((kb & 1) == 1 || kb == k_stages - 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sf_free[slot]);
+                }
+                if (it >= kStages && !mbar_try_wait(&empty[s], ph ^ 1) &&
+                    !mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t base = tq + kTmemSf0 + s * kTmemSfStride;
+                tmem_st_32x32b_x16(base, ra);
+                tmem_st_32x32b_x32(base + kTmemSfbOff, rb);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[s]);
+                if (++s == kStages) { s = 0; ph ^= 1u; }
             }
-            const uint32_t base = tq + kTmemSf0 + s * kTmemSfStride;
-            tmem_st_32x32b_x16(base, ra);
-            tmem_st_32x32b_x32(base + kTmemSfbOff, rb);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sf_full[s]);
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -463,8 +528,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
 }
 
 template <bool kOutF32>
-int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, const LinearArgs& a,
-                  cudaStream_t st) {
+int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, const CUtensorMap& tsa,
+                  const CUtensorMap& tsb, const LinearArgs& a, cudaStream_t st) {
     const uint32_t smem = kSmemBytes + 1024;
     auto kern = linear_kernel<kOutF32>;
     static std::atomic<uint64_t> smem_set{0};
@@ -472,7 +537,7 @@ int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMa
     const int tiles = a.m_tiles * a.n_tiles;
     const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
     const int grid = tiles < sms ? tiles : sms;
-    kern<<<grid, kThreads, smem, st>>>(ta, tb, ty, a);
+    kern<<<grid, kThreads, smem, st>>>(ta, tb, ty, tsa, tsb, a);
     return launch_status(cudaGetLastError());
 }
 
@@ -519,6 +584,13 @@ extern "C" int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const fl
     if (out_dtype == 0 &&
         !encode_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, N, M, ldy * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
         return SVDQ_ERR_CUDA;
+    // Scale atoms viewed as [row block][K / 64 atoms x 2 halves][256 bytes]: one box
+    // holds the 8 atoms of two stages (A: one row block, W: two).
+    CUtensorMap tsa, tsb;
+    const uint64_t halves = static_cast<uint64_t>(K / 64) * 2;
+    if (!encode_tmap_3d_u8(&tsa, a_sf, 256, halves, static_cast<uint64_t>(m_tiles), 256, halves * 256, 256, 16, 1) ||
+        !encode_tmap_3d_u8(&tsb, w_sf, 256, halves, static_cast<uint64_t>(N / 128), 256, halves * 256, 256, 16, 2))
+        return SVDQ_ERR_CUDA;
     LinearArgs a{};
     a.a_sf = a_sf;
     a.w_sf = w_sf;
@@ -539,5 +611,5 @@ extern "C" int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const fl
 
     a.err = err;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return out_dtype ? launch_linear<true>(ta, tb, ty, a, st) : launch_linear<false>(ta, tb, ty, a, st);
+    return out_dtype ? launch_linear<true>(ta, tb, ty, tsa, tsb, a, st) : launch_linear<false>(ta, tb, ty, tsa, tsb, a, st);
 }
