@@ -409,10 +409,12 @@ int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const Quan
     QuantArgs a = base;
     a.n_chunks = static_cast<int>(K / kBK);
     const int64_t m_tiles = (M + kBM - 1) / kBM;
-    // Split K so the grid covers every SM about once (one CTA fits per SM), up to a cluster of 4.
-    const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
-    int split = static_cast<int>((sms + m_tiles - 1) / m_tiles);
-    split = split < 1 ? 1 : (split > kMaxSplit ? kMaxSplit : split);
+    // Split K across up to 4 CTAs of a cluster, only as far as the grid still runs in one
+    // wave (one CTA fits per SM): a second wave costs more than the split saves (measured
+    // on B200: 12288 x 5120 takes 54 us unsplit, 60 us split in two or four).
+    const int64_t sms = device_sm_count() > 0 ? device_sm_count() : 148;
+    int64_t per_tile = sms / m_tiles;
+    int split = static_cast<int>(per_tile < 1 ? 1 : (per_tile > kMaxSplit ? kMaxSplit : per_tile));
     if (split > a.n_chunks) split = a.n_chunks;
     a.split = split;
     if (m_tiles > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
