@@ -28,7 +28,10 @@
 // (atomicMax; division by 2688 is monotonic, so the max of the quotients is
 // the quotient of the max), and lambda[1] counts finished strips; the last
 // strip writes the final s_g (1 when every maximum is 0) and lambda[1].  So the
-// call is two launches: a zeroing kernel and the reduction.
+// call is two launches: a zeroing kernel and the reduction.  The reduction is a
+// programmatic dependent of the zeroing kernel: its loads of X and W start while
+// the zeroing runs, and its consumers wait for it (griddepcontrol.wait) before
+// their first write to the outputs.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -64,6 +67,7 @@ struct CalibArgs {
 
 __global__ void __launch_bounds__(256)
 calib_zero_kernel(float* ax, float* aw, int64_t K, float* lambda, float* s_g) {
+    pdl_launch_dependents();                  // the reduction may start streaming at once
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < K; j += stride) {
         ax[j] = 0.0f;
@@ -167,6 +171,7 @@ calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
 
     if (a.n_units == 0) {
         // No rows selected and no weight: one CTA per strip forms lambda = 1.
+        pdl_wait();
         if (warp < kConsumerWarps) strip_lambda(a, g);
         return;
     }
@@ -213,6 +218,7 @@ calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     }
 
     // ---------------------------------------------------------------- consumers
+    pdl_wait();                               // the zeroing kernel's writes are complete and visible
     uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
     int64_t cur = -1;                          // (strip << 1) | matrix of the running maxima
     auto merge = [&](int64_t key) {
@@ -343,6 +349,15 @@ extern "C" int svdq_calib_lambda(const void* X, int64_t M, int64_t K, int64_t ld
     const uint32_t smem = kSmemBytes + 1024;
     static std::atomic<uint64_t> smem_set{0};
     if (!set_dynamic_smem_once(calib_stream_kernel, smem, smem_set)) return SVDQ_ERR_CUDA;
-    calib_stream_kernel<<<static_cast<unsigned>(grid), kThreads, smem, cs>>>(tx, tw, a);
-    return launch_status(cudaGetLastError());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = cs;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return launch_status(cudaLaunchKernelEx(&cfg, calib_stream_kernel, tx, tw, a));
 }

@@ -275,6 +275,18 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
     return r;
 }
 
+// Programmatic dependent launch.  The first kernel lets the next one in the
+// stream (launched with programmatic stream serialization) start early; that
+// kernel must wait for the first one's completion and memory before it touches
+// anything the first one writes.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Full cluster barrier (every thread of every CTA of the cluster).
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
