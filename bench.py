@@ -63,6 +63,23 @@ def workload_bytes(m, k, n, r, m_cal):
     return dict(quantize=quant, calib=calib, score=score)
 
 
+def max_over_ranks(ms: float, device=None) -> float:
+    """The job's time: the largest of the ranks' times (the default process group's
+    MAX all-reduce; the value itself when there is no group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return flops_per_rank * world / (ms_max * 1e-3) / 1e12
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling during the timed region."""
 
@@ -437,13 +454,10 @@ def run_gpu(args):
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
     step_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in step_evs]))
     kern_ms = per.mean(axis=0)       # calib, quantize, linear, score
-    t_local = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-    step_ms_max = float(t_local.item())
+    step_ms_max = max_over_ranks(step_ms, dev)
 
     flops = 2.0 * m * n * k
-    value = flops * world / (step_ms_max * 1e-3) / 1e12
+    value = whole_job_tflops(flops, world, step_ms_max)
     peaks = read_peaks()
     fp4_peak = peaks["bf16"] * FP4_PER_BF16
     lin_tflops = flops / (kern_ms[2] * 1e-3) / 1e12
@@ -497,10 +511,8 @@ def run_gpu(args):
     pipeline(args.steps, start_event=e0)
     e1.record(comp)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = flops * world / (float(e2e_ms.item()) * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    e2e_value = whole_job_tflops(flops, world, e2e_ms)
     rel = rel_host.tolist()
     # the graphs replay the same calls on the same data: same scores, bit for bit
     graph_matches_eager = bool(torch.equal(g_res[2].cpu(), rel_host) and torch.equal(s_res[2].cpu(), rel_host))
