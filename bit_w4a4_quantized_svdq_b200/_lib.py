@@ -52,6 +52,11 @@ SIGNATURES = {
     "svdq_residual": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_int,
                               c_void_p, c_void_p]),
     "svdq_device_error": (c_int, [c_void_p, POINTER(c_uint32)]),
+    "svdq_linear_score": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                  c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_int64, POINTER(SvdqSeg), c_int,
+                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_int64, c_int64, c_int64,
+                                  c_void_p]),
+    "svdq_linear_score_workspace_bytes": (c_size_t, [c_int]),
 }
 
 _lib = None

@@ -43,6 +43,8 @@
 // and the TMA unit spends a roughly fixed time per copy, so the scale atoms
 // travel in as few copies as possible (two per two stages instead of three per
 // stage).
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -76,7 +78,12 @@ constexpr uint32_t kOffLrA = kOffSf + 2 * kSfSlot;
 constexpr uint32_t kOffLrB = kOffLrA + kLrA;
 constexpr uint32_t kOffBar = kOffLrB + kLrB;
 constexpr uint32_t kOffBias = kOffBar + 256;          // 2 x 256 bf16 bias staging
-constexpr uint32_t kSmemBytes = kOffBias + 2 * kBN * 2;
+constexpr uint32_t kOffScore = kOffBias + 2 * kBN * 2;  // scoring: row sums, segment sums, segment rows
+constexpr uint32_t kScoreBytes = 2 * kBM * 16 + kMaxSegments * 16 + kMaxSegments * 8;
+constexpr uint32_t kSmemBytes = kOffScore + kScoreBytes;
+// Scoring: reference strips of 128 rows x 64 bf16 columns, three in the low-rank area.
+constexpr uint32_t kStripBytes = kBM * 128;
+static_assert(3 * kStripBytes <= kLrA + kLrB, "three reference strips fit the low-rank operand area");
 static_assert(kSmemBytes + 1024 <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
 
 // Tensor-memory columns: accumulator [0, 256), then one block-scale buffer per
@@ -101,7 +108,47 @@ struct LinearArgs {
     int m_tiles, n_tiles;
     int n_fastest;            // tile order: 1 = N fastest (the weight stays in L2), 0 = M fastest
     uint32_t* err;
+    // Scoring fused into the epilogue (bf16 output only; the reference comes by tensor map).
+    int write_y;              // 0: the output itself is not written
+    double* seg_part;         // [gridDim.x][n_seg][2] per-CTA (num, den) of every segment
+    double* num;
+    double* den;
+    double* rel;
+    SegTable segs;
 };
+
+// Scoring of eight output elements against the reference: the fp32 8-term
+// partial sums of the standalone scoring kernel (differences and squares in fp32,
+// in column order).
+__device__ __forceinline__ void score8(const uint32_t (&q)[4], const uint4& rv, float& n8, float& d8) {
+    const uint32_t wr[4] = {rv.x, rv.y, rv.z, rv.w};
+    n8 = 0.0f;
+    d8 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float r_lo = bf16_lo(wr[i]), r_hi = bf16_hi(wr[i]);
+        const float e_lo = __fsub_rn(bf16_lo(q[i]), r_lo);
+        const float e_hi = __fsub_rn(bf16_hi(q[i]), r_hi);
+        n8 = __fmaf_rn(e_lo, e_lo, n8);
+        n8 = __fmaf_rn(e_hi, e_hi, n8);
+        d8 = __fmaf_rn(r_lo, r_lo, d8);
+        d8 = __fmaf_rn(r_hi, r_hi, d8);
+    }
+}
+
+// hi + lo += x for an unevaluated fp32 pair: TwoSum (Knuth, TAOCP vol. 2,
+// 4.2.2; Moller 1965) makes s + e == hi + x exactly, the rounding errors gather
+// in lo.  A row's partials summed this way stay within a few units of 2^-48 of
+// their exact sum, so the one fp64 conversion per row replaces an fp64 addition
+// per partial (fp64 instructions slow the tensor-core main loop that shares the SM).
+__device__ __forceinline__ void pair_add(float& hi, float& lo, float x) {
+    const float s = __fadd_rn(hi, x);
+    const float bp = __fsub_rn(s, hi);
+    const float ap = __fsub_rn(s, bp);
+    const float e = __fadd_rn(__fsub_rn(hi, ap), __fsub_rn(x, bp));
+    hi = s;
+    lo = __fadd_rn(lo, e);
+}
 
 // Output tile -> (M block, N block).  The order decides what the CTAs working
 // at the same time share: walking the smaller operand's blocks fastest keeps
@@ -122,10 +169,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return l | (h << 16);
 }
 
-template <bool kOutF32>
+template <bool kOutF32, bool kScore>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-              const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_sfa,
+              const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_r,
+              const __grid_constant__ CUtensorMap tmap_sfa,
               const __grid_constant__ CUtensorMap tmap_sfb, LinearArgs args) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -137,7 +185,9 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     uint64_t* stage_free = lr_full + 1;                     // epilogue done with the staging area
     uint64_t* sf_data = stage_free + 1;                     // 2 slots: scale atoms landed
     uint64_t* sf_free = sf_data + 2;                        // 2 slots: the writers have read them
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_free + 2);
+    uint64_t* strip_full = sf_free + 2;                     // scoring: reference strips 0..3 landed
+    uint64_t* ring_free0 = strip_full + 4;                  // scoring: column half 0 done with slot 0
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring_free0 + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5;
@@ -161,6 +211,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         mbar_init(acc_empty, kEpiWarps);
         mbar_init(lr_full, 1);
         mbar_init(stage_free, kEpiWarps);
+        for (int i = 0; i < 4; ++i) mbar_init(&strip_full[i], 1);
+        mbar_init(ring_free0, kEpiWarps / 2);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -405,6 +457,191 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 if (++s == kStages) { s = 0; ph ^= 1u; }
             }
         }
+    } else if constexpr (kScore) {
+        // ------------------------------------------------------------ epilogue with scoring
+        // The plain epilogue's output path plus the tile's scoring against the
+        // reference output.  The reference comes in by TMA as strips of 128 rows x
+        // 64 columns (16 KB, 128-byte swizzle) into a three-slot ring over the
+        // low-rank operand area, which is free from "accumulator full" (this
+        // tile's low-rank MMAs have completed) until every epilogue warp has
+        // signalled stage_free.  Strips 0 and 2 (the first 64 columns of each
+        // column half) and strip 1 go out at "accumulator full"; strip 3 takes
+        // strip 0's slot once the four warps of column half 0 are done with it.
+        // Each lane scores its own row against its converted output values, so no
+        // value moves between lanes; the bf16 output, when written, is staged over
+        // the reference chunks it replaces (each lane rewrites exactly the bytes it
+        // read) and leaves by a TMA store.  The tile loop is left only at its top,
+        // through a barrier that ORs the abort flag over the epilogue warps, so a
+        // wait that runs out never strands the other warps at a barrier.
+        const int ew = warp - kEpiWarp0;                    // 0..7
+        const int quarter = warp & 3;                       // lane quarter this warp may access
+        const int half = ew >> 2;                           // column half of the tile
+        const int etid = ew * 32 + lane;                    // 0..255
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * (kBN / 2);
+        uint16_t* bias_s = reinterpret_cast<uint16_t*>(smem + kOffBias);
+        uint8_t* ring = smem + kOffLrA;
+        double2* rowsum = reinterpret_cast<double2*>(smem + kOffScore);   // [column half][tile row] (num, den)
+        double2* segsum = rowsum + 2 * kBM;                              // [segment] this CTA's (num, den)
+        int2* segrows = reinterpret_cast<int2*>(segsum + kMaxSegments);  // [segment] rows [begin, end)
+        const int n_seg = args.segs.n;
+        for (int i = etid; i < kMaxSegments; i += kEpiWarps * 32) {
+            segsum[i] = make_double2(0.0, 0.0);
+            if (i < n_seg) {
+                const int64_t b = args.segs.begin[i];
+                const int64_t e = b + (args.segs.prefix[i + 1] - args.segs.prefix[i]);
+                segrows[i] = make_int2(static_cast<int>(b), static_cast<int>(e));
+            }
+        }
+        if (etid == 0) prefetch_tmap(&tmap_r);
+        const int32_t M32 = static_cast<int32_t>(args.M);
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            int m_blk, n_blk;
+            tile_coords(args, tile, m_blk, n_blk);
+            const int32_t col0 = n_blk * kBN;
+            const int32_t m0 = m_blk * kBM;
+            uint16_t* bt = bias_s + (local & 1) * kBN;
+            bt[etid] = args.bias ? args.bias[col0 + etid] : static_cast<uint16_t>(0);
+            // bias staged, the previous tile's row sums consumed; leave together on abort
+            if (bar_sync_or<1, kEpiWarps * 32>(*abort_flag != 0u)) break;
+            bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, local & 1, abort_flag, args.err, kErrWaitMma));
+            tc_fence_after();
+            if (ok && etid == 0) {
+#pragma unroll
+                for (int i = 0; i < 3; ++i) {               // slots 0, 1, 2 <- strips 0, 2, 1
+                    const int strip = i == 0 ? 0 : 3 - i;
+                    mbar_arrive_expect_tx(&strip_full[strip], kStripBytes);
+                    tma_load_2d(ring + i * kStripBytes, &tmap_r, &strip_full[strip], col0 + strip * 64, m0);
+                }
+            }
+            const uint16_t* bw = bt + half * (kBN / 2);
+            // This warp's 128 accumulator columns as bf16 pairs (pk[h][j]: columns
+            // 64 h + 2 j, 64 h + 2 j + 1), the accumulator released after the last read.
+            // The first two 32-column pieces are read together, the last two one at
+            // a time (the first half's values are held meanwhile).
+            uint32_t pk[2][32];
+            if (ok) {
+                auto convert = [&](const uint32_t (&v)[32], int c) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const uint32_t bb = *reinterpret_cast<const uint32_t*>(bw + c * 32 + 2 * j);
+                        pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(fmaf(alpha, __uint_as_float(v[2 * j]), bf16_lo(bb)),
+                                                                   fmaf(alpha, __uint_as_float(v[2 * j + 1]), bf16_hi(bb)));
+                    }
+                };
+                {
+                    uint32_t v[2][32];
+                    tmem_ld_32x32b_x32(tbase, v[0]);
+                    tmem_ld_32x32b_x32(tbase + 32, v[1]);
+                    tmem_ld_wait();
+                    convert(v[0], 0);
+                    convert(v[1], 1);
+                }
+#pragma unroll
+                for (int c = 2; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase + c * 32, v);
+                    tmem_ld_wait();
+                    if (c == 3) {                   // the accumulator has been read: next tile's MMAs may start
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(acc_empty);
+                    }
+                    convert(v, c);
+                }
+            }
+            // The row's 8-column groups in column order: fp32 within a group, exact
+            // fp32 pairs across, fp64 from the row on.
+            float nh = 0.0f, nl = 0.0f, dh = 0.0f, dl = 0.0f;
+            const int32_t grow0 = m0 + quarter * 32;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                // half 0: strips 0 (slot 0), 1 (slot 2); half 1: strips 2 (slot 1), 3 (slot 0 again).
+                // Each strip has its own barrier, completed once per tile.
+                const int strip = 2 * half + h;
+                const int slot = h == 0 ? half : 2 - 2 * half;
+                if (ok)
+                    ok = __all_sync(0xffffffffu, mbar_wait(&strip_full[strip], local & 1, abort_flag, args.err, kErrWaitRef));
+                uint8_t* part = ring + slot * kStripBytes + quarter * 4096;
+                if (ok) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4* p = reinterpret_cast<uint4*>(part + lane * 128 + ((c ^ (lane & 7)) << 4));
+                        const uint4 rv = *p;
+                        const uint32_t q[4] = {pk[h][4 * c], pk[h][4 * c + 1], pk[h][4 * c + 2], pk[h][4 * c + 3]};
+                        float n8, d8;
+                        score8(q, rv, n8, d8);
+                        pair_add(nh, nl, n8);
+                        pair_add(dh, dl, d8);
+                        if (args.write_y) *p = make_uint4(q[0], q[1], q[2], q[3]);
+                    }
+                    if (args.write_y) {
+                        fence_async_shared();
+                        __syncwarp();
+                        if (lane == 0 && grow0 < M32) {     // boxes wholly below row M are skipped
+                            tma_store_2d(&tmap_y, part, col0 + half * (kBN / 2) + h * 64, grow0);
+                            bulk_commit_group();
+                        }
+                    }
+                }
+                if (h == 0 && half == 0) {
+                    // slot 0 is free for strip 3 once column half 0's four warps (and their stores) are done with it
+                    if (args.write_y && lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(ring_free0);
+                    if (ew == 0) {
+                        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ring_free0, local & 1, abort_flag, args.err, kErrWaitRef));
+                        if (ok && lane == 0) {
+                            mbar_arrive_expect_tx(&strip_full[3], kStripBytes);
+                            tma_load_2d(ring, &tmap_r, &strip_full[3], col0 + 3 * 64, m0);
+                        }
+                    }
+                }
+            }
+            if (args.write_y && lane == 0) bulk_wait_read_all();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stage_free);         // the ring is no longer read
+            rowsum[half * kBM + quarter * 32 + lane] =
+                grow0 + static_cast<int32_t>(lane) < M32
+                    ? make_double2(static_cast<double>(nh) + static_cast<double>(nl),
+                                   static_cast<double>(dh) + static_cast<double>(dl))
+                    : make_double2(0.0, 0.0);
+            asm volatile("bar.sync 1, %0;" :: "n"(kEpiWarps * 32) : "memory");
+            // The tile's rows of each segment (both halves of a row together, lanes
+            // striding over the rows, then a fixed shuffle tree); segment s belongs
+            // to epilogue warp s mod 8.
+            const int32_t m1 = min(m0 + kBM, M32);
+            for (int sg = ew; sg < n_seg; sg += kEpiWarps) {
+                const int2 se = segrows[sg];
+                const int lo = max(se.x, m0), hi = min(se.y, m1);
+                if (lo >= hi) continue;
+                double n = 0.0, d = 0.0;
+                for (int rr = lo - m0 + static_cast<int>(lane); rr < hi - m0; rr += 32) {
+                    const double2 a = rowsum[rr], b = rowsum[kBM + rr];
+                    n += a.x + b.x;
+                    d += a.y + b.y;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    n += __shfl_xor_sync(0xffffffffu, n, o);
+                    d += __shfl_xor_sync(0xffffffffu, d, o);
+                }
+                if (lane == 0) {
+                    segsum[sg].x += n;
+                    segsum[sg].y += d;
+                }
+            }
+        }
+        if (args.write_y) {
+            if (lane == 0) bulk_wait_all();          // bulk stores complete before the CTA exits
+            __syncwarp();
+        }
+        for (int sg = ew; sg < n_seg; sg += kEpiWarps) {
+            if (lane == 0) {
+                args.seg_part[(static_cast<int64_t>(blockIdx.x) * n_seg + sg) * 2] = segsum[sg].x;
+                args.seg_part[(static_cast<int64_t>(blockIdx.x) * n_seg + sg) * 2 + 1] = segsum[sg].y;
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         // Two warps per tensor-memory lane quarter, each owning 128 of the 256
@@ -525,36 +762,79 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if constexpr (kScore) {
+        {
+            // Every CTA's segment sums are written (the launch is cooperative, so all
+            // CTAs are resident and the grid barrier is safe); CTA 0 adds them in
+            // CTA order.
+            cooperative_groups::this_grid().sync();
+            if (blockIdx.x == 0 && warp == kEpiWarp0) {
+                const int n = args.segs.n;
+                for (int sg = 0; sg < n; ++sg) {
+                    double num = 0.0, den = 0.0;
+                    for (int c = lane; c < static_cast<int>(gridDim.x); c += 32) {
+                        num += __ldcg(args.seg_part + (static_cast<int64_t>(c) * n + sg) * 2);
+                        den += __ldcg(args.seg_part + (static_cast<int64_t>(c) * n + sg) * 2 + 1);
+                    }
+                    for (int o = 16; o > 0; o >>= 1) {
+                        num += __shfl_xor_sync(0xffffffffu, num, o);
+                        den += __shfl_xor_sync(0xffffffffu, den, o);
+                    }
+                    if (lane == 0) {
+                        args.num[sg] = num;
+                        args.den[sg] = den;
+                        double rel;
+                        if (den > 0.0) rel = sqrt(num / den);
+                        else rel = (num == 0.0) ? 0.0 : __longlong_as_double(0x7FF0000000000000LL);
+                        args.rel[sg] = rel;
+                    }
+                }
+            }
+        }
+    }
 }
 
-template <bool kOutF32>
-int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, const CUtensorMap& tsa,
-                  const CUtensorMap& tsb, const LinearArgs& a, cudaStream_t st) {
+// Persistent grid: one CTA per SM (at most one fits), never more CTAs than tiles.
+inline int linear_grid(int m_tiles, int n_tiles) {
+    const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
+    const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+    return static_cast<int>(tiles < sms ? tiles : sms);
+}
+
+template <bool kOutF32, bool kScore>
+int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, const CUtensorMap& tr,
+                  const CUtensorMap& tsa, const CUtensorMap& tsb, const LinearArgs& a, cudaStream_t st) {
+    static_assert(!(kOutF32 && kScore), "scoring is fused into the bf16 epilogue only");
     const uint32_t smem = kSmemBytes + 1024;
-    auto kern = linear_kernel<kOutF32>;
+    auto kern = linear_kernel<kOutF32, kScore>;
     static std::atomic<uint64_t> smem_set{0};
     if (!set_dynamic_smem_once(kern, smem, smem_set)) return SVDQ_ERR_CUDA;
     const int tiles = a.m_tiles * a.n_tiles;
-    const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
-    const int grid = tiles < sms ? tiles : sms;
-    kern<<<grid, kThreads, smem, st>>>(ta, tb, ty, tsa, tsb, a);
-    return launch_status(cudaGetLastError());
+    const int grid = linear_grid(a.m_tiles, a.n_tiles);
+    (void)tiles;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;      // scoring ends with a grid barrier
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = kScore ? 1 : 0;
+    return launch_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, tr, tsa, tsb, a));
 }
 
-}  // namespace
-}  // namespace svdq
-
-extern "C" int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g_act,
-                           const float* D, int r,
-                           const uint8_t* w_codes, const uint8_t* w_sf, const float* s_g_w,
-                           const void* up, const void* bias,
-                           void* Y, int64_t ldy, int out_dtype,
-                           int64_t M, int64_t N, int64_t K, void* stream) {
-    using namespace svdq;
-    if (a_codes == nullptr || a_sf == nullptr || w_codes == nullptr || w_sf == nullptr || Y == nullptr ||
-        s_g_act == nullptr || s_g_w == nullptr)
+// Validation, tensor maps and kernel arguments shared by the entry points.
+int linear_prepare(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g_act, const float* D, int r,
+                   const uint8_t* w_codes, const uint8_t* w_sf, const float* s_g_w, const void* up,
+                   const void* bias, void* Y, int64_t ldy, int out_dtype, int64_t M, int64_t N, int64_t K,
+                   CUtensorMap* ta, CUtensorMap* tb, CUtensorMap* ty, CUtensorMap* tsa, CUtensorMap* tsb,
+                   LinearArgs* a) {
+    if (a_codes == nullptr || a_sf == nullptr || w_codes == nullptr || w_sf == nullptr || s_g_act == nullptr ||
+        s_g_w == nullptr)
         return SVDQ_ERR_INVALID_ARG;
-    if (M < 1 || N < 1 || K < 1 || ldy < N) return SVDQ_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < 1 || (Y != nullptr && ldy < N)) return SVDQ_ERR_INVALID_ARG;
     if (out_dtype != 0 && out_dtype != 1) return SVDQ_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(s_g_act) & 3u) || (reinterpret_cast<uintptr_t>(s_g_w) & 3u))
         return SVDQ_ERR_MISALIGNED;
@@ -567,49 +847,111 @@ extern "C" int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const fl
     if (m_tiles * n_tiles > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
     if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(Y))
         return SVDQ_ERR_MISALIGNED;
-    if ((ldy * (out_dtype ? 4 : 2)) % 16 != 0) return SVDQ_ERR_MISALIGNED;
+    if (Y != nullptr && (ldy * (out_dtype ? 4 : 2)) % 16 != 0) return SVDQ_ERR_MISALIGNED;
     if (r > 0 && (!aligned16(D) || !aligned16(up))) return SVDQ_ERR_MISALIGNED;
     if (bias && !aligned16(bias)) return SVDQ_ERR_MISALIGNED;
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
     uint32_t* err = device_error_word();
     if (err == nullptr) return SVDQ_ERR_CUDA;
 
-    CUtensorMap ta, tb;
-    if (!encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a_codes, K / 2, M, K / 2, 128, 128,
+    if (!encode_tmap_2d(ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a_codes, K / 2, M, K / 2, 128, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_codes, K / 2, N, K / 2, 128, 256,
+        !encode_tmap_2d(tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_codes, K / 2, N, K / 2, 128, 256,
                         CU_TENSOR_MAP_SWIZZLE_128B))
         return SVDQ_ERR_CUDA;
-    CUtensorMap ty = ta;
-    if (out_dtype == 0 &&
-        !encode_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, N, M, ldy * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+    *ty = *ta;
+    if (out_dtype == 0 && Y != nullptr &&
+        !encode_tmap_2d(ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, N, M, ldy * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
         return SVDQ_ERR_CUDA;
     // Scale atoms viewed as [row block][K / 64 atoms x 2 halves][256 bytes]: one box
     // holds the 8 atoms of two stages (A: one row block, W: two).
-    CUtensorMap tsa, tsb;
     const uint64_t halves = static_cast<uint64_t>(K / 64) * 2;
-    if (!encode_tmap_3d_u8(&tsa, a_sf, 256, halves, static_cast<uint64_t>(m_tiles), 256, halves * 256, 256, 16, 1) ||
-        !encode_tmap_3d_u8(&tsb, w_sf, 256, halves, static_cast<uint64_t>(N / 128), 256, halves * 256, 256, 16, 2))
+    if (!encode_tmap_3d_u8(tsa, a_sf, 256, halves, static_cast<uint64_t>(m_tiles), 256, halves * 256, 256, 16, 1) ||
+        !encode_tmap_3d_u8(tsb, w_sf, 256, halves, static_cast<uint64_t>(N / 128), 256, halves * 256, 256, 16, 2))
         return SVDQ_ERR_CUDA;
-    LinearArgs a{};
-    a.a_sf = a_sf;
-    a.w_sf = w_sf;
-    a.D = D;
-    a.up = static_cast<const uint16_t*>(up);
-    a.bias = static_cast<const uint16_t*>(bias);
-    a.Y = Y;
-    a.ldy = ldy;
-    a.M = M;
-    a.N = N;
-    a.K = K;
-    a.s_g_act = s_g_act;
-    a.s_g_w = s_g_w;
-    a.r = r;
-    a.m_tiles = static_cast<int>(m_tiles);
-    a.n_tiles = static_cast<int>(n_tiles);
-    a.n_fastest = N <= M ? 1 : 0;                        // the weight is the smaller operand
+    *a = LinearArgs{};
+    a->a_sf = a_sf;
+    a->w_sf = w_sf;
+    a->D = D;
+    a->up = static_cast<const uint16_t*>(up);
+    a->bias = static_cast<const uint16_t*>(bias);
+    a->Y = Y;
+    a->ldy = ldy;
+    a->M = M;
+    a->N = N;
+    a->K = K;
+    a->s_g_act = s_g_act;
+    a->s_g_w = s_g_w;
+    a->r = r;
+    a->m_tiles = static_cast<int>(m_tiles);
+    a->n_tiles = static_cast<int>(n_tiles);
+    a->n_fastest = N <= M ? 1 : 0;                       // the weight is the smaller operand
+    a->err = err;
+    a->write_y = Y != nullptr ? 1 : 0;
+    return SVDQ_OK;
+}
 
-    a.err = err;
+}  // namespace
+}  // namespace svdq
+
+extern "C" int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g_act,
+                           const float* D, int r,
+                           const uint8_t* w_codes, const uint8_t* w_sf, const float* s_g_w,
+                           const void* up, const void* bias,
+                           void* Y, int64_t ldy, int out_dtype,
+                           int64_t M, int64_t N, int64_t K, void* stream) {
+    using namespace svdq;
+    if (Y == nullptr) return SVDQ_ERR_INVALID_ARG;
+    CUtensorMap ta, tb, ty, tsa, tsb;
+    LinearArgs a;
+    const int st0 = linear_prepare(a_codes, a_sf, s_g_act, D, r, w_codes, w_sf, s_g_w, up, bias, Y, ldy, out_dtype,
+                                   M, N, K, &ta, &tb, &ty, &tsa, &tsb, &a);
+    if (st0 != SVDQ_OK) return st0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return out_dtype ? launch_linear<true>(ta, tb, ty, tsa, tsb, a, st) : launch_linear<false>(ta, tb, ty, tsa, tsb, a, st);
+    return out_dtype ? launch_linear<true, false>(ta, tb, ty, ta, tsa, tsb, a, st)
+                     : launch_linear<false, false>(ta, tb, ty, ta, tsa, tsb, a, st);
+}
+
+extern "C" size_t svdq_linear_score_workspace_bytes(int n_seg) {
+    if (n_seg < 1 || n_seg > svdq::kMaxSegments) return 0;
+    return static_cast<size_t>(1024) * static_cast<size_t>(n_seg) * 2 * sizeof(double);
+}
+
+extern "C" int svdq_linear_score(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g_act,
+                                 const float* D, int r,
+                                 const uint8_t* w_codes, const uint8_t* w_sf, const float* s_g_w,
+                                 const void* up, const void* bias,
+                                 void* Y, int64_t ldy,
+                                 const void* Yref, int64_t ldr,
+                                 const svdq_seg* segs, int n_seg,
+                                 double* num, double* den, double* rel,
+                                 void* workspace, size_t workspace_bytes,
+                                 int64_t M, int64_t N, int64_t K, void* stream) {
+    using namespace svdq;
+    if (Yref == nullptr || num == nullptr || den == nullptr || rel == nullptr || workspace == nullptr)
+        return SVDQ_ERR_INVALID_ARG;
+    if (segs == nullptr || n_seg < 1 || n_seg > kMaxSegments || ldr < N) return SVDQ_ERR_INVALID_ARG;
+    if (!aligned16(Yref) || (ldr * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(workspace) & 7u) ||
+        (reinterpret_cast<uintptr_t>(num) & 7u) || (reinterpret_cast<uintptr_t>(den) & 7u) ||
+        (reinterpret_cast<uintptr_t>(rel) & 7u))
+        return SVDQ_ERR_MISALIGNED;
+    CUtensorMap ta, tb, ty, tsa, tsb;
+    LinearArgs a;
+    const int st0 = linear_prepare(a_codes, a_sf, s_g_act, D, r, w_codes, w_sf, s_g_w, up, bias, Y, ldy, 0, M, N,
+                                   K, &ta, &tb, &ty, &tsa, &tsb, &a);
+    if (st0 != SVDQ_OK) return st0;
+    const int grid = linear_grid(a.m_tiles, a.n_tiles);
+    if (workspace_bytes < static_cast<size_t>(grid) * n_seg * 2 * sizeof(double)) return SVDQ_ERR_INVALID_ARG;
+    const int sst = make_seg_table(segs, n_seg, M, &a.segs);
+    if (sst != SVDQ_OK) return sst;
+    // The reference in strips of 64 columns x 128 rows, 128-byte swizzle (rows past M read as zeros).
+    CUtensorMap tr;
+    if (!encode_tmap_2d(&tr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Yref, N, M, ldr * 2, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return SVDQ_ERR_CUDA;
+    a.seg_part = static_cast<double*>(workspace);
+    a.num = num;
+    a.den = den;
+    a.rel = rel;
+    return launch_linear<false, true>(ta, tb, ty, tr, tsa, tsb, a, static_cast<cudaStream_t>(stream));
 }

@@ -107,6 +107,45 @@ def svdq_linear(a_codes: torch.Tensor, a_sf: torch.Tensor, s_g_act: torch.Tensor
     return out
 
 
+def linear_score_workspace_bytes(n_seg: int) -> int:
+    return int(_lib.load().svdq_linear_score_workspace_bytes(int(n_seg)))
+
+
+def svdq_linear_score(a_codes: torch.Tensor, a_sf: torch.Tensor, s_g_act: torch.Tensor, d: Optional[torch.Tensor],
+                      w_codes: torch.Tensor, w_sf: torch.Tensor, s_g_w: torch.Tensor, up: Optional[torch.Tensor],
+                      bias: Optional[torch.Tensor], yref: torch.Tensor, segs: Sequence[Tuple[int, int]],
+                      out: Optional[torch.Tensor] = None, write_out: bool = True,
+                      workspace: Optional[torch.Tensor] = None, stream=None):
+    """The bf16 linear and, in the same kernel, its per-segment (num, den, rel) against
+    yref.  Returns (out or None, num, den, rel); write_out=False skips the output."""
+    lib = _lib.load()
+    _check_bf16(yref, "yref")
+    m, kh = a_codes.shape
+    n = w_codes.shape[0]
+    k = 2 * kh
+    r = 0 if d is None else int(d.shape[1])
+    if tuple(yref.shape) != (m, n):
+        raise ValueError(f"yref must be [{m}, {n}], got {tuple(yref.shape)}")
+    dev = a_codes.device
+    if write_out and out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    if not write_out:
+        out = None
+    ldy = _row_stride(out, "out") if out is not None else n
+    arr, n_seg = _lib.seg_array(segs)
+    num = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    den = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    rel = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    if workspace is None:
+        workspace = torch.empty(linear_score_workspace_bytes(n_seg), dtype=torch.uint8, device=dev)
+    _lib.check("svdq_linear_score", lib.svdq_linear_score(
+        _ptr(a_codes), _ptr(a_sf), _ptr(s_g_act), _ptr(d), r, _ptr(w_codes), _ptr(w_sf), _ptr(s_g_w),
+        _ptr(up), _ptr(bias), _ptr(out), ldy, _ptr(yref), _row_stride(yref, "yref"), arr, n_seg,
+        _ptr(num), _ptr(den), _ptr(rel), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        m, n, k, _stream(stream)))
+    return out, num, den, rel
+
+
 def score_workspace_bytes(segs: Sequence[Tuple[int, int]], n: int) -> int:
     arr, n_seg = _lib.seg_array(segs)
     return int(_lib.load().svdq_score_workspace_bytes(arr, n_seg, n))

@@ -173,6 +173,48 @@ int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g_ac
                 int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
+ * svdq_linear_score -- svdq_linear (bf16 output) and, in the same kernel, the
+ * scoring of that output against a reference ("MiniMax-H3 NVFP4 -- what the
+ * smoothing scale should be calibrated on", section "The metric that picks the
+ * winner also hides the cost": rel-L2 against the bf16 layer, per row set).
+ * For each segment s = [begin, end):
+ *
+ *   num[s] = sum over its rows, all N columns, of (Yq - Yref)^2
+ *   den[s] = sum of Yref^2,   rel[s] = sqrt(num / den)
+ *
+ * where Yq is the bf16 value svdq_linear writes.  Each group of 8 consecutive
+ * columns is summed in fp32 (the arithmetic of svdq_score_lambda); a row's
+ * groups within each 128-column half of a 256-column tile are added as an
+ * exact fp32 pair (TwoSum: the pair is within a few units of 2^-48 of the
+ * exact sum of its groups), converted to fp64 once, and everything beyond is
+ * fp64 in a fixed order: deterministic, and equal to svdq_score_lambda on the
+ * written output up to rounding of relative size ~1e-13.  rel is 0 when num
+ * is 0 and den is 0, +inf when only den is 0.
+ *
+ * Arguments as svdq_linear, plus: Y may be NULL (the output is not written; the
+ * scores still are, and the call is faster).  Yref: device bf16 [M, N], 16-byte
+ * aligned, row stride ldr >= N (ldr * 2 a multiple of 16); it is read by TMA in
+ * 128-row x 64-column boxes.  segs: host array of n_seg (1..64) row ranges within [0, M]
+ * (they may overlap).  num, den, rel: device fp64 [n_seg].  workspace: device
+ * memory, 8-byte aligned, of at least svdq_linear_score_workspace_bytes(n_seg)
+ * bytes, owned by the caller; its contents are overwritten.  Calls that share a
+ * workspace must not overlap.  The launch is cooperative (all CTAs resident).
+ */
+int svdq_linear_score(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g_act,
+                      const float* D, int r,
+                      const uint8_t* w_codes, const uint8_t* w_sf, const float* s_g_w,
+                      const void* up, const void* bias,
+                      void* Y, int64_t ldy,
+                      const void* Yref, int64_t ldr,
+                      const svdq_seg* segs, int n_seg,
+                      double* num, double* den, double* rel,
+                      void* workspace, size_t workspace_bytes,
+                      int64_t M, int64_t N, int64_t K, void* stream);
+
+/* Workspace bytes svdq_linear_score needs for n_seg segments (0 if n_seg is out of range). */
+size_t svdq_linear_score_workspace_bytes(int n_seg);
+
+/*
  * svdq_score_workspace_bytes -- device workspace svdq_score_lambda needs for
  * these segments and N columns (a multiple of 256 bytes, at least 256).
  */
