@@ -309,7 +309,19 @@ def all_configs(P, S, dev, fp4_peak, hbm_peak, flush, flush_read):
         r["score"] = {"ms": t, "GB/s": by / (t * 1e-3) / 1e9, "frac_hbm": by / (t * 1e-3) / 1e9 / hbm_peak}
         _, _, rel = P.svdq_score_lambda(y, yref, segs_mod, workspace=ws)
         r["rel_l2_vs_bf16"] = dict(zip([sg.name for sg in L.segments], rel.cpu().tolist()))
-        del x, w, bias, cal, lin, q, y, yref, ws
+        # the scoring fused into the linear's epilogue, with and without writing the output
+        wf = torch.empty(P.linear_score_workspace_bytes(len(segs_mod)), dtype=torch.uint8, device=dev)
+        la = (q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf, lin.s_g_w, lin.up, lin.bias)
+        sep = r["linear"]["ms"] + r["score"]["ms"]
+        for key, write in (("linear_score", True), ("linear_score_only", False)):
+            t = _graph_ms(lambda: P.svdq_linear_score(*la, yref=yref, segs=segs_mod, out=y if write else None,
+                                                      write_out=write, workspace=wf), flush, flush_read)
+            _, _, _, rel_f = P.svdq_linear_score(*la, yref=yref, segs=segs_mod, out=y if write else None,
+                                                 write_out=write, workspace=wf)
+            same = bool(np.allclose(rel_f.cpu().numpy(), rel.cpu().numpy(), rtol=1e-9, atol=0))
+            r[key] = {"ms": t, "TFLOP/s": fl / (t * 1e-3) / 1e12, "linear_plus_score_ms": sep,
+                      "speedup_vs_separate": sep / t, "rel_matches_separate": same}
+        del x, w, bias, cal, lin, q, y, yref, ws, wf
         torch.cuda.empty_cache()
         return r
 
