@@ -49,6 +49,13 @@ Readings where the pages are silent (each repeated in the design doc):
      the down factor is stored with lambda folded in (L1s = diag(1/lambda) L1)
      as a [r, K] "down" weight and L2^T as an [N, r] "up" weight, both bf16.
   R10 rel-L2 of a segment is ||Yq - Yref||_F / ||Yref||_F over its rows.
+  R11 The bits-lost proxy uses per-modality channel absmax statistics: the
+      channel's absmax is RN32(ax_j * (1/lambda_j)) (the smoothed statistic
+      the kernel's group scale sees; max over rows commutes with the monotone
+      rounded product), the group absmax is the largest of its 16 channels,
+      and the figure for a modality is the mean of log2(group / channel) over
+      the channels whose smoothed absmax is > 0 (a zero channel has nothing to
+      lose); 0 if none counts.
 
 Pins (``tests/test_oracle_pins.py``) hold every function to something other
 than itself: independent float-format rounding, torch's float8 conversion,
@@ -395,6 +402,36 @@ def score(yq_bits: np.ndarray, yref_bits: np.ndarray, segments: Sequence[Tuple[i
         den.append(d_s)
         rel.append(math.sqrt(n_s / d_s) if d_s > 0 else (0.0 if n_s == 0 else math.inf))
     return np.array(num), np.array(den), np.array(rel)
+
+
+def bits_lost(ax: np.ndarray, inv_lam: Optional[np.ndarray]) -> np.ndarray:
+    """Mean bits a channel loses to its group's shared scale, per candidate and modality.
+
+    "MiniMax-H3 NVFP4 -- what the smoothing scale should be calibrated on",
+    section "Why": 16 consecutive input channels share one FP8 scale set by the
+    group's absmax, so a channel whose own absmax is below the group's loses
+    log2(group_absmax / channel_absmax) bits; lambda reshapes that profile
+    because the kernel sees X / lambda (statistics only, no GEMM).  Reading R11.
+
+    ax: fp32 [n_mod, K] per-modality channel absmax of X (``calib`` over the
+    modality's rows); inv_lam: fp32 [n_cand, K] candidate 1/lambda rows, or None
+    for lambda = 1.  Returns fp64 [n_cand, n_mod].
+    """
+    ax = np.asarray(ax, dtype=np.float32)
+    ax = ax.reshape(1, -1) if ax.ndim == 1 else ax
+    n_mod, k = ax.shape
+    assert k % BLOCK == 0
+    il = np.ones((1, k), np.float32) if inv_lam is None else np.asarray(inv_lam, np.float32).reshape(-1, k)
+    out = np.zeros((il.shape[0], n_mod), dtype=np.float64)
+    for c in range(il.shape[0]):
+        for m in range(n_mod):
+            chan = (ax[m] * il[c]).astype(np.float32)                  # RN32 product (R5)
+            group = np.repeat(chan.reshape(-1, BLOCK).max(axis=1), BLOCK)
+            counted = chan > 0
+            if counted.any():
+                ratio = group[counted].astype(np.float64) / chan[counted].astype(np.float64)
+                out[c, m] = float(np.mean(np.log2(ratio)))
+    return out
 
 
 # ----------------------------------------------------------------------------
