@@ -6,8 +6,8 @@ call fails with ImportError if it has not been built
 (``python -m bit_w4a4_quantized_svdq_b200.build``): there is no fallback.
 """
 from . import _lib
-from .ops import (linear_score_workspace_bytes, score_workspace_bytes, sf_bytes, svdq_calib_lambda,
-                  svdq_device_error, svdq_linear, svdq_linear_score, svdq_quantize_act, svdq_residual,
+from .ops import (linear_score_workspace_bytes, score_workspace_bytes, sf_bytes, svdq_bits_lost,
+                  svdq_calib_lambda, svdq_device_error, svdq_linear, svdq_linear_score, svdq_quantize_act, svdq_residual,
                   svdq_score_lambda, svdq_score_lambda_static)
 from .layer import SVDQW4A4Linear, lowrank_factors_device
 
@@ -19,7 +19,7 @@ def load():
 
 __all__ = [
     "svdq_calib_lambda", "svdq_quantize_act", "svdq_linear", "svdq_linear_score", "svdq_score_lambda",
-    "svdq_score_lambda_static", "linear_score_workspace_bytes",
+    "svdq_score_lambda_static", "linear_score_workspace_bytes", "svdq_bits_lost",
     "svdq_residual", "svdq_device_error", "sf_bytes", "score_workspace_bytes", "SVDQW4A4Linear",
     "lowrank_factors_device", "load",
 ]

@@ -207,6 +207,28 @@ def svdq_residual(w: torch.Tensor, lam: Optional[torch.Tensor], down: Optional[t
     return out
 
 
+def svdq_bits_lost(amax_x: torch.Tensor, inv_lambda: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Mean bits lost to the NVFP4 group scale, fp64 [n_cand, n_mod].
+
+    amax_x: fp32 [n_mod, K] (or [K]) per-modality channel absmax; inv_lambda:
+    fp32 [n_cand, K] (or [K]) candidate 1/lambda rows, None for lambda = 1."""
+    lib = _lib.load()
+    ax = amax_x if amax_x.dim() == 2 else amax_x.view(1, -1)
+    if ax.dtype != torch.float32 or not ax.is_cuda or ax.stride(1) != 1:
+        raise ValueError("amax_x must be a CUDA float32 tensor with unit column stride")
+    n_mod, k = ax.shape
+    il, n_cand, ld_lam = None, 1, k
+    if inv_lambda is not None:
+        il = inv_lambda if inv_lambda.dim() == 2 else inv_lambda.view(1, -1)
+        if il.dtype != torch.float32 or not il.is_cuda or il.stride(1) != 1 or il.shape[1] != k:
+            raise ValueError("inv_lambda must be a CUDA float32 [n_cand, K] tensor with unit column stride")
+        n_cand, ld_lam = il.shape[0], il.stride(0)
+    bits = torch.empty((n_cand, n_mod), dtype=torch.float64, device=ax.device)
+    _lib.check("svdq_bits_lost", lib.svdq_bits_lost(
+        _ptr(ax), ax.stride(0), n_mod, _ptr(il), ld_lam, n_cand, k, _ptr(bits), _stream(stream)))
+    return bits
+
+
 def svdq_device_error(stream=None) -> int:
     """Synchronise and return (then clear) the device error word; 0 = no timeout."""
     code = c_uint32(0)

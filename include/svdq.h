@@ -281,6 +281,29 @@ int svdq_residual(const void* W, int64_t N, int64_t K, int64_t ldw, const float*
                   const void* down, const void* up, int r, void* R, void* stream);
 
 /*
+ * svdq_bits_lost -- the bits-lost proxy ("MiniMax-H3 NVFP4 -- what the smoothing
+ * scale should be calibrated on", section "Why"): 16 consecutive input channels
+ * share one FP8 scale set by the group's absmax, so a channel whose absmax is
+ * below its group's loses log2(group_absmax / channel_absmax) bits; lambda
+ * reshapes that profile because the kernel sees X / lambda.  Statistics only:
+ *
+ *   c_j        = RN32(amax_x[m, j] * inv_lambda[c, j])    (amax_x alone if inv_lambda is NULL)
+ *   g_j        = max of c over the 16-channel group of j
+ *   bits[c, m] = mean over the channels j with c_j > 0 of log2(g_j / c_j)   (fp64; 0 if none)
+ *
+ * amax_x: device fp32 [n_mod, K], row stride ld_amax >= K, one row per modality:
+ * non-negative channel absmax of X over that modality's rows (the amax_x output
+ * of svdq_calib_lambda called on those rows).  inv_lambda: device fp32
+ * [n_cand, K], row stride ld_lam >= K, one candidate 1/lambda per row (as
+ * svdq_calib_lambda returns it), or NULL for lambda = 1 (then n_cand must be 1).
+ * bits: device fp64 [n_cand, n_mod], row-major, written.  K % 16 == 0, K >= 16;
+ * 1 <= n_mod, n_cand <= 65535.  Deterministic (fixed reduction order).
+ * Asynchronous on `stream`; arguments are checked before anything is launched.
+ */
+int svdq_bits_lost(const float* amax_x, int64_t ld_amax, int n_mod, const float* inv_lambda, int64_t ld_lam,
+                   int n_cand, int64_t K, double* bits, void* stream);
+
+/*
  * svdq_device_error -- synchronise `stream`, then read and clear the current
  * device's error word.  *code receives 0 when no bounded wait ran out since
  * the last call, otherwise a nonzero code naming the wait.  Returns

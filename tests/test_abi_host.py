@@ -130,3 +130,14 @@ def test_score_and_residual_reject_bad_arguments():
 def test_device_error_requires_output_pointer():
     lib = _lib.load()
     assert lib.svdq_device_error(None, None) == _lib.SVDQ_ERR_INVALID_ARG
+
+
+def test_bits_lost_rejects_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(FAKE)
+    assert lib.svdq_bits_lost(None, 64, 1, None, 64, 1, 64, p, None) == _lib.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_bits_lost(p, 64, 1, None, 64, 1, 40, p, None) == _lib.SVDQ_ERR_INVALID_ARG    # K % 16
+    assert lib.svdq_bits_lost(p, 32, 1, None, 64, 1, 64, p, None) == _lib.SVDQ_ERR_INVALID_ARG    # ld < K
+    assert lib.svdq_bits_lost(p, 64, 1, None, 64, 2, 64, p, None) == _lib.SVDQ_ERR_INVALID_ARG    # no lambda, 2 candidates
+    assert lib.svdq_bits_lost(p, 64, 0, p, 64, 1, 64, p, None) == _lib.SVDQ_ERR_INVALID_ARG       # no modality
+    assert lib.svdq_bits_lost(p, 64, 1, p, 64, 1, 64, ctypes.c_void_p(FAKE + 4), None) == _lib.SVDQ_ERR_MISALIGNED
