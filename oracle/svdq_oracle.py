@@ -56,6 +56,17 @@ Readings where the pages are silent (each repeated in the design doc):
       and the figure for a modality is the mean of log2(group / channel) over
       the channels whose smoothed absmax is > 0 (a zero channel has nothing to
       lose); 0 if none counts.
+  R12 Candidate smoothing scales over a migration-strength grid:
+      lambda_j(alpha) = ax_j^alpha / aw_j^(1 - alpha) (R8 is alpha = 0.5),
+      evaluated as RN32(2^(alpha log2 ax_j - (1 - alpha) log2 aw_j)) in fp64
+      from the fp32 alpha; 1 where either absmax is 0; 1/lambda and s_g per
+      candidate as in R5 and R3.
+  R13 The grid: 39 evenly spaced alpha in [0.05, 0.95] (the pages give only
+      the count of candidates).
+  R14 Selection: the candidate with the smallest sum over modalities of
+      w_m * rel_m (weights given by the caller: rows-proportional weights
+      reproduce the uniform-rows column, equal weights the per-modality view);
+      ties go to the lower index.
 
 Pins (``tests/test_oracle_pins.py``) hold every function to something other
 than itself: independent float-format rounding, torch's float8 conversion,
@@ -432,6 +443,43 @@ def bits_lost(ax: np.ndarray, inv_lam: Optional[np.ndarray]) -> np.ndarray:
                 ratio = group[counted].astype(np.float64) / chan[counted].astype(np.float64)
                 out[c, m] = float(np.mean(np.log2(ratio)))
     return out
+
+
+def alpha_grid(n: int = 39, lo: float = 0.05, hi: float = 0.95) -> np.ndarray:
+    """The migration-strength grid of R13 as fp32 values."""
+    return np.linspace(lo, hi, n).astype(np.float32)
+
+
+def lambda_grid(ax: np.ndarray, aw: np.ndarray, alphas: np.ndarray):
+    """Candidate lambda, 1/lambda and s_g for every alpha (R12).
+
+    "MiniMax-H3 NVFP4 -- what the smoothing scale should be calibrated on",
+    section "Calibration": a grid of lambda candidates built from absmax
+    statistics.  Returns (lam [n, K] fp32, inv_lam [n, K] fp32, s_g [n] fp32).
+    """
+    ax = np.asarray(ax, np.float32)
+    aw = np.asarray(aw, np.float32)
+    ok = (ax > 0) & (aw > 0)
+    lx = np.log2(np.where(ok, ax, np.float32(1)).astype(np.float64))
+    lw = np.log2(np.where(ok, aw, np.float32(1)).astype(np.float64))
+    lams, invs, sgs = [], [], []
+    for a in np.asarray(alphas, np.float32):
+        a64 = float(a)
+        t = a64 * lx - (1.0 - a64) * lw
+        lam = np.where(ok, np.exp2(t).astype(np.float32), np.float32(1.0)).astype(np.float32)
+        inv = (np.float32(1.0) / lam).astype(np.float32)
+        top = np.float32((ax * inv).astype(np.float32).max()) if ax.size else np.float32(0)
+        s_g = np.float32(top / np.float32(E2M1_MAX * E4M3_MAX)) if top > 0 else np.float32(1.0)
+        lams.append(lam)
+        invs.append(inv)
+        sgs.append(s_g)
+    return np.array(lams), np.array(invs), np.array(sgs, dtype=np.float32)
+
+
+def select_candidate(rel: np.ndarray, weights: np.ndarray) -> int:
+    """Index of the candidate with the smallest weighted sum of per-modality rel-L2 (R14)."""
+    total = np.asarray(rel, np.float64) @ np.asarray(weights, np.float64)
+    return int(np.argmin(total))
 
 
 # ----------------------------------------------------------------------------
