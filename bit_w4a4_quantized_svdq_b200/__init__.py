@@ -7,9 +7,9 @@ call fails with ImportError if it has not been built
 """
 from . import _lib
 from .ops import (linear_score_workspace_bytes, score_workspace_bytes, sf_bytes, svdq_bits_lost,
-                  svdq_calib_lambda, svdq_device_error, svdq_linear, svdq_linear_score, svdq_quantize_act, svdq_residual,
+                  svdq_calib_lambda, svdq_device_error, svdq_lambda_grid, svdq_linear, svdq_linear_score, svdq_quantize_act, svdq_residual,
                   svdq_score_lambda, svdq_score_lambda_static)
-from .layer import SVDQW4A4Linear, lowrank_factors_device
+from .layer import SVDQW4A4Linear, alpha_grid, lowrank_factors_device, search_lambda
 
 
 def load():
@@ -19,7 +19,7 @@ def load():
 
 __all__ = [
     "svdq_calib_lambda", "svdq_quantize_act", "svdq_linear", "svdq_linear_score", "svdq_score_lambda",
-    "svdq_score_lambda_static", "linear_score_workspace_bytes", "svdq_bits_lost",
+    "svdq_score_lambda_static", "linear_score_workspace_bytes", "svdq_bits_lost", "svdq_lambda_grid",
     "svdq_residual", "svdq_device_error", "sf_bytes", "score_workspace_bytes", "SVDQW4A4Linear",
-    "lowrank_factors_device", "load",
+    "lowrank_factors_device", "alpha_grid", "search_lambda", "load",
 ]

@@ -58,6 +58,8 @@ SIGNATURES = {
                                   c_void_p]),
     "svdq_linear_score_workspace_bytes": (c_size_t, [c_int]),
     "svdq_bits_lost": (c_int, [c_void_p, c_int64, c_int, c_void_p, c_int64, c_int, c_int64, c_void_p, c_void_p]),
+    "svdq_lambda_grid": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                 c_void_p]),
 }
 
 _lib = None

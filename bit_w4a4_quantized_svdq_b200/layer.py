@@ -17,6 +17,7 @@ from __future__ import annotations
 
 from typing import Optional, Sequence, Tuple
 
+import numpy as np
 import torch
 
 from . import ops
@@ -100,3 +101,64 @@ class SVDQW4A4Linear:
         return y.reshape(*lead, self.out_features)
 
     __call__ = forward
+
+
+def alpha_grid(n: int = 39, lo: float = 0.05, hi: float = 0.95) -> torch.Tensor:
+    """Migration strengths of the lambda search: n evenly spaced values in [lo, hi] (fp32, host)."""
+    return torch.from_numpy(np.linspace(lo, hi, n).astype(np.float32))
+
+
+def search_lambda(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.Tensor], rank: int,
+                  calib_segs: Optional[Sequence[Tuple[int, int]]], modality_segs: Sequence[Tuple[int, int]],
+                  weights: Optional[Sequence[float]] = None, alphas: Optional[torch.Tensor] = None,
+                  yref: Optional[torch.Tensor] = None, seed: int = 0) -> dict:
+    """Pick the smoothing scale from a grid of candidates by per-modality rel-L2 of the W4A4 output.
+
+    "MiniMax-H3 NVFP4 -- what the smoothing scale should be calibrated on":
+    section "Calibration" (lambda picked from a grid of candidates built from
+    absmax statistics under a modality mask) and section "The metric that picks
+    the winner also hides the cost" (rank candidates by rel-L2 against the bf16
+    layer on rows of each modality, not only on proportional rows).
+
+    Candidates lambda(alpha) = ax^alpha / aw^(1 - alpha) from the absmax of X over
+    ``calib_segs`` and of W (``svdq_lambda_grid``); each is converted (rank-r
+    factors, residual, NVFP4 weight), the activations quantised, and the linear
+    scored against ``yref`` (default: the bf16 layer, X W^T + b by a library GEMM)
+    on every modality in the GEMM's epilogue without writing its output
+    (``svdq_linear_score``).  The winner has the smallest sum of weights[m] *
+    rel[m] (equal weights by default; ties to the lower index).  The bits-lost
+    proxy of every candidate on every modality's statistics comes along
+    (``svdq_bits_lost``, one launch).
+
+    Returns dict(alpha [n] host fp32, lam / inv_lam [n, K], s_g [n], rel [n, n_mod]
+    and bits [n, n_mod] (device fp64), best (int), layer (the best candidate converted)).
+    """
+    dev = x.device
+    alphas = alpha_grid() if alphas is None else alphas.to(torch.float32).cpu()
+    n_mod = len(modality_segs)
+    wts = torch.ones(n_mod, dtype=torch.float64) if weights is None else torch.tensor(weights, dtype=torch.float64)
+    if wts.numel() != n_mod:
+        raise ValueError("one weight per modality")
+    cal = ops.svdq_calib_lambda(x, calib_segs, w)
+    grid = ops.svdq_lambda_grid(cal["amax_x"], cal["amax_w"], alphas.to(dev))
+    ax_mod = torch.stack([ops.svdq_calib_lambda(x, [seg], None)["amax_x"] for seg in modality_segs])
+    bits = ops.svdq_bits_lost(ax_mod, grid["inv_lam"])
+    if yref is None:
+        xb, wb = x.view(torch.bfloat16), w.view(torch.bfloat16)
+        yref = xb @ wb.t()
+        if bias is not None:
+            yref = yref + bias.view(torch.bfloat16)
+    ws = torch.empty(ops.linear_score_workspace_bytes(n_mod), dtype=torch.uint8, device=dev)
+    rel = torch.empty((alphas.numel(), n_mod), dtype=torch.float64, device=dev)
+    for c in range(alphas.numel()):
+        cand = dict(lam=grid["lam"][c], inv_lam=grid["inv_lam"][c], s_g=grid["s_g"][c:c + 1])
+        layer = SVDQW4A4Linear.convert(w, bias, cand, rank, seed=seed)
+        q = layer.quantize(x)
+        _, _, _, rel[c] = ops.svdq_linear_score(q["codes"], q["sf"], layer.s_g_act, q["d"], layer.w_codes,
+                                                layer.w_sf, layer.s_g_w, layer.up, layer.bias, yref, modality_segs,
+                                                write_out=False, workspace=ws)
+    total = rel.cpu() @ wts
+    best = int(torch.argmin(total))
+    cand = dict(lam=grid["lam"][best], inv_lam=grid["inv_lam"][best], s_g=grid["s_g"][best:best + 1])
+    return dict(alpha=alphas, lam=grid["lam"], inv_lam=grid["inv_lam"], s_g=grid["s_g"], rel=rel, bits=bits,
+                best=best, layer=SVDQW4A4Linear.convert(w, bias, cand, rank, seed=seed))

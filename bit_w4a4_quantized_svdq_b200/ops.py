@@ -229,6 +229,25 @@ def svdq_bits_lost(amax_x: torch.Tensor, inv_lambda: Optional[torch.Tensor] = No
     return bits
 
 
+def svdq_lambda_grid(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: torch.Tensor, stream=None) -> dict:
+    """Candidate lambda, 1/lambda [n_alpha, K] and s_g [n_alpha] for every alpha (fp32 device tensors)."""
+    lib = _lib.load()
+    for t, name in ((amax_x, "amax_x"), (amax_w, "amax_w"), (alpha, "alpha")):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.dim() != 1:
+            raise ValueError(f"{name} must be a contiguous 1-D CUDA float32 tensor")
+    k = amax_x.numel()
+    if amax_w.numel() != k:
+        raise ValueError("amax_x and amax_w differ in length")
+    n = alpha.numel()
+    dev = amax_x.device
+    lam = torch.empty((n, k), dtype=torch.float32, device=dev)
+    inv = torch.empty((n, k), dtype=torch.float32, device=dev)
+    s_g = torch.empty(n, dtype=torch.float32, device=dev)
+    _lib.check("svdq_lambda_grid", lib.svdq_lambda_grid(
+        _ptr(amax_x), _ptr(amax_w), k, _ptr(alpha), n, _ptr(lam), _ptr(inv), _ptr(s_g), _stream(stream)))
+    return dict(lam=lam, inv_lam=inv, s_g=s_g)
+
+
 def svdq_device_error(stream=None) -> int:
     """Synchronise and return (then clear) the device error word; 0 = no timeout."""
     code = c_uint32(0)

@@ -281,6 +281,26 @@ int svdq_residual(const void* W, int64_t N, int64_t K, int64_t ldw, const float*
                   const void* down, const void* up, int r, void* R, void* stream);
 
 /*
+ * svdq_lambda_grid -- lambda candidates over a migration-strength grid
+ * ("MiniMax-H3 NVFP4 -- what the smoothing scale should be calibrated on",
+ * section "Calibration": the smoothing scale is picked from a grid of
+ * candidates built from absmax statistics).  For each alpha[c]:
+ *
+ *   lambda[c, j]     = RN32(2^(alpha log2 amax_x[j] - (1 - alpha) log2 amax_w[j]))  (fp64
+ *                      inside; 1 where either absmax is 0; alpha = 0.5 is the
+ *                      square-root rule of svdq_calib_lambda, to within one fp32 ulp)
+ *   inv_lambda[c, j] = RN32(1 / lambda[c, j])
+ *   s_g[c]           = RN32(max_j RN32(amax_x[j] * inv_lambda[c, j]) / 2688), 1 if that max is 0
+ *
+ * amax_x, amax_w: device fp32 [K] (non-negative; e.g. svdq_calib_lambda's
+ * outputs).  alpha: device fp32 [n_alpha].  lambda, inv_lambda: device fp32
+ * [n_alpha, K] (contiguous rows), s_g: device fp32 [n_alpha], written.
+ * 1 <= n_alpha <= 65535.  Asynchronous on `stream`.
+ */
+int svdq_lambda_grid(const float* amax_x, const float* amax_w, int64_t K, const float* alpha, int n_alpha,
+                     float* lambda, float* inv_lambda, float* s_g, void* stream);
+
+/*
  * svdq_bits_lost -- the bits-lost proxy ("MiniMax-H3 NVFP4 -- what the smoothing
  * scale should be calibrated on", section "Why"): 16 consecutive input channels
  * share one FP8 scale set by the group's absmax, so a channel whose absmax is

@@ -141,3 +141,12 @@ def test_bits_lost_rejects_bad_arguments():
     assert lib.svdq_bits_lost(p, 64, 1, None, 64, 2, 64, p, None) == _lib.SVDQ_ERR_INVALID_ARG    # no lambda, 2 candidates
     assert lib.svdq_bits_lost(p, 64, 0, p, 64, 1, 64, p, None) == _lib.SVDQ_ERR_INVALID_ARG       # no modality
     assert lib.svdq_bits_lost(p, 64, 1, p, 64, 1, 64, ctypes.c_void_p(FAKE + 4), None) == _lib.SVDQ_ERR_MISALIGNED
+
+
+def test_lambda_grid_rejects_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(FAKE)
+    assert lib.svdq_lambda_grid(None, p, 64, p, 3, p, p, p, None) == _lib.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_lambda_grid(p, p, 0, p, 3, p, p, p, None) == _lib.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_lambda_grid(p, p, 64, p, 0, p, p, p, None) == _lib.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_lambda_grid(p, p, 64, p, 3, p, ctypes.c_void_p(FAKE + 2), p, None) == _lib.SVDQ_ERR_MISALIGNED
