@@ -337,7 +337,46 @@ def all_configs(P, S, dev, fp4_peak, hbm_peak, flush, flush_read):
         for name in ("1", "all", "video", "text"):
             out[f"config4_layer{layer}_M{L.m}_K{L.k}_N{L.n}_r{L.rank}_lambda_{name}"] = layer_calls(L, name)
         del L
+    out.update(lambda_search(P, S, dev, flush, flush_read))
     return out
+
+
+def lambda_search(P, S, dev, flush, flush_read):
+    """The 39-candidate lambda search on one sweep layer (rank 32, three modalities):
+    wall time of the whole search (host-driven; the randomized rank-32 factorisation of
+    every candidate is library QR/SVD), and the grid and bits-lost kernels timed alone."""
+    import time
+    import torch
+
+    def to_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
+
+    L = S.make_layer(4, layer=0)
+    x, w, bias = to_dev(L.x), to_dev(L.w), to_dev(L.bias)
+    segs_mod = [(sg.begin, sg.end) for sg in L.segments]
+    calib_segs = L.seg_ranges(L.calib_sets["all"])
+    P.search_lambda(x, w, bias, L.rank, calib_segs, segs_mod, alphas=P.alpha_grid(3))      # warm-up
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    res = P.search_lambda(x, w, bias, L.rank, calib_segs, segs_mod)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    n = int(res["alpha"].numel())
+    cal = P.svdq_calib_lambda(x, calib_segs, w)
+    alphas = res["alpha"].to(dev)
+    ax_mod = torch.stack([P.svdq_calib_lambda(x, [sg], None)["amax_x"] for sg in segs_mod])
+    t_grid = _graph_ms(lambda: P.svdq_lambda_grid(cal["amax_x"], cal["amax_w"], alphas), flush, flush_read)
+    inv = res["inv_lam"]
+    t_bits = _graph_ms(lambda: P.svdq_bits_lost(ax_mod, inv), flush, flush_read)
+    rel = res["rel"].cpu().numpy()
+    names = [sg.name for sg in L.segments]
+    return {f"lambda_search_config4_layer0_M{L.m}_K{L.k}_N{L.n}_r{L.rank}": {
+        "candidates": n, "wall_s": wall, "ms_per_candidate": wall / n * 1e3,
+        "best_alpha": float(res["alpha"][res["best"]]),
+        "rel_best": dict(zip(names, rel[res["best"]].tolist())),
+        "rel_alpha_0.5": dict(zip(names, rel[int(np.argmin(np.abs(res["alpha"].numpy() - 0.5)))].tolist())),
+        "lambda_grid_ms": t_grid, "bits_lost_ms": t_bits,
+        "bits_lost_best": dict(zip(names, res["bits"][res["best"]].cpu().tolist()))}}
 
 
 def run_gpu(args):

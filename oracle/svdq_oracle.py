@@ -49,21 +49,21 @@ Readings where the pages are silent (each repeated in the design doc):
      the down factor is stored with lambda folded in (L1s = diag(1/lambda) L1)
      as a [r, K] "down" weight and L2^T as an [N, r] "up" weight, both bf16.
   R10 rel-L2 of a segment is ||Yq - Yref||_F / ||Yref||_F over its rows.
-  R11 The bits-lost proxy uses per-modality channel absmax statistics: the
+  R15 The bits-lost proxy uses per-modality channel absmax statistics: the
       channel's absmax is RN32(ax_j * (1/lambda_j)) (the smoothed statistic
       the kernel's group scale sees; max over rows commutes with the monotone
       rounded product), the group absmax is the largest of its 16 channels,
       and the figure for a modality is the mean of log2(group / channel) over
       the channels whose smoothed absmax is > 0 (a zero channel has nothing to
       lose); 0 if none counts.
-  R12 Candidate smoothing scales over a migration-strength grid:
+  R16 Candidate smoothing scales over a migration-strength grid:
       lambda_j(alpha) = ax_j^alpha / aw_j^(1 - alpha) (R8 is alpha = 0.5),
       evaluated as RN32(2^(alpha log2 ax_j - (1 - alpha) log2 aw_j)) in fp64
       from the fp32 alpha; 1 where either absmax is 0; 1/lambda and s_g per
       candidate as in R5 and R3.
-  R13 The grid: 39 evenly spaced alpha in [0.05, 0.95] (the pages give only
+  R17 The grid: 39 evenly spaced alpha in [0.05, 0.95] (the pages give only
       the count of candidates).
-  R14 Selection: the candidate with the smallest sum over modalities of
+  R18 Selection: the candidate with the smallest sum over modalities of
       w_m * rel_m (weights given by the caller: rows-proportional weights
       reproduce the uniform-rows column, equal weights the per-modality view);
       ties go to the lower index.
@@ -422,7 +422,7 @@ def bits_lost(ax: np.ndarray, inv_lam: Optional[np.ndarray]) -> np.ndarray:
     section "Why": 16 consecutive input channels share one FP8 scale set by the
     group's absmax, so a channel whose own absmax is below the group's loses
     log2(group_absmax / channel_absmax) bits; lambda reshapes that profile
-    because the kernel sees X / lambda (statistics only, no GEMM).  Reading R11.
+    because the kernel sees X / lambda (statistics only, no GEMM).  Reading R15.
 
     ax: fp32 [n_mod, K] per-modality channel absmax of X (``calib`` over the
     modality's rows); inv_lam: fp32 [n_cand, K] candidate 1/lambda rows, or None
@@ -446,12 +446,12 @@ def bits_lost(ax: np.ndarray, inv_lam: Optional[np.ndarray]) -> np.ndarray:
 
 
 def alpha_grid(n: int = 39, lo: float = 0.05, hi: float = 0.95) -> np.ndarray:
-    """The migration-strength grid of R13 as fp32 values."""
+    """The migration-strength grid of R17 as fp32 values."""
     return np.linspace(lo, hi, n).astype(np.float32)
 
 
 def lambda_grid(ax: np.ndarray, aw: np.ndarray, alphas: np.ndarray):
-    """Candidate lambda, 1/lambda and s_g for every alpha (R12).
+    """Candidate lambda, 1/lambda and s_g for every alpha (R16).
 
     "MiniMax-H3 NVFP4 -- what the smoothing scale should be calibrated on",
     section "Calibration": a grid of lambda candidates built from absmax
@@ -477,7 +477,7 @@ def lambda_grid(ax: np.ndarray, aw: np.ndarray, alphas: np.ndarray):
 
 
 def select_candidate(rel: np.ndarray, weights: np.ndarray) -> int:
-    """Index of the candidate with the smallest weighted sum of per-modality rel-L2 (R14)."""
+    """Index of the candidate with the smallest weighted sum of per-modality rel-L2 (R18)."""
     total = np.asarray(rel, np.float64) @ np.asarray(weights, np.float64)
     return int(np.argmin(total))
 
