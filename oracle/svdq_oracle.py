@@ -67,6 +67,15 @@ Readings where the pages are silent (each repeated in the design doc):
       w_m * rel_m (weights given by the caller: rows-proportional weights
       reproduce the uniform-rows column, equal weights the per-modality view);
       ties go to the lower index.
+  R19 MXFP8 ("MiniMax-H3 -- MXFP8 (weight-quantized, vLLM-Omni native layout)",
+      section "Quant format": OCP microscaling FP8, E4M3 elements with one
+      E8M0 scale per 32 consecutive elements, symmetric round-to-nearest,
+      activations quantised dynamically per 32): per block the shared
+      exponent is e = floor(log2 amax) - 8 (8 = the exponent of E4M3's largest
+      power of two), clamped to [-127, 127] and -127 for an all-zero block; the
+      scale byte is e + 127; each element is the E4M3 code of v * 2^-e (an
+      exact product) rounded to nearest, ties to even, saturating at 448, sign
+      kept (-0 -> 0x80).  No smoothing, no low-rank branch, no tensor scale.
 
 Pins (``tests/test_oracle_pins.py``) hold every function to something other
 than itself: independent float-format rounding, torch's float8 conversion,
@@ -480,6 +489,57 @@ def select_candidate(rel: np.ndarray, weights: np.ndarray) -> int:
     """Index of the candidate with the smallest weighted sum of per-modality rel-L2 (R18)."""
     total = np.asarray(rel, np.float64) @ np.asarray(weights, np.float64)
     return int(np.argmin(total))
+
+
+# ----------------------------------------------------------------------------
+# MXFP8 W8A8 (page 5 "Quant format"; R19)
+# ----------------------------------------------------------------------------
+
+MX_BLOCK = 32
+E4M3_EMAX = 8                       # 448 = 1.75 * 2^8
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """Signed fp32 values -> E4M3 bytes: nearest, ties to even, satfinite at 448, sign kept."""
+    v = np.asarray(v, dtype=np.float32)
+    mag = e4m3_encode_nonneg(np.abs(v))
+    return (mag | np.where(np.signbit(v), np.uint8(0x80), np.uint8(0))).astype(np.uint8)
+
+
+def mx_shared_exponent(amax: np.ndarray) -> np.ndarray:
+    """floor(log2 amax) - 8, clamped to [-127, 127]; -127 where amax is 0 (R19)."""
+    amax = np.asarray(amax, dtype=np.float64)
+    _, e2 = np.frexp(amax)                    # amax = m 2^e2 with m in [0.5, 1): floor(log2) = e2 - 1
+    e = np.where(amax > 0, e2.astype(np.int64) - 1 - E4M3_EMAX, -127)
+    return np.clip(e, -127, 127)
+
+
+def mx_quantize(x_bits: np.ndarray):
+    """bf16 [R, K] -> (E4M3 codes u8 [R, K], E8M0 scale bytes u8 [R, K/32]) (R19)."""
+    x = bf16_to_f64(x_bits)
+    r, k = x.shape
+    if k % MX_BLOCK:
+        raise ValueError("K must be a multiple of 32")
+    blocks = x.reshape(r, k // MX_BLOCK, MX_BLOCK)
+    e = mx_shared_exponent(np.abs(blocks).max(axis=2))
+    scaled = blocks * np.exp2(-e.astype(np.float64))[:, :, None]      # exact: a power of two
+    codes = e4m3_encode(scaled.astype(np.float32))
+    return codes.reshape(r, k), (e + 127).astype(np.uint8)
+
+
+def mx_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """E4M3 codes [R, K] and E8M0 scale bytes [R, K/32] -> fp64 [R, K]."""
+    r, k = codes.shape
+    vals = e4m3_decode(codes).reshape(r, k // MX_BLOCK, MX_BLOCK)
+    return (vals * np.exp2(np.asarray(scales, np.float64) - 127.0)[:, :, None]).reshape(r, k)
+
+
+def mx_linear(a_codes, a_sf, w_codes, w_sf, bias_bits: Optional[np.ndarray]) -> np.ndarray:
+    """The W8A8 MXFP8 linear in fp64: dequant(A) dequant(W)^T + b."""
+    y = mx_dequantize(a_codes, a_sf) @ mx_dequantize(w_codes, w_sf).T
+    if bias_bits is not None:
+        y = y + bf16_to_f64(bias_bits)[None, :]
+    return y
 
 
 # ----------------------------------------------------------------------------
