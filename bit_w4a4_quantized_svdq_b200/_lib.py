@@ -60,6 +60,10 @@ SIGNATURES = {
     "svdq_bits_lost": (c_int, [c_void_p, c_int64, c_int, c_void_p, c_int64, c_int, c_int64, c_void_p, c_void_p]),
     "svdq_lambda_grid": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                                  c_void_p]),
+    "svdq_mxfp8_sf_bytes": (c_size_t, [c_int64, c_int64]),
+    "svdq_quantize_mxfp8": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
+    "svdq_linear_mxfp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64,
+                                  c_int64, c_int64, c_void_p]),
 }
 
 _lib = None

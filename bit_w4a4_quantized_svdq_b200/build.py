@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_PATH = os.path.join(PKG_DIR, "libsvdq.so")
 INCLUDE = os.path.join(os.path.dirname(PKG_DIR), "include")
 
-SOURCES = ["abi.cu", "calib.cu", "quantize.cu", "linear.cu", "score.cu", "residual.cu", "proxy.cu", "grid.cu"]
+SOURCES = ["abi.cu", "calib.cu", "quantize.cu", "linear.cu", "score.cu", "residual.cu", "proxy.cu", "grid.cu", "mxfp8.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

@@ -169,7 +169,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return l | (h << 16);
 }
 
-template <bool kOutF32, bool kScore>
+template <bool kOutF32, bool kScore, bool kMx>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
               const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_r,
@@ -193,9 +193,19 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     const int warp = threadIdx.x >> 5;
     const uint32_t lane = threadIdx.x & 31;
     const int num_tiles = args.m_tiles * args.n_tiles;
-    const int k_stages = static_cast<int>(args.K / kBK);
+    // Format constants.  NVFP4: 256 channels per 128-byte stage row, four scale
+    // atoms per 128 rows per stage (one per MMA of K = 64).  MXFP8: 128 channels
+    // per stage row, one scale atom per 128 rows per stage whose four bytes serve
+    // the stage's four MMAs of K = 32 (scale ids 0..3).
+    constexpr int kStageK = kMx ? 128 : kBK;
+    constexpr uint32_t kSfaPairT = kMx ? 1024 : kSfaPair;          // A scale bytes of two stages
+    constexpr uint32_t kSfSlotT = kMx ? 3072 : kSfSlot;            // A + W scale bytes of two stages
+    constexpr int kSfHalvesPerStage = kMx ? 2 : 8;                  // 256-byte scale pieces per row block
+    constexpr uint32_t kTmemSfStrideT = kMx ? 16 : kTmemSfStride;
+    constexpr uint32_t kTmemSfbOffT = kMx ? 4 : kTmemSfbOff;
+    const int k_stages = static_cast<int>(args.K / kStageK);
     const bool has_lr = args.r > 0;
-    const float alpha = __fmul_rn(__ldg(args.s_g_act), __ldg(args.s_g_w));
+    const float alpha = kMx ? 1.0f : __fmul_rn(__ldg(args.s_g_act), __ldg(args.s_g_w));
     const float inv_alpha = __frcp_rn(alpha);
 
     if (threadIdx.x == 0) {
@@ -244,10 +254,10 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 int m_blk, n_blk;
                 tile_coords(args, sf_tile, m_blk, n_blk);
                 uint8_t* dst = smem + kOffSf + slot * kSfSlot;
-                mbar_arrive_expect_tx(&sf_data[slot], kSfSlot);
+                mbar_arrive_expect_tx(&sf_data[slot], kSfSlotT);
                 // scale atoms of stages sf_kb and sf_kb + 1 (a last odd stage reads zeros past K)
-                tma_load_3d(dst, &tmap_sfa, &sf_data[slot], 0, sf_kb * 8, m_blk);
-                tma_load_3d(dst + kSfaPair, &tmap_sfb, &sf_data[slot], 0, sf_kb * 8, 2 * n_blk);
+                tma_load_3d(dst, &tmap_sfa, &sf_data[slot], 0, sf_kb * kSfHalvesPerStage, m_blk);
+                tma_load_3d(dst + kSfaPairT, &tmap_sfb, &sf_data[slot], 0, sf_kb * kSfHalvesPerStage, 2 * n_blk);
                 ++issued;
                 sf_kb += 2;
                 if (sf_kb >= k_stages) {
@@ -307,11 +317,18 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     }
                     tc_fence_after();
                     const uint64_t da = da0 + kStageDesc * s, db = db0 + kStageDesc * s;
-                    const uint32_t sf = tmem + kTmemSf0 + s * kTmemSfStride;
-                    mma_nvf4(tmem, da, db, idesc_f4, sf, sf + kTmemSfbOff, kb == 0 ? 0u : 1u);
-                    mma_nvf4(tmem, da + 2, db + 2, idesc_f4, sf + 4, sf + kTmemSfbOff + 8, 1u);
-                    mma_nvf4(tmem, da + 4, db + 4, idesc_f4, sf + 8, sf + kTmemSfbOff + 16, 1u);
-                    mma_nvf4(tmem, da + 6, db + 6, idesc_f4, sf + 12, sf + kTmemSfbOff + 24, 1u);
+                    const uint32_t sf = tmem + kTmemSf0 + s * kTmemSfStrideT;
+                    if constexpr (kMx) {
+                        mma_mxf8(tmem, da, db, idesc_mxf8(kBM, kBN, 0), sf, sf + kTmemSfbOffT, kb == 0 ? 0u : 1u);
+                        mma_mxf8(tmem, da + 2, db + 2, idesc_mxf8(kBM, kBN, 1), sf, sf + kTmemSfbOffT, 1u);
+                        mma_mxf8(tmem, da + 4, db + 4, idesc_mxf8(kBM, kBN, 2), sf, sf + kTmemSfbOffT, 1u);
+                        mma_mxf8(tmem, da + 6, db + 6, idesc_mxf8(kBM, kBN, 3), sf, sf + kTmemSfbOffT, 1u);
+                    } else {
+                        mma_nvf4(tmem, da, db, idesc_f4, sf, sf + kTmemSfbOff, kb == 0 ? 0u : 1u);
+                        mma_nvf4(tmem, da + 2, db + 2, idesc_f4, sf + 4, sf + kTmemSfbOff + 8, 1u);
+                        mma_nvf4(tmem, da + 4, db + 4, idesc_f4, sf + 8, sf + kTmemSfbOff + 16, 1u);
+                        mma_nvf4(tmem, da + 6, db + 6, idesc_f4, sf + 12, sf + kTmemSfbOff + 24, 1u);
+                    }
                     tc_commit(&empty[s]);
                     if (++s == kStages) { s = 0; ph ^= 1u; }
                 }
@@ -426,17 +443,30 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 // buffer: A scales of MMA kk at 4 kk + (row / 32); W scales of MMA
                 // kk at 16 + 8 kk + (row / 32), rows 128..255 at + 4.  Lane i reads
                 // row i of each 512-byte atom: its 4 words are the 4 columns.
-                const uint8_t* sfa = smem + kOffSf + slot * kSfSlot + (kb & 1) * 2048;
-                const uint8_t* sfb = smem + kOffSf + slot * kSfSlot + kSfaPair + (kb & 1) * 2048;
-                uint32_t ra[16], rb[32];
+                uint32_t ra[kMx ? 4 : 16], rb[kMx ? 8 : 32];
+                if constexpr (kMx) {
+                    // MXFP8: the stage's one A atom and one W atom per 128-row block
+                    // (slot layout: A [2 stages][512], then W [2 row blocks][2 stages][512]).
+                    const uint8_t* sfa = smem + kOffSf + slot * kSfSlot + (kb & 1) * 512;
+                    const uint8_t* sfb = smem + kOffSf + slot * kSfSlot + kSfaPairT + (kb & 1) * 512;
+                    const uint4 a = *reinterpret_cast<const uint4*>(sfa + lane * 16);
+                    const uint4 x = *reinterpret_cast<const uint4*>(sfb + lane * 16);
+                    const uint4 y = *reinterpret_cast<const uint4*>(sfb + 1024 + lane * 16);
+                    ra[0] = a.x; ra[1] = a.y; ra[2] = a.z; ra[3] = a.w;
+                    rb[0] = x.x; rb[1] = x.y; rb[2] = x.z; rb[3] = x.w;
+                    rb[4] = y.x; rb[5] = y.y; rb[6] = y.z; rb[7] = y.w;
+                } else {
+                    const uint8_t* sfa = smem + kOffSf + slot * kSfSlot + (kb & 1) * 2048;
+                    const uint8_t* sfb = smem + kOffSf + slot * kSfSlot + kSfaPair + (kb & 1) * 2048;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 a = *reinterpret_cast<const uint4*>(sfa + q * 512 + lane * 16);
-                    const uint4 x = *reinterpret_cast<const uint4*>(sfb + q * 512 + lane * 16);
-                    const uint4 y = *reinterpret_cast<const uint4*>(sfb + 4096 + q * 512 + lane * 16);
-                    ra[4 * q] = a.x; ra[4 * q + 1] = a.y; ra[4 * q + 2] = a.z; ra[4 * q + 3] = a.w;
-                    rb[8 * q] = x.x; rb[8 * q + 1] = x.y; rb[8 * q + 2] = x.z; rb[8 * q + 3] = x.w;
-                    rb[8 * q + 4] = y.x; rb[8 * q + 5] = y.y; rb[8 * q + 6] = y.z; rb[8 * q + 7] = y.w;
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 a = *reinterpret_cast<const uint4*>(sfa + q * 512 + lane * 16);
+                        const uint4 x = *reinterpret_cast<const uint4*>(sfb + q * 512 + lane * 16);
+                        const uint4 y = *reinterpret_cast<const uint4*>(sfb + 4096 + q * 512 + lane * 16);
+                        ra[4 * q] = a.x; ra[4 * q + 1] = a.y; ra[4 * q + 2] = a.z; ra[4 * q + 3] = a.w;
+                        rb[8 * q] = x.x; rb[8 * q + 1] = x.y; rb[8 * q + 2] = x.z; rb[8 * q + 3] = x.w;
+                        rb[8 * q + 4] = y.x; rb[8 * q + 5] = y.y; rb[8 * q + 6] = y.z; rb[8 * q + 7] = y.w;
+                    }
                 }
                 if ((kb & 1) == 1 || kb == k_stages - 1) {
                     __syncwarp();
@@ -447,9 +477,16 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     ok = false;
                     break;
                 }
-                const uint32_t base = tq + kTmemSf0 + s * kTmemSfStride;
-                tmem_st_32x32b_x16(base, ra);
-                tmem_st_32x32b_x32(base + kTmemSfbOff, rb);
+                const uint32_t base = tq + kTmemSf0 + s * kTmemSfStrideT;
+                if constexpr (kMx) {
+                    // columns: A 0..3, W rows 0..127 at 4..7 and rows 128..255 at 8..11
+                    const uint32_t r[16] = {ra[0], ra[1], ra[2], ra[3], rb[0], rb[1], rb[2], rb[3],
+                                            rb[4], rb[5], rb[6], rb[7], 0u, 0u, 0u, 0u};
+                    tmem_st_32x32b_x16(base, r);
+                } else {
+                    tmem_st_32x32b_x16(base, ra);
+                    tmem_st_32x32b_x32(base + kTmemSfbOff, rb);
+                }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -801,12 +838,12 @@ inline int linear_grid(int m_tiles, int n_tiles) {
     return static_cast<int>(tiles < sms ? tiles : sms);
 }
 
-template <bool kOutF32, bool kScore>
+template <bool kOutF32, bool kScore, bool kMx = false>
 int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, const CUtensorMap& tr,
                   const CUtensorMap& tsa, const CUtensorMap& tsb, const LinearArgs& a, cudaStream_t st) {
     static_assert(!(kOutF32 && kScore), "scoring is fused into the bf16 epilogue only");
     const uint32_t smem = kSmemBytes + 1024;
-    auto kern = linear_kernel<kOutF32, kScore>;
+    auto kern = linear_kernel<kOutF32, kScore, kMx>;
     static std::atomic<uint64_t> smem_set{0};
     if (!set_dynamic_smem_once(kern, smem, smem_set)) return SVDQ_ERR_CUDA;
     const int tiles = a.m_tiles * a.n_tiles;
@@ -830,17 +867,19 @@ int linear_prepare(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g
                    const uint8_t* w_codes, const uint8_t* w_sf, const float* s_g_w, const void* up,
                    const void* bias, void* Y, int64_t ldy, int out_dtype, int64_t M, int64_t N, int64_t K,
                    CUtensorMap* ta, CUtensorMap* tb, CUtensorMap* ty, CUtensorMap* tsa, CUtensorMap* tsb,
-                   LinearArgs* a) {
-    if (a_codes == nullptr || a_sf == nullptr || w_codes == nullptr || w_sf == nullptr || s_g_act == nullptr ||
-        s_g_w == nullptr)
+                   LinearArgs* a, bool mx = false) {
+    // mx: MXFP8 operands (one byte per element, E8M0 scales per 32, no tensor
+    // scales, no low-rank branch); otherwise NVFP4 (two elements per byte).
+    if (a_codes == nullptr || a_sf == nullptr || w_codes == nullptr || w_sf == nullptr ||
+        (!mx && (s_g_act == nullptr || s_g_w == nullptr)))
         return SVDQ_ERR_INVALID_ARG;
     if (M < 1 || N < 1 || K < 1 || (Y != nullptr && ldy < N)) return SVDQ_ERR_INVALID_ARG;
     if (out_dtype != 0 && out_dtype != 1) return SVDQ_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(s_g_act) & 3u) || (reinterpret_cast<uintptr_t>(s_g_w) & 3u))
         return SVDQ_ERR_MISALIGNED;
-    if (r != 0 && r != 16 && r != 32) return SVDQ_ERR_UNSUPPORTED;
+    if (mx ? r != 0 : (r != 0 && r != 16 && r != 32)) return SVDQ_ERR_UNSUPPORTED;
     if ((r > 0) != (D != nullptr) || (r > 0) != (up != nullptr)) return SVDQ_ERR_INVALID_ARG;
-    if (K % 256 != 0 || N % 256 != 0) return SVDQ_ERR_UNSUPPORTED;
+    if (K % (mx ? 128 : 256) != 0 || N % 256 != 0) return SVDQ_ERR_UNSUPPORTED;
     if (M > (int64_t(1) << 31) - 128 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 30))
         return SVDQ_ERR_UNSUPPORTED;
     const int64_t m_tiles = (M + 127) / 128, n_tiles = N / 256;
@@ -854,20 +893,25 @@ int linear_prepare(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g
     uint32_t* err = device_error_word();
     if (err == nullptr) return SVDQ_ERR_CUDA;
 
-    if (!encode_tmap_2d(ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a_codes, K / 2, M, K / 2, 128, 128,
+    const int64_t row_bytes = mx ? K : K / 2;
+    if (!encode_tmap_2d(ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a_codes, row_bytes, M, row_bytes, 128, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tmap_2d(tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_codes, K / 2, N, K / 2, 128, 256,
+        !encode_tmap_2d(tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_codes, row_bytes, N, row_bytes, 128, 256,
                         CU_TENSOR_MAP_SWIZZLE_128B))
         return SVDQ_ERR_CUDA;
     *ty = *ta;
     if (out_dtype == 0 && Y != nullptr &&
         !encode_tmap_2d(ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, N, M, ldy * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
         return SVDQ_ERR_CUDA;
-    // Scale atoms viewed as [row block][K / 64 atoms x 2 halves][256 bytes]: one box
-    // holds the 8 atoms of two stages (A: one row block, W: two).
-    const uint64_t halves = static_cast<uint64_t>(K / 64) * 2;
-    if (!encode_tmap_3d_u8(tsa, a_sf, 256, halves, static_cast<uint64_t>(m_tiles), 256, halves * 256, 256, 16, 1) ||
-        !encode_tmap_3d_u8(tsb, w_sf, 256, halves, static_cast<uint64_t>(N / 128), 256, halves * 256, 256, 16, 2))
+    // Scale atoms viewed as [row block][atoms x 2 halves][256 bytes]: one box
+    // holds the atoms of two stages (A: one row block, W: two).  NVFP4: K / 64
+    // atoms per row block, 4 per stage; MXFP8: K / 128 atoms, 1 per stage.
+    const uint64_t halves = mx ? static_cast<uint64_t>(K / 128) * 2 : static_cast<uint64_t>(K / 64) * 2;
+    const uint32_t box_halves = mx ? 4 : 16;
+    if (!encode_tmap_3d_u8(tsa, a_sf, 256, halves, static_cast<uint64_t>(m_tiles), 256, halves * 256, 256,
+                           box_halves, 1) ||
+        !encode_tmap_3d_u8(tsb, w_sf, 256, halves, static_cast<uint64_t>(N / 128), 256, halves * 256, 256,
+                           box_halves, 2))
         return SVDQ_ERR_CUDA;
     *a = LinearArgs{};
     a->a_sf = a_sf;
@@ -910,6 +954,19 @@ extern "C" int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const fl
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return out_dtype ? launch_linear<true, false>(ta, tb, ty, ta, tsa, tsb, a, st)
                      : launch_linear<false, false>(ta, tb, ty, ta, tsa, tsb, a, st);
+}
+
+extern "C" int svdq_linear_mxfp8(const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* w_codes,
+                                 const uint8_t* w_sf, const void* bias, void* Y, int64_t ldy, int64_t M, int64_t N,
+                                 int64_t K, void* stream) {
+    using namespace svdq;
+    if (Y == nullptr) return SVDQ_ERR_INVALID_ARG;
+    CUtensorMap ta, tb, ty, tsa, tsb;
+    LinearArgs a;
+    const int st0 = linear_prepare(a_codes, a_sf, nullptr, nullptr, 0, w_codes, w_sf, nullptr, nullptr, bias, Y, ldy,
+                                   0, M, N, K, &ta, &tb, &ty, &tsa, &tsb, &a, true);
+    if (st0 != SVDQ_OK) return st0;
+    return launch_linear<false, false, true>(ta, tb, ty, ta, tsa, tsb, a, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" size_t svdq_linear_score_workspace_bytes(int n_seg) {

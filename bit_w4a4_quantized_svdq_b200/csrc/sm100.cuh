@@ -247,6 +247,19 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint6
            "r"(sfa_tmem), "r"(sfb_tmem) : "memory");
 }
 
+// Block-scaled FP8 MMA: kind::mxf8f6f4, one E8M0 scale per 32 elements
+// (scale_vec::1X), K = 32 per instruction.  Each 32-bit tensor-memory scale word
+// holds four scale bytes; the instruction descriptor's scale ids pick the byte.
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate),
+           "r"(sfa_tmem), "r"(sfb_tmem) : "memory");
+}
+
 // Copy a 32-row x 128-bit shared-memory block into tensor memory, replicated
 // into all four 32-lane quarters (the layout block scales are read from).
 __device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
@@ -375,6 +388,19 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(uint32_t m, uint32_t n) {
          | ((n >> 3) << 17)     // N / 8
          | (0u << 23)           // scale format: E4M3
          | ((m >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with E4M3 A/B and E8M0 block scales (one
+// per 32 elements), both K-major, K = 32 per instruction; `sf_id` selects the
+// byte of the A and B scale words this instruction uses.
+__host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t m, uint32_t n, uint32_t sf_id) {
+    return (sf_id << 4)         // B scale factor id
+         | (0u << 7)            // A format: E4M3
+         | (0u << 10)           // B format: E4M3
+         | ((n >> 3) << 17)     // N / 8
+         | (1u << 23)           // scale format: E8M0
+         | ((m >> 4) << 24)     // M / 16
+         | (sf_id << 29);       // A scale factor id
 }
 
 // ---------------------------------------------------------------------------

@@ -248,6 +248,41 @@ def svdq_lambda_grid(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: torch.Te
     return dict(lam=lam, inv_lam=inv, s_g=s_g)
 
 
+def mxfp8_sf_bytes(rows: int, k: int) -> int:
+    return int(_lib.load().svdq_mxfp8_sf_bytes(rows, k))
+
+
+def svdq_quantize_mxfp8(x: torch.Tensor, out: Optional[dict] = None, stream=None) -> dict:
+    """bf16 [M, K] -> dict(codes u8 [M, K] E4M3, sf u8 E8M0 scales in the tensor-core layout)."""
+    lib = _lib.load()
+    _check_bf16(x, "x")
+    m, k = x.shape
+    nbytes = mxfp8_sf_bytes(m, k)
+    if nbytes == 0:
+        raise ValueError("K must be a positive multiple of 128")
+    if out is None:
+        out = dict(codes=torch.empty((m, k), dtype=torch.uint8, device=x.device),
+                   sf=torch.empty(nbytes, dtype=torch.uint8, device=x.device))
+    _lib.check("svdq_quantize_mxfp8", lib.svdq_quantize_mxfp8(
+        _ptr(x), m, k, _row_stride(x, "x"), _ptr(out["codes"]), _ptr(out["sf"]), _stream(stream)))
+    return out
+
+
+def svdq_linear_mxfp8(a_codes: torch.Tensor, a_sf: torch.Tensor, w_codes: torch.Tensor, w_sf: torch.Tensor,
+                      bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """Y bf16 [M, N] = dequant(A) dequant(W)^T + bias on the MXFP8 tensor-core path."""
+    lib = _lib.load()
+    m, k = a_codes.shape
+    n = w_codes.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=a_codes.device)
+    _lib.check("svdq_linear_mxfp8", lib.svdq_linear_mxfp8(
+        _ptr(a_codes), _ptr(a_sf), _ptr(w_codes), _ptr(w_sf), _ptr(bias), _ptr(out), _row_stride(out, "out"),
+        m, n, k, _stream(stream)))
+    return out
+
+
 def svdq_device_error(stream=None) -> int:
     """Synchronise and return (then clear) the device error word; 0 = no timeout."""
     code = c_uint32(0)

@@ -281,6 +281,38 @@ int svdq_residual(const void* W, int64_t N, int64_t K, int64_t ldw, const float*
                   const void* down, const void* up, int r, void* R, void* stream);
 
 /*
+ * MXFP8 W8A8 variant ("MiniMax-H3 -- MXFP8 (weight-quantized, vLLM-Omni native
+ * layout)", section "Quant format": OCP microscaling FP8, E4M3 elements with one
+ * E8M0 scale per 32 elements, symmetric round-to-nearest; activations quantised
+ * dynamically per 32).  No smoothing, no low-rank branch, no tensor scales.
+ *
+ * svdq_mxfp8_sf_bytes -- bytes of the scale array of `rows` rows:
+ * ceil(rows / 128) * 128 * K / 32 (0 unless K is a positive multiple of 128).
+ *
+ * svdq_quantize_mxfp8 -- X bf16 [M, K] (device, row stride ldx elements, ldx >= K,
+ * ldx * 2 a multiple of 16, 16-byte aligned) -> codes u8 [M, K] (device, row
+ * stride K, 16-byte aligned): E4M3 of x * 2^-e per 32-element block, e = floor(log2
+ * amax) - 8 clamped to [-127, 127] (-127 for an all-zero block), nearest even,
+ * saturating at 448, sign kept; sf u8 (device, 4-byte aligned,
+ * svdq_mxfp8_sf_bytes(M, K) bytes): the E8M0 bytes e + 127 in the tensor-core
+ * scale layout of svdq_quantize_act (128-row x 4-block atoms), rows M.. of the
+ * padding set to 0.  Used for activations and, once, for weights [N, K].
+ * K % 128 == 0 (SVDQ_ERR_UNSUPPORTED otherwise).
+ *
+ * svdq_linear_mxfp8 -- Y[m, n] = bf16( sum_k dec(A)[m, k] dec(W)[n, k] + bias[n] ),
+ * dec(v) = E4M3(v) * 2^(scale - 127), fp32 accumulation on the tensor cores
+ * (tcgen05 kind::mxf8f6f4 with E8M0 block scales).  A from svdq_quantize_mxfp8 of
+ * X [M, K], W from it on the weight [N, K]; bias bf16 [N] or NULL; Y bf16 [M, N]
+ * (device, row stride ldy >= N, ldy * 2 a multiple of 16, 16-byte aligned).
+ * K % 128 == 0, N % 256 == 0, M >= 1.  Asynchronous on `stream`.
+ */
+size_t svdq_mxfp8_sf_bytes(int64_t rows, int64_t K);
+int svdq_quantize_mxfp8(const void* X, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* sf,
+                        void* stream);
+int svdq_linear_mxfp8(const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* w_codes, const uint8_t* w_sf,
+                      const void* bias, void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
  * svdq_lambda_grid -- lambda candidates over a migration-strength grid
  * ("MiniMax-H3 NVFP4 -- what the smoothing scale should be calibrated on",
  * section "Calibration": the smoothing scale is picked from a grid of

@@ -150,3 +150,17 @@ def test_lambda_grid_rejects_bad_arguments():
     assert lib.svdq_lambda_grid(p, p, 0, p, 3, p, p, p, None) == _lib.SVDQ_ERR_INVALID_ARG
     assert lib.svdq_lambda_grid(p, p, 64, p, 0, p, p, p, None) == _lib.SVDQ_ERR_INVALID_ARG
     assert lib.svdq_lambda_grid(p, p, 64, p, 3, p, ctypes.c_void_p(FAKE + 2), p, None) == _lib.SVDQ_ERR_MISALIGNED
+
+
+def test_mxfp8_sizes_and_bad_arguments():
+    lib = _lib.load()
+    p = ctypes.c_void_p(FAKE)
+    assert lib.svdq_mxfp8_sf_bytes(1, 128) == 128 * 4
+    assert lib.svdq_mxfp8_sf_bytes(129, 5120) == 256 * 160
+    assert lib.svdq_mxfp8_sf_bytes(4, 96) == 0
+    assert lib.svdq_quantize_mxfp8(None, 4, 128, 128, p, p, None) == _lib.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_quantize_mxfp8(p, 4, 192, 192, p, p, None) == _lib.SVDQ_ERR_UNSUPPORTED
+    assert lib.svdq_quantize_mxfp8(p, 4, 128, 100, p, p, None) == _lib.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_linear_mxfp8(p, p, p, p, None, None, 256, 4, 256, 128, None) == _lib.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_linear_mxfp8(p, p, p, p, None, p, 256, 4, 256, 192, None) == _lib.SVDQ_ERR_UNSUPPORTED
+    assert lib.svdq_linear_mxfp8(p, p, p, p, None, p, 256, 4, 200, 128, None) == _lib.SVDQ_ERR_UNSUPPORTED
