@@ -321,6 +321,22 @@ def all_configs(P, S, dev, fp4_peak, hbm_peak, flush, flush_read):
             same = bool(np.allclose(rel_f.cpu().numpy(), rel.cpu().numpy(), rtol=1e-9, atol=0))
             r[key] = {"ms": t, "TFLOP/s": fl / (t * 1e-3) / 1e12, "linear_plus_score_ms": sep,
                       "speedup_vs_separate": sep / t, "rel_matches_separate": same}
+        if calib_name == "all":
+            # the MXFP8 W8A8 variant of the same layer (no smoothing, no low-rank branch)
+            qa = P.svdq_quantize_mxfp8(x)
+            qw = P.svdq_quantize_mxfp8(w)
+            t = _graph_ms(lambda: P.svdq_quantize_mxfp8(x, out=qa), flush, flush_read)
+            by = (2 + 1 + 1.0 / 32) * L.m * L.k
+            r["mxfp8_quantize"] = {"ms": t, "GB/s": by / (t * 1e-3) / 1e9,
+                                   "frac_hbm": by / (t * 1e-3) / 1e9 / hbm_peak}
+            t = _graph_ms(lambda: P.svdq_linear_mxfp8(qa["codes"], qa["sf"], qw["codes"], qw["sf"], lin.bias, out=y),
+                          flush, flush_read)
+            fp8_peak = fp4_peak / 2.0
+            r["mxfp8_linear"] = {"ms": t, "TFLOP/s": fl / (t * 1e-3) / 1e12,
+                                 "frac_fp8": fl / (t * 1e-3) / 1e12 / fp8_peak, "fp8_peak": fp8_peak}
+            _, _, rel_mx = P.svdq_score_lambda(y, yref, segs_mod, workspace=ws)
+            r["mxfp8_rel_l2_vs_bf16"] = dict(zip([sg.name for sg in L.segments], rel_mx.cpu().tolist()))
+            del qa, qw
         del x, w, bias, cal, lin, q, y, yref, ws, wf
         torch.cuda.empty_cache()
         return r
