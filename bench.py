@@ -395,6 +395,50 @@ def lambda_search(P, S, dev, flush, flush_read):
         "bits_lost_best": dict(zip(names, res["bits"][res["best"]].cpu().tolist()))}}
 
 
+def profile_case(name: str) -> int:
+    """A few launches of one kernel on the attention-projection workload, for a profiler:
+    two warm-up launches, then three (capture with -s 2 -c 1..3 on the kernel's name)."""
+    import torch
+
+    import bit_w4a4_quantized_svdq_b200 as P
+    import synthetic as S
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    L = S.make_layer(CONFIG_INDEX)
+
+    def to_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
+
+    x, w, bias = to_dev(L.x), to_dev(L.w), to_dev(L.bias)
+    segs_mod = [(sg.begin, sg.end) for sg in L.segments]
+    if name == "linear_score":
+        cal = P.svdq_calib_lambda(x, L.seg_ranges(L.calib_sets["all"]), w)
+        lin = P.SVDQW4A4Linear.convert(w, bias, cal, L.rank)
+        q = P.svdq_quantize_act(x, cal["inv_lam"], lin.s_g_act, lin.down)
+        yref = x.view(torch.bfloat16) @ w.view(torch.bfloat16).t() + bias.view(torch.bfloat16)
+        wf = torch.empty(P.linear_score_workspace_bytes(len(segs_mod)), dtype=torch.uint8, device=dev)
+        args = (q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf, lin.s_g_w, lin.up, lin.bias)
+        run = lambda: P.svdq_linear_score(*args, yref=yref, segs=segs_mod, write_out=False, workspace=wf)
+    elif name in ("mxfp8_linear", "mxfp8_quantize"):
+        qa = P.svdq_quantize_mxfp8(x)
+        qw = P.svdq_quantize_mxfp8(w)
+        y = torch.empty((L.m, L.n), dtype=torch.bfloat16, device=dev)
+        if name == "mxfp8_linear":
+            run = lambda: P.svdq_linear_mxfp8(qa["codes"], qa["sf"], qw["codes"], qw["sf"], bias, out=y)
+        else:
+            run = lambda: P.svdq_quantize_mxfp8(x, out=qa)
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    torch.cuda.synchronize()
+    for _ in range(5):
+        run()
+    torch.cuda.synchronize()
+    assert P.svdq_device_error() == 0
+    print(json.dumps({"profile_case": name, "launches": 5}))
+    return 0
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -649,11 +693,15 @@ def main():
     ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-large", action="store_true", help="skip the two largest-shape GEMM measurements")
+    ap.add_argument("--profile-case", default=None, choices=["linear_score", "mxfp8_linear", "mxfp8_quantize"],
+                    help="only launch one kernel five times on the attention-projection workload (for ncu)")
     ap.add_argument("--all-configs", action="store_true",
                     help="also time every call on every configured workload (adds a few minutes)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "svdq":
         args.warmup = 3
+    if args.profile_case:
+        return profile_case(args.profile_case)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)
