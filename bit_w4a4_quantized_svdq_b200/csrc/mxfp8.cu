@@ -39,31 +39,40 @@ __device__ __forceinline__ int64_t mx_sf_offset(int64_t row, int64_t blk, int64_
 }
 
 __global__ void __launch_bounds__(kMxThreads)
-mx_quantize_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int64_t ldx, int64_t rows_pad,
+mx_quantize_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int64_t ldx, uint32_t n_units,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
     const int lane = threadIdx.x & 31;
-    const int64_t segs_per_row = (K + 255) / 256;
-    const int64_t n_units = rows_pad * segs_per_row;
-    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kMxThreads / 32);
+    const uint32_t segs_per_row = static_cast<uint32_t>((K + 255) / 256);
+    const uint32_t warps = gridDim.x * (kMxThreads / 32);
     const int64_t blocks_per_row = K / 32;
-    for (int64_t u0 = (static_cast<int64_t>(blockIdx.x) * (kMxThreads / 32) + (threadIdx.x >> 5)) * kMxSegs;
-         u0 < n_units; u0 += warps * kMxSegs) {
+    for (uint32_t u0 = (blockIdx.x * (kMxThreads / 32) + (threadIdx.x >> 5)) * kMxSegs; u0 < n_units;
+         u0 += warps * kMxSegs) {
+        // (row, segment) of the warp's units: one division, then carried along the row
+        int64_t rows[kMxSegs], cols[kMxSegs];
+        {
+            uint32_t row = u0 / segs_per_row, seg = u0 - row * segs_per_row;
+#pragma unroll
+            for (int i = 0; i < kMxSegs; ++i) {
+                rows[i] = row;
+                cols[i] = static_cast<int64_t>(seg) * 256 + lane * 8;
+                if (++seg == segs_per_row) {
+                    seg = 0;
+                    ++row;
+                }
+            }
+        }
         uint4 v[kMxSegs];
 #pragma unroll
         for (int i = 0; i < kMxSegs; ++i) {
-            const int64_t u = u0 + i;
-            const int64_t row = u / segs_per_row;
-            const int64_t col = (u - row * segs_per_row) * 256 + lane * 8;
-            v[i] = (u < n_units && row < M && col < K)
-                       ? __ldg(reinterpret_cast<const uint4*>(X + row * ldx + col))
+            v[i] = (u0 + i < n_units && rows[i] < M && cols[i] < K)
+                       ? __ldg(reinterpret_cast<const uint4*>(X + rows[i] * ldx + cols[i]))
                        : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int i = 0; i < kMxSegs; ++i) {
-            const int64_t u = u0 + i;
-            if (u >= n_units) break;                 // warp-uniform
-            const int64_t row = u / segs_per_row;
-            const int64_t col = (u - row * segs_per_row) * 256 + lane * 8;
+            if (u0 + i >= n_units) break;            // warp-uniform
+            const int64_t row = rows[i];
+            const int64_t col = cols[i];
             const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
             // |bf16| as bits with the sign cleared: integer order is value order
             uint32_t m2 = 0;
@@ -75,15 +84,14 @@ mx_quantize_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int64_t
             const int bexp = static_cast<int>(m >> 7);                  // biased exponent of amax (bf16 = fp32's)
             const int e = bexp == 0 ? -127 : max(bexp - 127 - 8, -127);
             const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // 2^-e
+            const uint64_t inv2 = pack_f32x2(inv, inv);
             uint32_t q[2];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const uint32_t a = w[2 * j], b = w[2 * j + 1];
-                const uint32_t lo = cvt_e4m3x2(__fmul_rn(__uint_as_float(a << 16), inv),
-                                               __fmul_rn(__uint_as_float(a & 0xFFFF0000u), inv));
-                const uint32_t hi = cvt_e4m3x2(__fmul_rn(__uint_as_float(b << 16), inv),
-                                               __fmul_rn(__uint_as_float(b & 0xFFFF0000u), inv));
-                q[j] = lo | (hi << 16);
+                float p0, p1, p2, p3;
+                unpack_f32x2(mul_f32x2(bf16x2_to_f32x2(w[2 * j]), inv2), p0, p1);
+                unpack_f32x2(mul_f32x2(bf16x2_to_f32x2(w[2 * j + 1]), inv2), p2, p3);
+                q[j] = cvt_e4m3x2(p0, p1) | (cvt_e4m3x2(p2, p3) << 16);
             }
             if (row < M && col < K)
                 *reinterpret_cast<uint2*>(codes + row * K + col) = make_uint2(q[0], q[1]);
@@ -120,11 +128,12 @@ extern "C" int svdq_quantize_mxfp8(const void* X, int64_t M, int64_t K, int64_t 
         return SVDQ_ERR_MISALIGNED;
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
     const int64_t rows_pad = (M + 127) / 128 * 128;
-    const int64_t units = rows_pad * ((K + 255) / 256);
+    const int64_t units = rows_pad * ((K + 255) / 256);            // 256-element row segments
+    if (units > 0x7FFFFFFFLL) return SVDQ_ERR_UNSUPPORTED;
     const int64_t warps_needed = (units + kMxSegs - 1) / kMxSegs;
     const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
     const int64_t blocks = std::min<int64_t>((warps_needed + 7) / 8, static_cast<int64_t>(sms) * 8);
     mx_quantize_kernel<<<static_cast<unsigned>(blocks), kMxThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint16_t*>(X), M, K, ldx, rows_pad, codes, sf);
+        static_cast<const uint16_t*>(X), M, K, ldx, static_cast<uint32_t>(units), codes, sf);
     return launch_status(cudaGetLastError());
 }
