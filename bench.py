@@ -40,7 +40,7 @@ FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (
 # DRAM bytes (read + write) per launch from one ncu capture of the current kernels on this
 # workload (profiles/linear_kernel_*.md, profiles/quantize_act_kernel_*.md); set to None
 # whenever the kernel changes until it is captured again.
-LINEAR_TRAFFIC_BYTES = 27.45e6 + 2.43e6
+LINEAR_TRAFFIC_BYTES = 27.45e6 + 0.68e6      # ncu dram read + write per launch (launch-list capture)
 QUANTIZE_TRAFFIC_BYTES = 42.32e6 + 0.11e6
 
 
