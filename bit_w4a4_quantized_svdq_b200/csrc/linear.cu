@@ -61,6 +61,8 @@ constexpr int kSfWarp0 = 3;                   // warps 3..6 write block scales i
 constexpr int kSfWarps = 4;
 constexpr int kEpiWarp0 = 7;                  // warps 7..14: epilogue
 constexpr int kEpiWarps = 8;
+static_assert(kSfWarp0 == 3 && kSfWarp0 + kSfWarps == kEpiWarp0 && kEpiWarp0 + kEpiWarps == kThreads / 32,
+              "warp roles: 0 producer, 1 MMA issuer, 2 low-rank builder, 3..6 scale writers, 7..14 epilogue");
 
 constexpr uint32_t kATile = kBM * kBKBytes;          // 16 KB
 constexpr uint32_t kBTile = kBN * kBKBytes;          // 32 KB
@@ -846,9 +848,7 @@ int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMa
     auto kern = linear_kernel<kOutF32, kScore, kMx>;
     static std::atomic<uint64_t> smem_set{0};
     if (!set_dynamic_smem_once(kern, smem, smem_set)) return SVDQ_ERR_CUDA;
-    const int tiles = a.m_tiles * a.n_tiles;
     const int grid = linear_grid(a.m_tiles, a.n_tiles);
-    (void)tiles;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);

@@ -20,6 +20,16 @@
  *     per-token activation quantisation, one fused kernel.
  *   - "DeltaQuant on MiniMax-H3", section "The activation scale bound held":
  *     static activation global scale from a bound, saturated groups counted.
+ *   - "MiniMax-H3 -- MXFP8 (weight-quantized, vLLM-Omni native layout)",
+ *     section "Quant format": the MXFP8 W8A8 variant (E4M3 values, one E8M0
+ *     scale per 32 elements).
+ *
+ * Entry points: the hot path svdq_calib_lambda -> svdq_quantize_act ->
+ * svdq_linear -> svdq_score_lambda; svdq_linear_score (the linear with the
+ * scoring in its epilogue); svdq_lambda_grid and svdq_bits_lost (lambda
+ * candidates and the statistics-only proxy); svdq_quantize_mxfp8 and
+ * svdq_linear_mxfp8 (MXFP8 variant); svdq_residual (offline weight
+ * conversion); sizes, status strings and svdq_device_error.
  *
  * Conventions for every call
  *   - All pointers marked "device" are CUDA device pointers owned by the
