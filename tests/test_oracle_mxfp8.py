@@ -80,3 +80,29 @@ def test_linear_on_representable_inputs_is_a_plain_matmul():
     np.testing.assert_array_equal(O.mx_linear(a_c, a_s, w_c, w_s, None), a @ w.T)
     b = _bits(rng.standard_normal(40))
     np.testing.assert_array_equal(O.mx_linear(a_c, a_s, w_c, w_s, b), a @ w.T + O.bf16_to_f64(b)[None, :])
+
+
+def _golden_mx_blocks():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "mxfp8_blocks.txt")
+    rows = []
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        vals, scale, codes = (part.split() for part in line.split("|"))
+        parse = lambda t: float.fromhex(t) if "0x" in t else float(t)
+        rows.append((np.array([parse(t) for t in vals], dtype=np.float32), int(scale[0], 16),
+                     np.array([int(c, 16) for c in codes], dtype=np.uint8)))
+    return rows
+
+
+def test_golden_hand_worked_blocks():
+    rows = _golden_mx_blocks()
+    assert len(rows) == 4
+    for x, scale, codes in rows:
+        bits = S.f32_to_bf16_bits(x)
+        np.testing.assert_array_equal(S.bf16_bits_to_f32(bits).astype(np.float32), x)   # the values are exact bf16
+        got_codes, got_scale = O.mx_quantize(bits[None, :])
+        assert int(got_scale[0, 0]) == scale
+        np.testing.assert_array_equal(got_codes[0], codes)
