@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -38,7 +39,7 @@ CONFIG_INDEX = 1
 L2_FLUSH_BYTES = 256 << 20
 FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
 # DRAM bytes (read + write) per launch from one ncu capture of the current kernels on this
-# workload (profiles/linear_kernel_*.md, profiles/quantize_act_kernel_*.md); set to None
+# workload (the kernels' ncu summaries under profiles/); set to None
 # whenever the kernel changes until it is captured again.
 LINEAR_TRAFFIC_BYTES = 27.45e6 + 0.68e6      # ncu dram read + write per launch (launch-list capture)
 QUANTIZE_TRAFFIC_BYTES = 42.32e6 + 0.11e6
@@ -85,7 +86,7 @@ class ClockSampler:
 
     def __init__(self, index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"svdq_bench_clocks_rank{index}.csv")
         self.index = index
 
     def start(self):

@@ -32,7 +32,7 @@ Pages are cited by title and section.
 * The number formats (E2M1 codes, one E4M3 scale per 16 elements, one FP32
   tensor scale) are those the pages name for NVFP4.
 
-Readings where the pages are silent (each repeated in the design doc):
+Readings where the pages are silent:
   R1 E2M1 rounding is round-to-nearest, ties to the even code, magnitudes
      above 6 saturate to 6, the sign bit is always kept (so -0.1 -> code 0x8).
   R2 The E4M3 block scale is the round-to-nearest-even encoding of
