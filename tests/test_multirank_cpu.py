@@ -57,3 +57,22 @@ def test_two_ranks_take_the_slowest_time(local_ms):
 def test_single_process_is_its_own_maximum():
     assert bench.max_over_ranks(0.123) == 0.123
     assert bench.whole_job_tflops(2.0e11, 1, 0.1) == pytest.approx(2000.0)
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    # `bench.py --impl reference` launched as two ranks: rank 0 runs the oracle arm
+    # and prints the one JSON line, the other rank exits 0 without work
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"]
+    res = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, res.stdout[-2000:]
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
