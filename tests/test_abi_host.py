@@ -164,3 +164,17 @@ def test_mxfp8_sizes_and_bad_arguments():
     assert lib.svdq_linear_mxfp8(p, p, p, p, None, None, 256, 4, 256, 128, None) == _lib.SVDQ_ERR_INVALID_ARG
     assert lib.svdq_linear_mxfp8(p, p, p, p, None, p, 256, 4, 256, 192, None) == _lib.SVDQ_ERR_UNSUPPORTED
     assert lib.svdq_linear_mxfp8(p, p, p, p, None, p, 256, 4, 200, 128, None) == _lib.SVDQ_ERR_UNSUPPORTED
+
+
+def test_missing_library_fails_loudly():
+    # the CUDA library is the only implementation: without it every call raises
+    # instead of falling back to anything else (fresh interpreter: the handle is cached)
+    import subprocess
+    import sys
+    code = ("import sys; sys.path.insert(0, '.');"
+            "from bit_w4a4_quantized_svdq_b200 import _lib\n"
+            "try:\n    _lib.load('/nonexistent/libsvdq.so')\nexcept ImportError as e:\n"
+            "    print('raised', 'build it' in str(e))\nelse:\n    print('loaded')")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert res.stdout.strip() == "raised True", res.stdout + res.stderr
