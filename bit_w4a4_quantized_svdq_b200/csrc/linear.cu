@@ -36,6 +36,17 @@
 // The low-rank MMAs close each tile, so their operand area doubles as the
 // epilogue's output staging: builder -> MMA -> epilogue -> builder.
 //
+// Instantiations (linear_kernel<out fp32, score, MXFP8>):
+//   <0|1, 0, 0>  svdq_linear: the NVFP4 linear, bf16 or fp32 output
+//   <0, 1, 0>    svdq_linear_score: the same, with the tile scored against a bf16
+//                reference in the epilogue (reference strips by TMA into the low-rank
+//                area, per-row exact fp32 pair sums, per-segment fp64 sums, a grid
+//                barrier and a final sum in CTA order); writing Y is optional
+//   <0, 0, 1>    svdq_linear_mxfp8: E4M3 operands with E8M0 scales per 32 on
+//                kind::mxf8f6f4 MMAs; 128 channels per stage, one scale atom per 128
+//                rows per stage serving its four K = 32 MMAs through the scale ids;
+//                no tensor scales, no low-rank branch
+//
 // What paces the main loop (measured on B200 with a stripped main-loop kernel):
 // the tensor pipe keeps only a short queue, so every instruction the issuing
 // thread runs between MMAs shows up as idle tensor cycles (hence one barrier
