@@ -3,9 +3,16 @@
 Argument marshalling only: torch tensors provide device memory and the
 current CUDA stream; every computation runs in ``libsvdq.so``.  bf16 tensors
 may be ``torch.bfloat16`` or raw ``int16``/``uint16`` bit patterns.
+
+Every call runs on the device that holds its tensors: all tensor arguments
+must share one CUDA device, which is made current for the call (the library
+looks up its per-device state -- error word, SM count, static arrays -- on the
+current device), and the default stream is that device's current stream.
 """
 from __future__ import annotations
 
+import functools
+import inspect
 from ctypes import byref, c_uint32
 from typing import Optional, Sequence, Tuple
 
@@ -14,6 +21,47 @@ import torch
 from . import _lib
 
 Segs = Optional[Sequence[Tuple[int, int]]]
+
+
+def _tensors_in(v):
+    if isinstance(v, torch.Tensor):
+        yield v
+    elif isinstance(v, dict):
+        for x in v.values():
+            yield from _tensors_in(x)
+    elif isinstance(v, (list, tuple)):
+        for x in v:
+            yield from _tensors_in(x)
+
+
+def _on_tensor_device(fn):
+    """Run ``fn`` with the device of its tensor arguments current.
+
+    Raises ValueError when the tensors sit on more than one device, on a
+    non-CUDA device, or when an explicit stream belongs to another device."""
+    params = list(inspect.signature(fn).parameters)
+    stream_pos = params.index("stream") if "stream" in params else None
+
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        devs = {t.device for a in (*args, *kwargs.values()) for t in _tensors_in(a)}
+        if not devs:
+            return fn(*args, **kwargs)
+        if len(devs) > 1:
+            names = ", ".join(sorted(str(d) for d in devs))
+            raise ValueError(f"{fn.__name__}: tensor arguments are on different devices ({names})")
+        dev = devs.pop()
+        if dev.type != "cuda":
+            raise ValueError(f"{fn.__name__}: tensor arguments must be CUDA tensors, got {dev}")
+        stream = kwargs.get("stream")
+        if stream is None and stream_pos is not None and len(args) > stream_pos:
+            stream = args[stream_pos]
+        if stream is not None and stream.device != dev:
+            raise ValueError(f"{fn.__name__}: stream is on {stream.device}, tensors on {dev}")
+        with torch.cuda.device(dev):
+            return fn(*args, **kwargs)
+
+    return wrapper
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -42,6 +90,7 @@ def sf_bytes(rows: int, k: int) -> int:
     return int(_lib.load().svdq_sf_bytes(rows, k))
 
 
+@_on_tensor_device
 def svdq_calib_lambda(x: torch.Tensor, segs: Segs = None, w: Optional[torch.Tensor] = None,
                       stream=None) -> dict:
     """Per-channel absmax, lambda, 1/lambda and the static tensor scale (device tensors)."""
@@ -67,6 +116,7 @@ def svdq_calib_lambda(x: torch.Tensor, segs: Segs = None, w: Optional[torch.Tens
     return dict(amax_x=ax, amax_w=aw, lam=lam, inv_lam=inv, s_g=s_g)
 
 
+@_on_tensor_device
 def svdq_quantize_act(x: torch.Tensor, inv_lambda: Optional[torch.Tensor], s_g: torch.Tensor,
                       down: Optional[torch.Tensor] = None, sat_count: Optional[torch.Tensor] = None,
                       out: Optional[dict] = None, stream=None) -> dict:
@@ -87,6 +137,7 @@ def svdq_quantize_act(x: torch.Tensor, inv_lambda: Optional[torch.Tensor], s_g: 
     return out
 
 
+@_on_tensor_device
 def svdq_linear(a_codes: torch.Tensor, a_sf: torch.Tensor, s_g_act: torch.Tensor, d: Optional[torch.Tensor],
                 w_codes: torch.Tensor, w_sf: torch.Tensor, s_g_w: torch.Tensor, up: Optional[torch.Tensor],
                 bias: Optional[torch.Tensor], out_dtype: torch.dtype = torch.bfloat16,
@@ -111,6 +162,7 @@ def linear_score_workspace_bytes(n_seg: int) -> int:
     return int(_lib.load().svdq_linear_score_workspace_bytes(int(n_seg)))
 
 
+@_on_tensor_device
 def svdq_linear_score(a_codes: torch.Tensor, a_sf: torch.Tensor, s_g_act: torch.Tensor, d: Optional[torch.Tensor],
                       w_codes: torch.Tensor, w_sf: torch.Tensor, s_g_w: torch.Tensor, up: Optional[torch.Tensor],
                       bias: Optional[torch.Tensor], yref: torch.Tensor, segs: Sequence[Tuple[int, int]],
@@ -151,6 +203,7 @@ def score_workspace_bytes(segs: Sequence[Tuple[int, int]], n: int) -> int:
     return int(_lib.load().svdq_score_workspace_bytes(arr, n_seg, n))
 
 
+@_on_tensor_device
 def svdq_score_lambda(yq: torch.Tensor, yref: torch.Tensor, segs: Sequence[Tuple[int, int]],
                       workspace: Optional[torch.Tensor] = None, stream=None):
     """Per-segment (num, den, rel) fp64 device tensors."""
@@ -175,6 +228,7 @@ def svdq_score_lambda(yq: torch.Tensor, yref: torch.Tensor, segs: Sequence[Tuple
     return num, den, rel
 
 
+@_on_tensor_device
 def svdq_score_lambda_static(yq: torch.Tensor, yref: torch.Tensor, segs: Sequence[Tuple[int, int]], stream=None):
     """svdq_score_lambda without a workspace: partial sums in the library's static array."""
     lib = _lib.load()
@@ -194,6 +248,7 @@ def svdq_score_lambda_static(yq: torch.Tensor, yref: torch.Tensor, segs: Sequenc
     return num, den, rel
 
 
+@_on_tensor_device
 def svdq_residual(w: torch.Tensor, lam: Optional[torch.Tensor], down: Optional[torch.Tensor],
                   up: Optional[torch.Tensor], stream=None) -> torch.Tensor:
     """R = bf16(W diag(lambda) - (diag(lambda) down^T up^T)^T), computed in fp64."""
@@ -207,6 +262,7 @@ def svdq_residual(w: torch.Tensor, lam: Optional[torch.Tensor], down: Optional[t
     return out
 
 
+@_on_tensor_device
 def svdq_bits_lost(amax_x: torch.Tensor, inv_lambda: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Mean bits lost to the NVFP4 group scale, fp64 [n_cand, n_mod].
 
@@ -229,6 +285,7 @@ def svdq_bits_lost(amax_x: torch.Tensor, inv_lambda: Optional[torch.Tensor] = No
     return bits
 
 
+@_on_tensor_device
 def svdq_lambda_grid(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: torch.Tensor, stream=None) -> dict:
     """Candidate lambda, 1/lambda [n_alpha, K] and s_g [n_alpha] for every alpha (fp32 device tensors)."""
     lib = _lib.load()
@@ -252,6 +309,7 @@ def mxfp8_sf_bytes(rows: int, k: int) -> int:
     return int(_lib.load().svdq_mxfp8_sf_bytes(rows, k))
 
 
+@_on_tensor_device
 def svdq_quantize_mxfp8(x: torch.Tensor, out: Optional[dict] = None, stream=None) -> dict:
     """bf16 [M, K] -> dict(codes u8 [M, K] E4M3, sf u8 E8M0 scales in the tensor-core layout)."""
     lib = _lib.load()
@@ -268,6 +326,7 @@ def svdq_quantize_mxfp8(x: torch.Tensor, out: Optional[dict] = None, stream=None
     return out
 
 
+@_on_tensor_device
 def svdq_linear_mxfp8(a_codes: torch.Tensor, a_sf: torch.Tensor, w_codes: torch.Tensor, w_sf: torch.Tensor,
                       bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                       stream=None) -> torch.Tensor:

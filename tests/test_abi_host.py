@@ -178,3 +178,23 @@ def test_missing_library_fails_loudly():
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     res = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
     assert res.stdout.strip() == "raised True", res.stdout + res.stderr
+
+
+def test_wrappers_reject_tensors_on_different_devices():
+    """The binding makes the tensors' device current for the call, so tensors
+    split over two devices (or off the GPU) are refused before any launch."""
+    import torch
+
+    from bit_w4a4_quantized_svdq_b200 import ops
+
+    cpu = torch.zeros((4, 8), dtype=torch.uint8)
+    meta = torch.empty((4, 8), dtype=torch.uint8, device="meta")
+    f32 = torch.zeros(1, dtype=torch.float32)
+    with pytest.raises(ValueError, match="different devices"):
+        ops.svdq_linear(cpu, cpu, f32, None, meta, cpu, f32, None, None)
+    with pytest.raises(ValueError, match="different devices"):
+        ops.svdq_score_lambda(cpu.view(torch.int16), meta.view(torch.int16), [(0, 4)])
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        ops.svdq_quantize_act(cpu.view(torch.int16), None, f32)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        ops.svdq_calib_lambda(cpu.view(torch.int16), None, None)
