@@ -1,11 +1,14 @@
 """Benchmark of the SVDQuant-style NVFP4 W4A4 linear on B200.
 
 One step = one pass of the whole hot path over one batch: svdq_calib_lambda
-(absmax over the packed rows), svdq_quantize_act (smooth + NVFP4 + fused
-down-projection), svdq_linear (FP4 tcgen05 GEMM + low-rank + bias) and
-svdq_score_lambda (per-modality rel-L2 against the bf16 layer).  The workload
-is the DiT attention projection: 4096 packed rows (text 29 | video 4039 |
-audio 28), K = N = 5120, rank 32, synthetic seeded data.
+(absmax over the packed rows and the weight, lambda, the static tensor scale),
+svdq_quantize_act (smooth + NVFP4 + fused down-projection), svdq_linear (FP4
+tcgen05 GEMM + low-rank + bias) and svdq_score_lambda (per-modality rel-L2
+against the bf16 layer).  The headline workload is the largest configured
+layer, the FFN down-projection: 16384 packed rows (text 115 | video 16155 |
+audio 114), K = 20480, N = 5120, rank 32, lambda calibrated on all rows,
+synthetic seeded data.  The attention projection (4096 x 5120 x 5120) and the
+FFN up-projection (16384 x 5120 -> 20480) are reported beside it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl svdq|reference]
 
@@ -18,7 +21,6 @@ from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -34,15 +36,25 @@ import numpy as np  # noqa: E402
 
 METRIC = "W4A4 linear TFLOP/s and % of B200 dense-FP4 peak; quantize GB/s vs HBM peak"
 UNIT = "TFLOP/s"
-WORKLOAD = "dit_attention_projection_M4096_K5120_N5120_r32"
-CONFIG_INDEX = 1
+HEADLINE_CONFIG = 3
+WORKLOADS = {
+    0: "tiny_M256_K512_N512_r16",
+    1: "dit_attention_projection_M4096_K5120_N5120_r32",
+    2: "ffn_up_projection_M16384_K5120_N20480_r32",
+    3: "ffn_down_projection_M16384_K20480_N5120_r32",
+}
+SECONDARY_CONFIGS = (1, 2)
+L2_BYTES = 126 << 20
 L2_FLUSH_BYTES = 256 << 20
 FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
-# DRAM bytes (read + write) per launch from one ncu capture of the current kernels on this
-# workload (the kernels' ncu summaries under profiles/); set to None
-# whenever the kernel changes until it is captured again.
-LINEAR_TRAFFIC_BYTES = 27.45e6 + 0.68e6      # ncu dram read + write per launch (launch-list capture)
-QUANTIZE_TRAFFIC_BYTES = 42.32e6 + 0.11e6
+# DRAM bytes (read + write) per launch of the linear on each workload, from one
+# ncu capture of the current kernel (summaries under profiles/); None until the
+# current kernel has been captured on that workload.
+LINEAR_TRAFFIC_BYTES = {}
+QUANTIZE_TRAFFIC_BYTES = {}
+# Our kernels per step: calib (zeroing + stream), quantize, linear, score (one
+# cooperative kernel when rows are back to back).
+LAUNCHES_PER_STEP = 5
 
 
 def read_peaks():
@@ -56,10 +68,10 @@ def read_peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
-def workload_bytes(m, k, n, r, m_cal):
+def workload_bytes(m, k, n, r, m_cal, with_w=True):
     """Algorithmic bytes of the HBM-bound kernels (one launch each)."""
     quant = m * k * 2 + m * k // 2 + m * k // 16 + m * r * 4
-    calib = m_cal * k * 2 + n * k * 2
+    calib = m_cal * k * 2 + (n * k * 2 if with_w else 0)
     score = 2 * m * n * 2
     return dict(quantize=quant, calib=calib, score=score)
 
@@ -166,15 +178,25 @@ class OracleArm:
         return 2.0 * rows * layer.n * layer.k / dt / 1e12, dt, rows
 
 
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     import synthetic as S
 
-    layer = S.make_layer(CONFIG_INDEX)
+    cfg = args.config
+    layer = S.make_layer(cfg)
     arm = OracleArm(layer)
-    rows = 256
+    rows = min(layer.m, 128)
     for _ in range(min(args.warmup, 1)):
         arm.run(8)
     times, vals = [], []
@@ -188,33 +210,29 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "rows_per_step": rows, "note": "CPU oracle on a row sample"},
+        "config": {"workload": WORKLOADS[cfg], "M": layer.m, "K": layer.k, "N": layer.n, "rank": layer.rank,
+                   "rows_per_step": rows, "note": "CPU oracle on a row sample"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{rows} of 4096 rows per step, full K and N"},
+                         "sample": f"{rows} evenly spaced of {layer.m} rows per step, full K and N "
+                                   "(calibration of the sample, quantisation, fp64 W4A4 linear, score)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
     return 0
 
 
-def _oracle_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-        return int(n)
-    except Exception:
-        return os.cpu_count() or 1
-
-
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def _graph_ms(fn, flush, flush_read, reps=10, warmup=3):
-    """Median time of `fn` captured as one CUDA graph, L2 flushed before each replay."""
+def _to_dev(a, dev):
     import torch
-    fn()
-    torch.cuda.synchronize()
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
+
+
+def _capture(fn):
+    """`fn` captured as one CUDA graph (on a side stream, as capture requires)."""
+    import torch
     g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -222,6 +240,15 @@ def _graph_ms(fn, flush, flush_read, reps=10, warmup=3):
         with torch.cuda.graph(g, stream=side):
             fn()
     torch.cuda.current_stream().wait_stream(side)
+    return g
+
+
+def _graph_ms(fn, flush, flush_read, reps=10, warmup=3):
+    """Median time of `fn` captured as one CUDA graph, L2 flushed before each replay."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = _capture(fn)
     for _ in range(warmup):
         g.replay()
     times = []
@@ -238,38 +265,333 @@ def _graph_ms(fn, flush, flush_read, reps=10, warmup=3):
     return float(np.median(times))
 
 
-LARGE_SHAPES = ((2, "ffn_up_projection_M16384_K5120_N20480_r32"), (3, "ffn_down_projection_M16384_K20480_N5120_r32"))
+class Workload:
+    """One configured layer on the device: inputs, the converted layer, the bf16
+    reference output and the step's buffers, plus the step itself."""
 
-
-def largest_shapes(P, S, dev, fp4_peak, flush, flush_read, steps=10, warmup=3):
-    """The fused W4A4 linear on the two largest configured shapes, inputs
-    prepared by the same path (calibration, weight conversion, quantisation);
-    each call is one CUDA graph, timed with CUDA events, L2 flushed before each."""
-    import torch
-    out = {}
-    for cfg, name in LARGE_SHAPES:
+    def __init__(self, P, S, cfg, dev, calib_name="all"):
+        import torch
+        self.P, self.cfg, self.dev = P, cfg, dev
         L = S.make_layer(cfg)
-        x = torch.from_numpy(np.ascontiguousarray(L.x).view(np.int16)).to(dev)
-        w = torch.from_numpy(np.ascontiguousarray(L.w).view(np.int16)).to(dev)
-        bias = torch.from_numpy(np.ascontiguousarray(L.bias).view(np.int16)).to(dev)
-        segs = L.seg_ranges(L.calib_sets["all"])
-        cal = P.svdq_calib_lambda(x, segs, w)
-        lin = P.SVDQW4A4Linear.convert(w, bias, cal, L.rank)
-        q = P.svdq_quantize_act(x, cal["inv_lam"], lin.s_g_act, lin.down)
-        y = torch.empty((L.m, L.n), dtype=torch.bfloat16, device=dev)
-        ms = _graph_ms(lambda: P.svdq_linear(q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf,
-                                             lin.s_g_w, lin.up, lin.bias, out=y), flush, flush_read,
-                       reps=steps, warmup=warmup)
-        flops = 2.0 * L.m * L.n * L.k
-        # accuracy against the bf16 layer (sanity: the same quantity the step scores)
-        yref = torch.matmul(x.view(torch.bfloat16), w.view(torch.bfloat16).t()) + bias.view(torch.bfloat16)
-        rel = float(torch.linalg.vector_norm(y.float() - yref.float()) / torch.linalg.vector_norm(yref.float()))
-        out[name] = {"M": L.m, "K": L.k, "N": L.n, "rank": L.rank, "linear_ms": ms,
-                     "linear_tflops": flops / (ms * 1e-3) / 1e12,
-                     "frac_of_fp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak, "rel_l2_vs_bf16": rel}
-        del x, w, bias, cal, lin, q, y, yref
-        torch.cuda.empty_cache()
-    return out
+        self.layer = L
+        self.m, self.k, self.n, self.r = L.m, L.k, L.n, L.rank
+        self.segs_all = L.seg_ranges(L.calib_sets[calib_name])
+        self.segs_mod = [(s.begin, s.end) for s in L.segments]
+        self.m_cal = sum(e - b for b, e in self.segs_all)
+        self.x = _to_dev(L.x, dev)
+        self.w = _to_dev(L.w, dev)
+        self.bias = _to_dev(L.bias, dev)
+        # offline: calibration and weight conversion, the bf16 reference output
+        cal = P.svdq_calib_lambda(self.x, self.segs_all, self.w)
+        self.lin = P.SVDQW4A4Linear.convert(self.w, self.bias, cal, self.r)
+        self.yref = (torch.matmul(self.x.view(torch.bfloat16), self.w.view(torch.bfloat16).t())
+                     + self.bias.view(torch.bfloat16))
+        m, k, n, r = self.m, self.k, self.n, self.r
+        self.q_out = dict(codes=torch.empty((m, k // 2), dtype=torch.uint8, device=dev),
+                          sf=torch.empty(P.sf_bytes(m, k), dtype=torch.uint8, device=dev),
+                          d=torch.empty((m, r), dtype=torch.float32, device=dev))
+        self.y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        self.ws = torch.empty(P.score_workspace_bytes(self.segs_mod, n), dtype=torch.uint8, device=dev)
+        self.flops = 2.0 * m * n * k
+
+    # the four calls of the step (eager; also what the graphs capture)
+    def calib(self, xx):
+        return self.P.svdq_calib_lambda(xx, self.segs_all, self.w)
+
+    def quantize(self, xx, cal):
+        lin = self.lin
+        return self.P.svdq_quantize_act(xx, cal["inv_lam"], lin.s_g_act, lin.down, out=self.q_out)
+
+    def linear(self, q, y):
+        lin = self.lin
+        return self.P.svdq_linear(q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf, lin.s_g_w,
+                                  lin.up, lin.bias, out=y)
+
+    def score(self, y):
+        return self.P.svdq_score_lambda(y, self.yref, self.segs_mod, workspace=self.ws)
+
+    def step(self, xx, y=None):
+        y = self.y if y is None else y
+        cal = self.calib(xx)
+        q = self.quantize(xx, cal)
+        self.linear(q, y)
+        return self.score(y)
+
+    def kernel_times(self, flush, flush_read, reps):
+        """Each call of the step as its own CUDA graph, timed from a cold L2."""
+        x = self.x
+        cal = self.calib(x)
+        q = self.quantize(x, cal)
+        out = {}
+        out["calib"] = _graph_ms(lambda: self.calib(x), flush, flush_read, reps)
+        out["quantize"] = _graph_ms(lambda: self.quantize(x, cal), flush, flush_read, reps)
+        out["linear"] = _graph_ms(lambda: self.linear(q, self.y), flush, flush_read, reps)
+        out["score"] = _graph_ms(lambda: self.score(self.y), flush, flush_read, reps)
+        return out
+
+    def fractions(self, kern_ms, peaks):
+        fp4_peak = peaks["bf16"] * FP4_PER_BF16
+        by = workload_bytes(self.m, self.k, self.n, self.r, self.m_cal)
+        lin_tflops = self.flops / (kern_ms["linear"] * 1e-3) / 1e12
+        rates = {name: by[name] / (kern_ms[name] * 1e-3) / 1e9 for name in ("calib", "quantize", "score")}
+        return {
+            "kernels_ms": kern_ms,
+            "linear_tflops": lin_tflops, "linear_frac_of_fp4_peak": lin_tflops / fp4_peak,
+            "gbs": rates, "frac_of_hbm": {k: v / peaks["hbm"] for k, v in rates.items()},
+            "algorithmic_bytes": by,
+        }
+
+
+def time_step(wl, steps, warmup, flush=None, flush_read=None, world=1):
+    """ms per step of the whole step captured as one CUDA graph.  With flush
+    buffers, the L2 is flushed before every step outside the events (per-step
+    events, mean); without, the steps run back to back between one pair of events."""
+    import torch
+    import torch.distributed as dist
+    g = _capture(lambda: wl.step(wl.x))
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+    else:
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            flush_read.sum()
+            evs[i][0].record()
+            g.replay()
+            evs[i][1].record()
+        torch.cuda.synchronize()
+        ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    if world > 1:
+        dist.barrier()
+    del g
+    return ms
+
+
+def time_e2e(wl, steps, warmup, world=1):
+    """The same step end to end through the public API: every step copies its
+    activations from pinned host memory to the device and its result (Y, bf16
+    [M, N]) and per-modality rel-L2 back.  Copies run on their own streams,
+    double-buffered, so step i's compute overlaps step i+1's upload and step i-1's
+    download.  Returns (ms per step, h2d bytes, d2h bytes, rel of the last step)."""
+    import torch
+    import torch.distributed as dist
+    x_host = torch.from_numpy(np.ascontiguousarray(wl.layer.x).view(np.int16)).pin_memory()
+    x_devs = [torch.empty_like(wl.x) for _ in range(2)]
+    y_devs = [torch.empty_like(wl.y) for _ in range(2)]
+    y_host = [torch.empty(wl.y.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    n_seg = len(wl.segs_mod)
+    rel_host = [torch.empty(n_seg, dtype=torch.float64).pin_memory() for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    copied = [torch.cuda.Event() for _ in range(2)]
+    consumed = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    drained = [torch.cuda.Event() for _ in range(2)]
+
+    def upload(i):
+        b = i % 2
+        with torch.cuda.stream(h2d):
+            if i >= 2:
+                h2d.wait_event(consumed[b])          # step i - 2 has finished reading x_devs[b]
+            x_devs[b].copy_(x_host, non_blocking=True)
+            copied[b].record(h2d)
+
+    def compute(i):
+        b = i % 2
+        comp.wait_event(copied[b])
+        if i >= 2:
+            comp.wait_event(drained[b])              # step i - 2's output has left y_devs[b]
+        res = wl.step(x_devs[b], y_devs[b])
+        consumed[b].record(comp)
+        computed[b].record(comp)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(computed[b])
+            y_host[b].copy_(y_devs[b], non_blocking=True)
+            rel_host[b].copy_(res[2], non_blocking=True)
+            res[2].record_stream(d2h)                # allocated on the compute stream, read here
+            drained[b].record(d2h)
+
+    def pipeline(n, start=None):
+        if start is not None:
+            h2d.wait_event(start)
+        upload(0)
+        for i in range(n):
+            if i + 1 < n:
+                upload(i + 1)
+            compute(i)
+        comp.wait_event(drained[(n - 1) % 2])
+
+    pipeline(max(2, warmup))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    pipeline(steps, start=e0)
+    e1.record(comp)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    last = (steps - 1) % 2
+    rel = rel_host[last].tolist()
+    # the output that came back to the host is the layer's output of the device-timed step
+    same = bool(torch.equal(y_host[last].view(torch.int16), wl.y.cpu().view(torch.int16)))
+    h2d_bytes = wl.x.numel() * 2
+    d2h_bytes = wl.y.numel() * 2 + 8 * n_seg
+    del x_host, x_devs, y_devs, y_host
+    return ms, h2d_bytes, d2h_bytes, rel, same
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    import bit_w4a4_quantized_svdq_b200 as P
+    import synthetic as S
+
+    peaks = read_peaks()
+    fp4_peak = peaks["bf16"] * FP4_PER_BF16
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_read = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    cfg = args.config
+    wl = Workload(P, S, cfg, dev)
+    m, k, n, r = wl.m, wl.k, wl.n, wl.r
+    for _ in range(args.warmup):
+        wl.step(wl.x)
+    torch.cuda.synchronize()
+    eager_rel = wl.step(wl.x)[2].cpu()
+
+    # ---- device-timed region: inputs resident in HBM.  Inputs larger than L2
+    # run back to back; smaller ones get an L2 flush before every step.
+    big = wl.x.numel() * 2 > L2_BYTES and wl.w.numel() * 2 > L2_BYTES
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    step_ms = time_step(wl, args.steps, args.warmup, None if big else flush, None if big else flush_read, world)
+    clocks = sampler.stop()
+    step_ms_max = max_over_ranks(step_ms, dev)
+    value = whole_job_tflops(wl.flops, world, step_ms_max)
+    graph_rel = wl.score(wl.y)[2].cpu()
+    graph_matches_eager = bool(torch.equal(graph_rel, eager_rel))
+
+    # per-call breakdown (each call one graph, cold L2) and the roofline figures
+    kern = wl.kernel_times(flush, flush_read, reps=max(5, min(args.steps, 20)))
+    fr = wl.fractions(kern, peaks)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d_b, d2h_b, rel, same = time_e2e(wl, args.steps, args.warmup, world)
+        e2e_ms_max = max_over_ranks(e2e_ms, dev)
+        e2e = {"value": whole_job_tflops(wl.flops, world, e2e_ms_max), "unit": UNIT, "ms_per_step": e2e_ms_max,
+               "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b, "output_matches_device_step": same,
+               "how": "public API, eager calls; each step copies X from pinned host memory to the device and "
+                      "Y (bf16) plus the per-modality rel-L2 back to pinned host memory, the copies on their own "
+                      "streams overlapping the neighbouring steps' compute (two device buffers each way)"}
+    else:
+        rel = eager_rel.tolist()
+    err = P.svdq_device_error()
+
+    names = [s.name for s in wl.layer.segments]
+    layer = wl.layer
+    del wl
+    torch.cuda.empty_cache()
+
+    # ---- the other configured layers (1 GPU only): the step and its calls
+    others = {}
+    if world == 1 and not args.no_secondary:
+        for c2 in SECONDARY_CONFIGS:
+            if c2 == cfg:
+                continue
+            w2 = Workload(P, S, c2, dev)
+            big2 = w2.x.numel() * 2 > L2_BYTES and w2.w.numel() * 2 > L2_BYTES
+            ms2 = time_step(w2, max(10, min(args.steps, 20)), args.warmup, None if big2 else flush,
+                            None if big2 else flush_read)
+            k2 = w2.kernel_times(flush, flush_read, reps=10)
+            f2 = w2.fractions(k2, peaks)
+            others[WORKLOADS[c2]] = {"M": w2.m, "K": w2.k, "N": w2.n, "rank": w2.r, "ms_per_step": ms2,
+                                     "tflops_per_step": w2.flops / (ms2 * 1e-3) / 1e12,
+                                     "l2": "back to back (inputs larger than L2)" if big2 else
+                                           "flushed before every step", **f2}
+            del w2
+            torch.cuda.empty_cache()
+    per_config = None
+    if world == 1 and args.all_configs:
+        per_config = all_configs(P, S, dev, fp4_peak, peaks["hbm"], flush, flush_read)
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            # a bounded row sample of the same workload: about 10-20 s of host work
+            arm = OracleArm(layer)
+            rows = min(layer.m, 384)
+            runs = [arm.run(rows) for _ in range(2)]
+            dt = sum(x[1] for x in runs)
+            cpu = {"value": 2 * 2.0 * rows * n * k / dt / 1e12, "unit": UNIT, "cores": _oracle_threads(),
+                   "kind": "oracle",
+                   "sample": f"{rows} evenly spaced of the {m} rows, full K={k} and N={n}, twice ({dt:.1f} s): "
+                             "calibration of the sample, quantisation, the W4A4 linear in fp64, scores"}
+        lin_tflops = fr["linear_tflops"]
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) -> fp32 accum, bf16 out", "data": "synthetic",
+            "config": {"workload": WORKLOADS[cfg], "M": m, "K": k, "N": n, "rank": r, "rows_per_gpu": m,
+                       "lambda": "calibrated on all rows",
+                       "segments": {s.name: [s.begin, s.end] for s in layer.segments},
+                       "parallelism": f"replicas x{world}",
+                       "l2": ("inputs larger than L2 (X %d MB, W %d MB vs 126 MB): steps back to back" %
+                              (m * k * 2 // 10**6, n * k * 2 // 10**6)) if big else
+                             "flushed between steps: 256 MiB write, then 256 MiB read (cold, clean L2)",
+                       "timing": "the step (calib + quantize + linear + score) as one CUDA graph, CUDA events "
+                                 "around the K replays; kernels_ms from one graph per call, cold L2"},
+            **fr,
+            "roofline": {"bound": "tensor", "kernel": "svdq_linear", "achieved": lin_tflops, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": lin_tflops / fp4_peak,
+                         "traffic": LINEAR_TRAFFIC_BYTES.get(cfg),
+                         "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} x {FP4_PER_BF16:g} "
+                                        "(nominal dense FP4/BF16 ratio)"},
+            "roofline_hbm": {"bound": "hbm", "kernel": "svdq_quantize_act", "achieved": fr["gbs"]["quantize"],
+                             "peak": peaks["hbm"], "unit": "GB/s", "frac": fr["frac_of_hbm"]["quantize"],
+                             "traffic": QUANTIZE_TRAFFIC_BYTES.get(cfg),
+                             "peak_source": f"{peaks['source']} copy bandwidth"},
+            "e2e": e2e,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clocks,
+            "rel_l2_vs_bf16": dict(zip(names, rel)),
+            "device_error": err,
+            "graph_replay_matches_eager": graph_matches_eager,
+            "other_configs": others or None,
+            "all_configs": per_config,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
 
 
 def all_configs(P, S, dev, fp4_peak, hbm_peak, flush, flush_read):
@@ -278,7 +600,7 @@ def all_configs(P, S, dev, fp4_peak, hbm_peak, flush, flush_read):
     import torch
 
     def to_dev(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
+        return _to_dev(a, dev)
 
     def layer_calls(L, calib_name):
         x, w, bias = to_dev(L.x), to_dev(L.w), to_dev(L.bias)
@@ -362,11 +684,10 @@ def lambda_search(P, S, dev, flush, flush_read):
     """The 39-candidate lambda search on one sweep layer (rank 32, three modalities):
     wall time of the whole search (host-driven; the randomized rank-32 factorisation of
     every candidate is library QR/SVD), and the grid and bits-lost kernels timed alone."""
-    import time
     import torch
 
     def to_dev(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
+        return _to_dev(a, dev)
 
     L = S.make_layer(4, layer=0)
     x, w, bias = to_dev(L.x), to_dev(L.w), to_dev(L.bias)
@@ -396,9 +717,12 @@ def lambda_search(P, S, dev, flush, flush_read):
         "bits_lost_best": dict(zip(names, res["bits"][res["best"]].cpu().tolist()))}}
 
 
-def profile_case(name: str) -> int:
-    """A few launches of one kernel on the attention-projection workload, for a profiler:
-    two warm-up launches, then three (capture with -s 2 -c 1..3 on the kernel's name)."""
+PROFILE_CASES = ("step", "calib", "quantize", "linear", "score", "linear_score", "mxfp8_linear", "mxfp8_quantize")
+
+
+def profile_case(name: str, cfg: int) -> int:
+    """A few launches of one call on one configured workload, for a profiler: two
+    warm-up launches, then three (capture with -s 2 -c 1..3 on the kernel's name)."""
     import torch
 
     import bit_w4a4_quantized_svdq_b200 as P
@@ -406,22 +730,9 @@ def profile_case(name: str) -> int:
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    L = S.make_layer(CONFIG_INDEX)
-
-    def to_dev(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
-
-    x, w, bias = to_dev(L.x), to_dev(L.w), to_dev(L.bias)
-    segs_mod = [(sg.begin, sg.end) for sg in L.segments]
-    if name == "linear_score":
-        cal = P.svdq_calib_lambda(x, L.seg_ranges(L.calib_sets["all"]), w)
-        lin = P.SVDQW4A4Linear.convert(w, bias, cal, L.rank)
-        q = P.svdq_quantize_act(x, cal["inv_lam"], lin.s_g_act, lin.down)
-        yref = x.view(torch.bfloat16) @ w.view(torch.bfloat16).t() + bias.view(torch.bfloat16)
-        wf = torch.empty(P.linear_score_workspace_bytes(len(segs_mod)), dtype=torch.uint8, device=dev)
-        args = (q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf, lin.s_g_w, lin.up, lin.bias)
-        run = lambda: P.svdq_linear_score(*args, yref=yref, segs=segs_mod, write_out=False, workspace=wf)
-    elif name in ("mxfp8_linear", "mxfp8_quantize"):
+    if name in ("mxfp8_linear", "mxfp8_quantize"):
+        L = S.make_layer(cfg)
+        x, w, bias = _to_dev(L.x, dev), _to_dev(L.w, dev), _to_dev(L.bias, dev)
         qa = P.svdq_quantize_mxfp8(x)
         qw = P.svdq_quantize_mxfp8(w)
         y = torch.empty((L.m, L.n), dtype=torch.bfloat16, device=dev)
@@ -430,259 +741,30 @@ def profile_case(name: str) -> int:
         else:
             run = lambda: P.svdq_quantize_mxfp8(x, out=qa)
     else:
-        raise SystemExit(f"unknown profile case {name}")
+        wl = Workload(P, S, cfg, dev)
+        cal = wl.calib(wl.x)
+        q = wl.quantize(wl.x, cal)
+        if name == "step":
+            run = lambda: wl.step(wl.x)
+        elif name == "calib":
+            run = lambda: wl.calib(wl.x)
+        elif name == "quantize":
+            run = lambda: wl.quantize(wl.x, cal)
+        elif name == "linear":
+            run = lambda: wl.linear(q, wl.y)
+        elif name == "score":
+            run = lambda: wl.score(wl.y)
+        else:
+            wf = torch.empty(P.linear_score_workspace_bytes(len(wl.segs_mod)), dtype=torch.uint8, device=dev)
+            lin = wl.lin
+            args = (q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf, lin.s_g_w, lin.up, lin.bias)
+            run = lambda: P.svdq_linear_score(*args, yref=wl.yref, segs=wl.segs_mod, write_out=False, workspace=wf)
     torch.cuda.synchronize()
     for _ in range(5):
         run()
     torch.cuda.synchronize()
     assert P.svdq_device_error() == 0
-    print(json.dumps({"profile_case": name, "launches": 5}))
-    return 0
-
-
-def run_gpu(args):
-    import torch
-    import torch.distributed as dist
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-
-    import bit_w4a4_quantized_svdq_b200 as P
-    import synthetic as S
-
-    layer = S.make_layer(CONFIG_INDEX)
-    m, k, n, r = layer.m, layer.k, layer.n, layer.rank
-    segs_all = layer.seg_ranges(layer.calib_sets["all"])
-    segs_mod = [(s.begin, s.end) for s in layer.segments]
-
-    def dev_bits(b):
-        return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev)
-
-    x = dev_bits(layer.x)
-    w = dev_bits(layer.w)
-    bias = dev_bits(layer.bias)
-    # offline: calibration and weight conversion, the bf16 reference output
-    calib = P.svdq_calib_lambda(x, segs_all, w)
-    lin = P.SVDQW4A4Linear.convert(w, bias, calib, r)
-    yref = torch.matmul(x.view(torch.bfloat16), w.view(torch.bfloat16).t()) + bias.view(torch.bfloat16)
-    q_out = dict(codes=torch.empty((m, k // 2), dtype=torch.uint8, device=dev),
-                 sf=torch.empty(P.sf_bytes(m, k), dtype=torch.uint8, device=dev),
-                 d=torch.empty((m, r), dtype=torch.float32, device=dev))
-    y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(P.score_workspace_bytes(segs_mod, n), dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    flush_read = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
-
-    def step(xx, ev=None):
-        if ev is not None:
-            ev[0].record()
-        cal = P.svdq_calib_lambda(xx, segs_all, w)
-        if ev is not None:
-            ev[1].record()
-        q = P.svdq_quantize_act(xx, cal["inv_lam"], lin.s_g_act, lin.down, out=q_out)
-        if ev is not None:
-            ev[2].record()
-        P.svdq_linear(q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf, lin.s_g_w, lin.up,
-                      lin.bias, out=y)
-        if ev is not None:
-            ev[3].record()
-        res = P.svdq_score_lambda(y, yref, segs_mod, workspace=ws)
-        if ev is not None:
-            ev[4].record()
-        return res
-
-    # calib (zero + reduce), quantize, linear, score (one cooperative kernel; rows are back to back)
-    launches_per_step = 2 + 1 + 1 + 1
-    for _ in range(args.warmup):
-        step(x)
-    torch.cuda.synchronize()
-
-    # One CUDA graph per call of the step, so the device-timed region measures
-    # the kernels and not the host-side argument marshalling between them.
-    graphs = [torch.cuda.CUDAGraph() for _ in range(4)]
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        with torch.cuda.graph(graphs[0], stream=side):
-            g_cal = P.svdq_calib_lambda(x, segs_all, w)
-        with torch.cuda.graph(graphs[1], stream=side, pool=graphs[0].pool()):
-            P.svdq_quantize_act(x, g_cal["inv_lam"], lin.s_g_act, lin.down, out=q_out)
-        with torch.cuda.graph(graphs[2], stream=side, pool=graphs[0].pool()):
-            P.svdq_linear(q_out["codes"], q_out["sf"], lin.s_g_act, q_out["d"], lin.w_codes, lin.w_sf, lin.s_g_w,
-                          lin.up, lin.bias, out=y)
-        with torch.cuda.graph(graphs[3], stream=side, pool=graphs[0].pool()):
-            g_res = P.svdq_score_lambda(y, yref, segs_mod, workspace=ws)
-        # the whole step (calib -> quantize -> linear -> score) as one graph
-        g_step = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_step, stream=side, pool=graphs[0].pool()):
-            s_cal = P.svdq_calib_lambda(x, segs_all, w)
-            P.svdq_quantize_act(x, s_cal["inv_lam"], lin.s_g_act, lin.down, out=q_out)
-            P.svdq_linear(q_out["codes"], q_out["sf"], lin.s_g_act, q_out["d"], lin.w_codes, lin.w_sf, lin.s_g_w,
-                          lin.up, lin.bias, out=y)
-            s_res = P.svdq_score_lambda(y, yref, segs_mod, workspace=ws)
-    torch.cuda.current_stream().wait_stream(side)
-    for _ in range(args.warmup):
-        g_step.replay()
-        for g in graphs:
-            g.replay()
-    torch.cuda.synchronize()
-
-    # ---- device-timed region: inputs resident in HBM, L2 flushed between steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.3)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    step_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        # L2 flush between steps, outside the events: write a buffer larger than
-        # L2, then read another one so the write-back of the dirty lines happens
-        # here and every step starts from a cold, clean L2.
-        flush.fill_(i & 0xFF)
-        flush_read.sum()
-        step_evs[i][0].record()
-        g_step.replay()
-        step_evs[i][1].record()
-    # per-call breakdown: the same calls, one graph each, events between them
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        flush_read.sum()
-        evs[i][0].record()
-        for j, g in enumerate(graphs):
-            g.replay()
-            evs[i][j + 1].record()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop()
-    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
-    step_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in step_evs]))
-    kern_ms = per.mean(axis=0)       # calib, quantize, linear, score
-    step_ms_max = max_over_ranks(step_ms, dev)
-
-    flops = 2.0 * m * n * k
-    value = whole_job_tflops(flops, world, step_ms_max)
-    peaks = read_peaks()
-    fp4_peak = peaks["bf16"] * FP4_PER_BF16
-    lin_tflops = flops / (kern_ms[2] * 1e-3) / 1e12
-    by = workload_bytes(m, k, n, r, m)
-    quant_gbs = by["quantize"] / (kern_ms[1] * 1e-3) / 1e9
-    calib_gbs = by["calib"] / (kern_ms[0] * 1e-3) / 1e9
-    score_gbs = by["score"] / (kern_ms[3] * 1e-3) / 1e9
-
-    # ---- end to end through the public layer API with host buffers.  Every
-    # step copies its activations from pinned host memory and reads its scores
-    # back; the copy of step i + 1 runs on a second stream while step i computes
-    # (two device buffers), so the step costs max(copy, compute), not their sum.
-    x_host = torch.from_numpy(np.ascontiguousarray(layer.x).view(np.int16)).pin_memory()
-    x_devs = [torch.empty_like(x), torch.empty_like(x)]
-    rel_host = torch.empty(len(segs_mod), dtype=torch.float64).pin_memory()
-    comp = torch.cuda.current_stream()
-    copy_stream = torch.cuda.Stream()
-    copied = [torch.cuda.Event(), torch.cuda.Event()]
-    consumed = [torch.cuda.Event(), torch.cuda.Event()]
-
-    def issue_copy(i):
-        b = i % 2
-        with torch.cuda.stream(copy_stream):
-            if i >= 2:
-                copy_stream.wait_event(consumed[b])      # step i - 2 has finished reading this buffer
-            x_devs[b].copy_(x_host, non_blocking=True)
-            copied[b].record(copy_stream)
-
-    def run_step(i):
-        b = i % 2
-        comp.wait_event(copied[b])
-        res = step(x_devs[b])
-        consumed[b].record(comp)
-        rel_host.copy_(res[2], non_blocking=True)
-
-    def pipeline(n, start_event=None):
-        if start_event is not None:
-            copy_stream.wait_event(start_event)
-        issue_copy(0)
-        for i in range(n):
-            if i + 1 < n:
-                issue_copy(i + 1)
-            run_step(i)
-
-    pipeline(max(2, args.warmup))
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(comp)
-    pipeline(args.steps, start_event=e0)
-    e1.record(comp)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
-    e2e_value = whole_job_tflops(flops, world, e2e_ms)
-    rel = rel_host.tolist()
-    # the graphs replay the same calls on the same data: same scores, bit for bit
-    graph_matches_eager = bool(torch.equal(g_res[2].cpu(), rel_host) and torch.equal(s_res[2].cpu(), rel_host))
-
-    err = P.svdq_device_error()
-    large = None
-    if world == 1 and not args.no_large:
-        large = largest_shapes(P, S, dev, fp4_peak, flush, flush_read)
-    per_config = None
-    if world == 1 and args.all_configs:
-        per_config = all_configs(P, S, dev, fp4_peak, peaks["hbm"], flush, flush_read)
-    line = None
-    if rank == 0:
-        cpu = None
-        if world == 1 and not args.no_cpu_baseline:
-            # the whole workload (all rows), two passes: about 10 s of host work
-            arm = OracleArm(layer)
-            runs = [arm.run(m) for _ in range(2)]
-            dt = sum(r[1] for r in runs)
-            v = 2 * 2.0 * m * n * k / dt / 1e12
-            cpu = {"value": v, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
-                   "sample": f"the full step (all {m} rows, K={k}, N={n}) twice, {dt:.1f} s"}
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) -> fp32 accum, bf16 out", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": m, "K": k, "N": n, "rank": r, "rows_per_gpu": m,
-                       "segments": {s.name: [s.begin, s.end] for s in layer.segments},
-                       "parallelism": f"replicas x{world}",
-                       "l2": "flushed between steps: 256 MiB write, then 256 MiB read (cold, clean L2)",
-                       "timing": "the step as one CUDA graph, CUDA events around it; kernels_ms from one graph per call"},
-            "kernels_ms": {"calib": kern_ms[0], "quantize": kern_ms[1], "linear": kern_ms[2],
-                           "score": kern_ms[3]},
-            "linear_tflops": lin_tflops, "quantize_gbs": quant_gbs, "calib_gbs": calib_gbs, "score_gbs": score_gbs,
-            "roofline": {"bound": "tensor", "kernel": "svdq_linear", "achieved": lin_tflops, "peak": fp4_peak,
-                         "unit": "TFLOP/s", "frac": lin_tflops / fp4_peak, "traffic": LINEAR_TRAFFIC_BYTES,
-                         "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} x {FP4_PER_BF16:g} "
-                                        "(nominal dense FP4/BF16 ratio)"},
-            "roofline_hbm": {"kernel": "svdq_quantize_act", "achieved": quant_gbs, "peak": peaks["hbm"],
-                             "unit": "GB/s", "frac": quant_gbs / peaks["hbm"], "traffic": QUANTIZE_TRAFFIC_BYTES,
-                             "bound": "hbm"},
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": m * k * 2,
-                    "d2h_bytes_per_step": 8 * len(segs_mod),
-                    "how": "public API, eager calls; each step's activations copied from pinned host memory "
-                           "(the next step's copy overlapped on a second stream), its scores read back"},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks,
-            "rel_l2_vs_bf16": dict(zip([s.name for s in layer.segments], rel)),
-            "device_error": err,
-            "graph_replay_matches_eager": graph_matches_eager,
-            "largest_shapes": large,
-            "all_configs": per_config,
-            "cpu_baseline": cpu,
-        }
-        print(json.dumps(line))
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    print(json.dumps({"profile_case": name, "config": cfg, "launches": 5}))
     return 0
 
 
@@ -692,17 +774,20 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
+    ap.add_argument("--config", type=int, default=HEADLINE_CONFIG, choices=sorted(WORKLOADS),
+                    help="configured workload of the step (default: the FFN down-projection, the largest)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-large", action="store_true", help="skip the two largest-shape GEMM measurements")
-    ap.add_argument("--profile-case", default=None, choices=["linear_score", "mxfp8_linear", "mxfp8_quantize"],
-                    help="only launch one kernel five times on the attention-projection workload (for ncu)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the other configured layers")
+    ap.add_argument("--profile-case", default=None, choices=PROFILE_CASES,
+                    help="only launch one call five times on the --config workload (for ncu)")
     ap.add_argument("--all-configs", action="store_true",
                     help="also time every call on every configured workload (adds a few minutes)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "svdq":
         args.warmup = 3
     if args.profile_case:
-        return profile_case(args.profile_case)
+        return profile_case(args.profile_case, args.config)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)
