@@ -1,7 +1,8 @@
 """Benchmark of the SVDQuant-style NVFP4 W4A4 linear on B200.
 
-One step = one pass of the whole hot path over one batch: svdq_calib_lambda
-(absmax over the packed rows and the weight, lambda, the static tensor scale),
+One step = one pass of the whole hot path over one batch: calibration
+(svdq_calib_lambda_stored_w: absmax over the packed rows, lambda against the
+weight's absmax kept from conversion, 1/lambda, the static tensor scale),
 svdq_quantize_act (smooth + NVFP4 + fused down-projection), svdq_linear (FP4
 tcgen05 GEMM + low-rank + bias) and svdq_score_lambda (per-modality rel-L2
 against the bf16 layer).  The headline workload is the largest configured
@@ -281,8 +282,11 @@ class Workload:
         self.x = _to_dev(L.x, dev)
         self.w = _to_dev(L.w, dev)
         self.bias = _to_dev(L.bias, dev)
-        # offline: calibration and weight conversion, the bf16 reference output
+        # offline: calibration and weight conversion, the bf16 reference output; the
+        # weight's absmax is a constant of the converted layer, kept for the step's
+        # calibration (which then reads X alone)
         cal = P.svdq_calib_lambda(self.x, self.segs_all, self.w)
+        self.amax_w = cal["amax_w"]
         self.lin = P.SVDQW4A4Linear.convert(self.w, self.bias, cal, self.r)
         self.yref = (torch.matmul(self.x.view(torch.bfloat16), self.w.view(torch.bfloat16).t())
                      + self.bias.view(torch.bfloat16))
@@ -296,7 +300,7 @@ class Workload:
 
     # the four calls of the step (eager; also what the graphs capture)
     def calib(self, xx):
-        return self.P.svdq_calib_lambda(xx, self.segs_all, self.w)
+        return self.P.svdq_calib_lambda_stored_w(xx, self.segs_all, self.amax_w)
 
     def quantize(self, xx, cal):
         lin = self.lin
@@ -331,7 +335,7 @@ class Workload:
 
     def fractions(self, kern_ms, peaks):
         fp4_peak = peaks["bf16"] * FP4_PER_BF16
-        by = workload_bytes(self.m, self.k, self.n, self.r, self.m_cal)
+        by = workload_bytes(self.m, self.k, self.n, self.r, self.m_cal, with_w=False)
         lin_tflops = self.flops / (kern_ms["linear"] * 1e-3) / 1e12
         rates = {name: by[name] / (kern_ms[name] * 1e-3) / 1e9 for name in ("calib", "quantize", "score")}
         return {

@@ -7,7 +7,7 @@ call fails with ImportError if it has not been built
 """
 from . import _lib
 from .ops import (linear_score_workspace_bytes, mxfp8_sf_bytes, score_workspace_bytes, sf_bytes,
-                  svdq_bits_lost, svdq_calib_lambda, svdq_device_error, svdq_lambda_grid, svdq_linear,
+                  svdq_bits_lost, svdq_calib_lambda, svdq_calib_lambda_stored_w, svdq_device_error, svdq_lambda_grid, svdq_linear,
                   svdq_linear_mxfp8, svdq_linear_score, svdq_quantize_act, svdq_quantize_mxfp8, svdq_residual,
                   svdq_score_lambda, svdq_score_lambda_static)
 from .layer import SVDQW4A4Linear, alpha_grid, lowrank_factors_device, search_lambda
@@ -19,7 +19,7 @@ def load():
 
 
 __all__ = [
-    "svdq_calib_lambda", "svdq_quantize_act", "svdq_linear", "svdq_linear_score", "svdq_score_lambda",
+    "svdq_calib_lambda", "svdq_calib_lambda_stored_w", "svdq_quantize_act", "svdq_linear", "svdq_linear_score", "svdq_score_lambda",
     "svdq_score_lambda_static", "linear_score_workspace_bytes", "svdq_bits_lost", "svdq_lambda_grid",
     "svdq_quantize_mxfp8", "svdq_linear_mxfp8", "mxfp8_sf_bytes",
     "svdq_residual", "svdq_device_error", "sf_bytes", "score_workspace_bytes", "SVDQW4A4Linear",

@@ -38,6 +38,8 @@ SIGNATURES = {
     "svdq_calib_lambda": (c_int, [c_void_p, c_int64, c_int64, c_int64, POINTER(SvdqSeg), c_int,
                                   c_void_p, c_int64, c_int64,
                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "svdq_calib_lambda_stored_w": (c_int, [c_void_p, c_int64, c_int64, c_int64, POINTER(SvdqSeg), c_int, c_void_p,
+                                           c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "svdq_quantize_act": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p,
                                   c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "svdq_linear": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int,
@@ -52,6 +54,7 @@ SIGNATURES = {
     "svdq_residual": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_int,
                               c_void_p, c_void_p]),
     "svdq_device_error": (c_int, [c_void_p, POINTER(c_uint32)]),
+    "svdq_debug_arm_calib_timeout": (c_int, [c_int64, c_int64]),
     "svdq_linear_score": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_int64, POINTER(SvdqSeg), c_int,
                                   c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_int64, c_int64, c_int64,

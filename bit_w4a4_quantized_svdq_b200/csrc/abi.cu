@@ -13,8 +13,8 @@ __device__ uint32_t g_device_error;
 namespace {
 constexpr int kMaxDevices = 64;
 uint32_t* g_err_ptr[kMaxDevices] = {};
-int g_is_sm100[kMaxDevices] = {};      // 0 unknown, 1 yes, 2 no
-int g_sm_count[kMaxDevices] = {};
+int g_is_sm100[kMaxDevices] = {};      // 0 unknown, 1 yes, 2 no (guarded by g_mutex)
+std::atomic<int> g_sm_count[kMaxDevices] = {};
 std::mutex g_mutex;
 
 int current_device() {
@@ -53,7 +53,7 @@ bool device_is_sm100() {
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         g_is_sm100[dev] = (major == 10 && minor == 0) ? 1 : 2;
-        g_sm_count[dev] = sms;
+        g_sm_count[dev].store(sms, std::memory_order_release);
     }
     return g_is_sm100[dev] == 1;
 }
@@ -61,8 +61,8 @@ bool device_is_sm100() {
 int device_sm_count() {
     const int dev = current_device();
     if (dev < 0) return 0;
-    if (g_sm_count[dev] == 0) device_is_sm100();
-    return g_sm_count[dev];
+    if (g_sm_count[dev].load(std::memory_order_acquire) == 0) device_is_sm100();
+    return g_sm_count[dev].load(std::memory_order_acquire);
 }
 
 static bool load_encoder() {

@@ -63,6 +63,11 @@ struct CalibArgs {
     float* inv_lambda;
     float* s_g;                               // holds max(strip maxima) until the last strip writes the scale
     uint32_t* err;
+    // Time-out test (armed from the host, one call): CTA 0's producer leaves its
+    // ring unit `skip_unit` unloaded, so a consumer's wait for it runs out after
+    // `wait_limit` cycles; -1 = off.  Every other CTA and call runs normally.
+    int64_t skip_unit;
+    long long wait_limit;
 };
 
 __global__ void __launch_bounds__(256)
@@ -168,6 +173,7 @@ calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_launch_dependents();                  // the quantiser's set-up may overlap this kernel
 
     if (a.n_units == 0) {
         // No rows selected and no weight: one CTA per strip forms lambda = 1.
@@ -177,6 +183,8 @@ calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     }
     const int64_t u_begin = g * a.n_units / G;
     const int64_t u_end = (g + 1) * a.n_units / G;
+    const int64_t skip = g == 0 ? a.skip_unit : -1;
+    const long long limit = skip >= 0 ? a.wait_limit : kWaitLimitCycles;
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------ producer
@@ -187,7 +195,8 @@ calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             for (int64_t u = u_begin; u < u_end; ++u, ++i) {
                 const int s = i % kSlots;
                 const uint32_t ph = (i / kSlots) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, a.err, kErrWaitEmpty)) break;
+                if (!mbar_wait_limit(&empty[s], ph ^ 1, abort_flag, a.err, kErrWaitEmpty, limit)) break;
+                if (i == skip) continue;              // time-out test: this unit never arrives
                 const int job = u < a.units[0] ? 0 : 1;
                 const int64_t local = job ? u - a.units[0] : u;
                 const int64_t strip = local / a.boxes[job];
@@ -210,6 +219,7 @@ calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                             static_cast<int32_t>(strip * kStripCols), static_cast<int32_t>(row0));
             }
             for (int j = (i > kSlots ? i - kSlots : 0); j < i; ++j) {   // bounded drain
+                if (j == skip) continue;
                 const long long t0 = clock64();
                 while (!mbar_try_wait(&full[j % kSlots], (j / kSlots) & 1) && clock64() - t0 < kWaitLimitCycles) {}
             }
@@ -256,7 +266,7 @@ calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     for (int64_t u = u_begin; u < u_end; ++u, ++i) {
         const int s = i % kSlots;
         const uint32_t ph = (i / kSlots) & 1;
-        if (!mbar_wait(&full[s], ph, abort_flag, a.err, kErrWaitFull)) break;
+        if (!mbar_wait_limit(&full[s], ph, abort_flag, a.err, kErrWaitFull, limit)) break;
         const uint32_t md = meta[s];
         const int64_t key = (static_cast<int64_t>(md >> 8) << 1) | ((md >> 7) & 1);
         const int valid = static_cast<int>(md & 0x7Fu);
@@ -282,15 +292,29 @@ calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     if (cur >= 0) merge(cur);
 }
 
+// One-shot time-out test arming (see svdq_debug_arm_calib_timeout).
+std::atomic<long long> g_arm_skip{-1};
+std::atomic<long long> g_arm_limit{0};
+
 }  // namespace
 }  // namespace svdq
 
-extern "C" int svdq_calib_lambda(const void* X, int64_t M, int64_t K, int64_t ldx,
-                                 const svdq_seg* segs, int n_seg,
-                                 const void* W, int64_t N, int64_t ldw,
-                                 float* amax_x, float* amax_w, float* lambda, float* inv_lambda,
-                                 float* s_g, void* stream) {
-    using namespace svdq;
+extern "C" int svdq_debug_arm_calib_timeout(int64_t unit, int64_t wait_limit_cycles) {
+    if (unit < 0 || wait_limit_cycles < 100000) return SVDQ_ERR_INVALID_ARG;
+    svdq::g_arm_limit.store(wait_limit_cycles);
+    svdq::g_arm_skip.store(unit);
+    return SVDQ_OK;
+}
+
+namespace svdq {
+namespace {
+
+// Shared by both entry points.  W != NULL: the weight's absmax is reduced into
+// amax_w here.  W == NULL and aw_in != NULL: aw_in is the stored absmax of the
+// weight (an input).  Both NULL: lambda = 1.
+int calib_launch(const void* X, int64_t M, int64_t K, int64_t ldx, const svdq_seg* segs, int n_seg,
+                 const void* W, int64_t N, int64_t ldw, const float* aw_in,
+                 float* amax_x, float* amax_w, float* lambda, float* inv_lambda, float* s_g, void* stream) {
     if (X == nullptr || amax_x == nullptr || lambda == nullptr || s_g == nullptr) return SVDQ_ERR_INVALID_ARG;
     if (M < 1 || K < 8 || K % 8 != 0 || ldx < K) return SVDQ_ERR_INVALID_ARG;
     if (W != nullptr && (amax_w == nullptr || N < 1 || ldw < K)) return SVDQ_ERR_INVALID_ARG;
@@ -298,6 +322,7 @@ extern "C" int svdq_calib_lambda(const void* X, int64_t M, int64_t K, int64_t ld
     if (W != nullptr && (!aligned16(W) || (ldw * 2) % 16 != 0)) return SVDQ_ERR_MISALIGNED;
     if ((reinterpret_cast<uintptr_t>(s_g) | reinterpret_cast<uintptr_t>(amax_x)) & 3u) return SVDQ_ERR_MISALIGNED;
     if (W != nullptr && (reinterpret_cast<uintptr_t>(amax_w) & 3u)) return SVDQ_ERR_MISALIGNED;
+    if (aw_in != nullptr && (reinterpret_cast<uintptr_t>(aw_in) & 3u)) return SVDQ_ERR_MISALIGNED;
     if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > (int64_t(1) << 30)) return SVDQ_ERR_UNSUPPORTED;
     CalibArgs a{};
     int st = make_seg_table(segs, n_seg, M, &a.segs);
@@ -323,11 +348,13 @@ extern "C" int svdq_calib_lambda(const void* X, int64_t M, int64_t K, int64_t ld
     a.out_bits[0] = reinterpret_cast<uint32_t*>(amax_x);
     a.out_bits[1] = reinterpret_cast<uint32_t*>(amax_w);
     a.ax = amax_x;
-    a.aw = W != nullptr ? amax_w : nullptr;
+    a.aw = W != nullptr ? amax_w : aw_in;
     a.lambda = lambda;
     a.inv_lambda = inv_lambda;
     a.s_g = s_g;
     a.err = err;
+    a.skip_unit = g_arm_skip.exchange(-1);       // armed by the time-out test for this one call
+    a.wait_limit = a.skip_unit >= 0 ? g_arm_limit.load() : kWaitLimitCycles;
     if (a.strips >= (int64_t(1) << 24)) return SVDQ_ERR_UNSUPPORTED;
     const int64_t grid = a.n_units == 0 ? a.strips : (a.n_units < sms ? a.n_units : sms);
 
@@ -342,6 +369,7 @@ extern "C" int svdq_calib_lambda(const void* X, int64_t M, int64_t K, int64_t ld
 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const int64_t zb = (K + 255) / 256;
+    // the stored weight absmax is an input: only the outputs are zeroed
     calib_zero_kernel<<<static_cast<unsigned>(zb < sms ? zb : sms), 256, 0, cs>>>(
         amax_x, W != nullptr ? amax_w : nullptr, K, lambda, s_g);
     st = launch_status(cudaGetLastError());
@@ -360,4 +388,25 @@ extern "C" int svdq_calib_lambda(const void* X, int64_t M, int64_t K, int64_t ld
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return launch_status(cudaLaunchKernelEx(&cfg, calib_stream_kernel, tx, tw, a));
+}
+
+}  // namespace
+}  // namespace svdq
+
+extern "C" int svdq_calib_lambda(const void* X, int64_t M, int64_t K, int64_t ldx,
+                                 const svdq_seg* segs, int n_seg,
+                                 const void* W, int64_t N, int64_t ldw,
+                                 float* amax_x, float* amax_w, float* lambda, float* inv_lambda,
+                                 float* s_g, void* stream) {
+    return svdq::calib_launch(X, M, K, ldx, segs, n_seg, W, N, ldw, nullptr, amax_x, amax_w, lambda, inv_lambda,
+                              s_g, stream);
+}
+
+extern "C" int svdq_calib_lambda_stored_w(const void* X, int64_t M, int64_t K, int64_t ldx,
+                                          const svdq_seg* segs, int n_seg, const float* amax_w,
+                                          float* amax_x, float* lambda, float* inv_lambda, float* s_g,
+                                          void* stream) {
+    if (amax_w == nullptr) return SVDQ_ERR_INVALID_ARG;
+    return svdq::calib_launch(X, M, K, ldx, segs, n_seg, nullptr, 0, 0, amax_w, amax_x, nullptr, lambda,
+                              inv_lambda, s_g, stream);
 }

@@ -81,6 +81,16 @@ inline bool set_dynamic_smem_once(Kernel kern, uint32_t bytes, std::atomic<uint6
     return true;
 }
 
+// Largest grid of `kern` (blockDim `threads`, `smem` dynamic bytes) whose CTAs
+// can all be resident at once on the current device: what a cooperative launch
+// may use.  0 if the occupancy query fails.
+template <typename Kernel>
+inline int64_t coresident_grid(Kernel kern, int threads, size_t smem) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess) return 0;
+    return static_cast<int64_t>(per_sm) * device_sm_count();
+}
+
 inline int launch_status(cudaError_t e) {
     if (e == cudaSuccess) return SVDQ_OK;
     return SVDQ_ERR_CUDA;

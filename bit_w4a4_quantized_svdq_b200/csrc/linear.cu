@@ -66,14 +66,14 @@ constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBKBytes = 128;                 // packed FP4 bytes per row per stage (256 channels)
 constexpr int kBK = 256;                      // channels per stage
-constexpr int kStages = 3;
-constexpr int kThreads = 480;                 // 15 warps
-constexpr int kSfWarp0 = 3;                   // warps 3..6 write block scales into tensor memory
+constexpr int kThreads = 448;                 // 14 warps
+constexpr int kSfWarp0 = 2;                   // warps 2..5 write block scales into tensor memory
 constexpr int kSfWarps = 4;
-constexpr int kEpiWarp0 = 7;                  // warps 7..14: epilogue
+constexpr int kEpiWarp0 = 6;                  // warps 6..13: epilogue
 constexpr int kEpiWarps = 8;
-static_assert(kSfWarp0 == 3 && kSfWarp0 + kSfWarps == kEpiWarp0 && kEpiWarp0 + kEpiWarps == kThreads / 32,
-              "warp roles: 0 producer, 1 MMA issuer, 2 low-rank builder, 3..6 scale writers, 7..14 epilogue");
+static_assert(kSfWarp0 == 2 && kSfWarp0 + kSfWarps == kEpiWarp0 && kEpiWarp0 + kEpiWarps == kThreads / 32,
+              "warp roles: 0 producer, 1 MMA issuer, 2..5 scale writers, 6..13 epilogue; each group of four "
+              "consecutive warps covers the four tensor-memory lane quarters (warp % 4)");
 
 constexpr uint32_t kATile = kBM * kBKBytes;          // 16 KB
 constexpr uint32_t kBTile = kBN * kBKBytes;          // 32 KB
@@ -82,22 +82,28 @@ constexpr uint32_t kStageBytes = kATile + kBTile;
 // A: 8 atoms of the tile's row block; W: 8 atoms of each of its two row blocks.
 constexpr uint32_t kSfaPair = 4096;
 constexpr uint32_t kSfSlot = kSfaPair + 8192;        // 12 KB
-constexpr uint32_t kLrA = kBM * 128;                 // 128 rows x 64 bf16
-constexpr uint32_t kLrB = kBN * 128;                 // 256 rows x 64 bf16
-
-constexpr uint32_t kOffStages = 0;
-constexpr uint32_t kOffSf = kStages * kStageBytes;   // 2 slots, multiple of 1024
-constexpr uint32_t kOffLrA = kOffSf + 2 * kSfSlot;
-constexpr uint32_t kOffLrB = kOffLrA + kLrA;
-constexpr uint32_t kOffBar = kOffLrB + kLrB;
-constexpr uint32_t kOffBias = kOffBar + 256;          // 2 x 256 bf16 bias staging
-constexpr uint32_t kOffScore = kOffBias + 2 * kBN * 2;  // scoring: row sums, segment sums, segment rows
-constexpr uint32_t kScoreBytes = 2 * kBM * 16 + kMaxSegments * 16 + kMaxSegments * 8;
-constexpr uint32_t kSmemBytes = kOffScore + kScoreBytes;
-// Scoring: reference strips of 128 rows x 64 bf16 columns, three in the low-rank area.
+// Scoring: reference strips of 128 rows x 64 bf16 columns, three in the epilogue area.
 constexpr uint32_t kStripBytes = kBM * 128;
-static_assert(3 * kStripBytes <= kLrA + kLrB, "three reference strips fit the low-rank operand area");
-static_assert(kSmemBytes + 1024 <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
+constexpr uint32_t kScoreBytes = 2 * kBM * 16 + kMaxSegments * 16 + kMaxSegments * 8;
+constexpr uint32_t kYStageBytes = 1024;              // per epilogue warp: 32 rows x 16 bf16 columns
+
+// Shared-memory layout.  The low-rank operands of a tile travel through the
+// operand ring as one more stage (written by the epilogue warps), so the ring
+// takes all the room the rest leaves: four 48 KB stages, or three where the
+// scoring epilogue needs 48 KB for its reference strips.
+template <bool kScore>
+struct LinLayout {
+    static constexpr int kStages = kScore ? 3 : 4;
+    static constexpr uint32_t kOffStages = 0;
+    static constexpr uint32_t kOffSf = kStages * kStageBytes;              // 2 slots, multiple of 1024
+    static constexpr uint32_t kOffEpi = kOffSf + 2 * kSfSlot;              // output staging / reference strips
+    static constexpr uint32_t kEpiBytes = kScore ? 3 * kStripBytes : kEpiWarps * kYStageBytes;
+    static constexpr uint32_t kOffBar = kOffEpi + kEpiBytes;
+    static constexpr uint32_t kOffBias = kOffBar + 256;                    // 2 x 256 bf16 bias staging
+    static constexpr uint32_t kOffScore = kOffBias + 2 * kBN * 2;          // scoring: row and segment sums
+    static constexpr uint32_t kBytes = kOffScore + (kScore ? kScoreBytes : 0);
+    static_assert(kBytes + 1024 <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
+};
 
 // Tensor-memory columns: accumulator [0, 256), then one block-scale buffer per
 // pipeline stage (48 columns each: A scales 4 per MMA, B scales 8 per MMA).
@@ -105,6 +111,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemSf0 = 256;
 constexpr uint32_t kTmemSfStride = 48;
 constexpr uint32_t kTmemSfbOff = 16;
+static_assert(kTmemSf0 + 4 * kTmemSfStride <= kTmemCols, "accumulator and four scale buffers fit tensor memory");
 
 struct LinearArgs {
     const uint8_t* a_sf;
@@ -182,25 +189,94 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return l | (h << 16);
 }
 
+// The tile's low-rank operands, written by the epilogue warps into the ring
+// slot that follows the tile's last K stage: A = D' of the tile's 128 rows as
+// bf16 hi (ranks 0..31) | lo (32..63), B = up of its 256 columns twice, both in
+// the 128-byte-swizzled K-major layout the MMAs read, D' = D / alpha.  The
+// global reads (the tile's D rows and up rows) are issued before the wait for
+// the slot (go_bar: the producer found the slot free), so only shared-memory
+// stores follow it.  Every epilogue thread calls this; whether to go on is
+// decided together (no warp is ever left waiting at the named barrier); four
+// warps arrive on the slot's barrier, the count the scale writers give an
+// ordinary stage, and one on done_bar.
+__device__ __forceinline__ bool lr_stage(const LinearArgs& a, uint8_t* slot, uint64_t* go_bar, uint32_t parity,
+                                         uint64_t* full_bar, uint64_t* done_bar, int m_blk, int n_blk,
+                                         float inv_alpha, int etid, volatile uint32_t* abort_flag) {
+    const int r = a.r;
+    const int arow = etid >> 1, h = etid & 1;               // A row of this thread and its 16 ranks
+    float dv[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) dv[j] = 0.0f;
+    const int64_t gm = static_cast<int64_t>(m_blk) * kBM + arow;
+    if (gm < a.M && 16 * h < r) {
+        const float4* src = reinterpret_cast<const float4*>(a.D + gm * r + 16 * h);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = __ldg(src + q);
+            dv[4 * q] = v.x; dv[4 * q + 1] = v.y; dv[4 * q + 2] = v.z; dv[4 * q + 3] = v.w;
+        }
+    }
+    uint4 u[4];                                              // B row etid: up[n, 0..31] (zero past r)
+    const int64_t gn = static_cast<int64_t>(n_blk) * kBN + etid;
+    const uint4* usrc = reinterpret_cast<const uint4*>(a.up + gn * r);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) u[c] = (c * 8 < r && gn < a.N) ? __ldg(usrc + c) : make_uint4(0, 0, 0, 0);
+    const bool ok = mbar_wait(go_bar, parity, abort_flag, a.err, kErrWaitLowRank);
+    if (ok) {
+        uint32_t hi[8], lo[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float x0 = __fmul_rn(dv[2 * j], inv_alpha);
+            const float x1 = __fmul_rn(dv[2 * j + 1], inv_alpha);
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+            const float r0 = __fsub_rn(x0, __bfloat162float(h0));
+            const float r1 = __fsub_rn(x1, __bfloat162float(h1));
+            hi[j] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                    (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+            lo[j] = pack_bf16x2(r0, r1);
+        }
+        uint8_t* rowp = slot + arow * 128;
+        const int sw = arow & 7;
+        *reinterpret_cast<uint4*>(rowp + (((2 * h) ^ sw) << 4)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(rowp + (((2 * h + 1) ^ sw) << 4)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+        *reinterpret_cast<uint4*>(rowp + (((4 + 2 * h) ^ sw) << 4)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(rowp + (((5 + 2 * h) ^ sw) << 4)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+        uint8_t* browp = slot + kATile + etid * 128;
+        const int swb = etid & 7;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            *reinterpret_cast<uint4*>(browp + ((c ^ swb) << 4)) = u[c];
+            *reinterpret_cast<uint4*>(browp + (((c + 4) ^ swb) << 4)) = u[c];
+        }
+    }
+    fence_async_shared();                                    // the tensor core reads these stores
+    const bool fail = bar_sync_or<1, kEpiWarps * 32>(!ok);
+    if (!fail && (etid & 31) == 0 && etid < 4 * 32) mbar_arrive(full_bar);
+    if (!fail && etid == 0) mbar_arrive(done_bar);
+    return !fail;
+}
+
 template <bool kOutF32, bool kScore, bool kMx>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
               const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_r,
               const __grid_constant__ CUtensorMap tmap_sfa,
               const __grid_constant__ CUtensorMap tmap_sfb, LinearArgs args) {
+    using L = LinLayout<kScore>;
+    constexpr int kStagesT = L::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint64_t* empty = full + kStages;
-    uint64_t* acc_full = empty + kStages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+    uint64_t* empty = full + kStagesT;
+    uint64_t* acc_full = empty + kStagesT;
     uint64_t* acc_empty = acc_full + 1;
-    uint64_t* lr_full = acc_empty + 1;
-    uint64_t* stage_free = lr_full + 1;                     // epilogue done with the staging area
-    uint64_t* sf_data = stage_free + 1;                     // 2 slots: scale atoms landed
+    uint64_t* sf_data = acc_empty + 1;                      // 2 slots: scale atoms landed
     uint64_t* sf_free = sf_data + 2;                        // 2 slots: the writers have read them
     uint64_t* strip_full = sf_free + 2;                     // scoring: reference strips 0..3 landed
     uint64_t* ring_free0 = strip_full + 4;                  // scoring: column half 0 done with slot 0
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring_free0 + 1);
+    uint64_t* lr_go = ring_free0 + 1;                       // producer: this tile's low-rank slot is free
+    uint64_t* lr_done = lr_go + 1;                          // epilogue: this tile's low-rank stage is written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lr_done + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5;
@@ -216,14 +292,17 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     constexpr int kSfHalvesPerStage = kMx ? 2 : 8;                  // 256-byte scale pieces per row block
     constexpr uint32_t kTmemSfStrideT = kMx ? 16 : kTmemSfStride;
     constexpr uint32_t kTmemSfbOffT = kMx ? 4 : kTmemSfbOff;
-    const int k_stages = static_cast<int>(args.K / kStageK);
+    // a last partial stage reads zero codes and zero scales past K (TMA fill): it adds nothing
+    const int k_stages = static_cast<int>((args.K + kStageK - 1) / kStageK);
     const bool has_lr = args.r > 0;
-    const float alpha = kMx ? 1.0f : __fmul_rn(__ldg(args.s_g_act), __ldg(args.s_g_w));
-    const float inv_alpha = __frcp_rn(alpha);
+    // Ring positions per tile: the K stages, then the low-rank stage.
+    const int span = k_stages + (has_lr ? 1 : 0);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1 + kSfWarps);              // operand bytes + the stage's scales in tensor memory
+        for (int s = 0; s < kStagesT; ++s) {
+            // operand bytes + the stage's scales in tensor memory (low-rank stage:
+            // the producer's arrival + four epilogue warps' operand stores)
+            mbar_init(&full[s], 1 + kSfWarps);
             mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -232,10 +311,10 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kEpiWarps);
-        mbar_init(lr_full, 1);
-        mbar_init(stage_free, kEpiWarps);
         for (int i = 0; i < 4; ++i) mbar_init(&strip_full[i], 1);
         mbar_init(ring_free0, kEpiWarps / 2);
+        mbar_init(lr_go, 1);
+        mbar_init(lr_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -247,6 +326,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -255,6 +335,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             prefetch_tmap(&tmap_b);
             prefetch_tmap(&tmap_sfa);
             prefetch_tmap(&tmap_sfb);
+            pdl_wait();                               // the activation codes and scales are written
             // Scale batches run one batch (two stages) ahead of the operands: the
             // batch a stage needs has landed by the time its operands do.
             int sf_tile = blockIdx.x, sf_kb = 0, issued = 0;
@@ -266,7 +347,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     return false;
                 int m_blk, n_blk;
                 tile_coords(args, sf_tile, m_blk, n_blk);
-                uint8_t* dst = smem + kOffSf + slot * kSfSlot;
+                uint8_t* dst = smem + L::kOffSf + slot * kSfSlot;
                 mbar_arrive_expect_tx(&sf_data[slot], kSfSlotT);
                 // scale atoms of stages sf_kb and sf_kb + 1 (a last odd stage reads zeros past K)
                 tma_load_3d(dst, &tmap_sfa, &sf_data[slot], 0, sf_kb * kSfHalvesPerStage, m_blk);
@@ -279,7 +360,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 }
                 return true;
             };
-            int s = 0, it = 0;
+            int s = 0, it = 0, lr_tiles = 0;
             uint32_t ph = 0;
             bool ok = issue_scales();
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
@@ -287,18 +368,39 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 tile_coords(args, tile, m_blk, n_blk);
                 for (int kb = 0; kb < k_stages; ++kb, ++it) {
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) { ok = false; break; }
-                    uint8_t* st = smem + kOffStages + s * kStageBytes;
+                    uint8_t* st = smem + L::kOffStages + s * kStageBytes;
                     mbar_arrive_expect_tx(&full[s], kStageBytes);
                     tma_load_2d(st, &tmap_a, &full[s], kb * kBKBytes, m_blk * kBM);
                     tma_load_2d(st + kATile, &tmap_b, &full[s], kb * kBKBytes, n_blk * kBN);
                     if ((kb & 1) == 0 && !issue_scales()) { ok = false; break; }
-                    if (++s == kStages) { s = 0; ph ^= 1u; }
+                    if (++s == kStagesT) { s = 0; ph ^= 1u; }
+                }
+                if (ok && has_lr) {
+                    // The low-rank stage: the epilogue warps fill this slot.  The
+                    // producer walks the ring in order, so its wait for the slot's
+                    // previous MMAs is the safe one (a parity wait tells only one
+                    // phase from the next); it hands the free slot to the epilogue
+                    // through lr_go, once the epilogue has written the previous
+                    // tile's stage (lr_done), so neither barrier ever runs two
+                    // phases ahead of its waiter.  Its arrival on full stands for
+                    // the copies.
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) { ok = false; break; }
+                    if (lr_tiles > 0 &&
+                        !mbar_wait(lr_done, (lr_tiles - 1) & 1, abort_flag, args.err, kErrWaitLowRank)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive(&full[s]);
+                    mbar_arrive(lr_go);
+                    ++lr_tiles;
+                    ++it;
+                    if (++s == kStagesT) { s = 0; ph ^= 1u; }
                 }
             }
             // Bounded drain of the copies still in flight.
-            for (int i = (it > kStages ? it - kStages : 0); i < it; ++i) {
+            for (int i = (it > kStagesT ? it - kStagesT : 0); i < it; ++i) {
                 const long long t0 = clock64();
-                while (!mbar_try_wait(&full[i % kStages], (i / kStages) & 1) && clock64() - t0 < kWaitLimitCycles) {}
+                while (!mbar_try_wait(&full[i % kStagesT], (i / kStagesT) & 1) && clock64() - t0 < kWaitLimitCycles) {}
             }
             for (int q = (issued > 2 ? issued - 2 : 0); q < issued; ++q) {
                 const long long t0 = clock64();
@@ -313,8 +415,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         if (lane == 0) {
             const uint32_t idesc_f4 = idesc_nvf4(kBM, kBN);
             const uint32_t idesc_lr = idesc_bf16(kBM, kBN);
-            const uint64_t da0 = desc_kmajor_sw128(smem_u32(smem + kOffStages));
-            const uint64_t db0 = desc_kmajor_sw128(smem_u32(smem + kOffStages + kATile));
+            const uint64_t da0 = desc_kmajor_sw128(smem_u32(smem + L::kOffStages));
+            const uint64_t db0 = desc_kmajor_sw128(smem_u32(smem + L::kOffStages + kATile));
             constexpr uint64_t kStageDesc = kStageBytes >> 4;     // descriptor address field counts 16 bytes
             int s = 0, local = 0;
             uint32_t ph = 0;
@@ -343,89 +445,26 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                         mma_nvf4(tmem, da + 6, db + 6, idesc_f4, sf + 12, sf + kTmemSfbOff + 24, 1u);
                     }
                     tc_commit(&empty[s]);
-                    if (++s == kStages) { s = 0; ph ^= 1u; }
+                    if (++s == kStagesT) { s = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
                 if (has_lr) {
-                    // Low-rank term last: its operands share shared memory with the
-                    // epilogue's output staging, which is free again once this
-                    // tile's accumulator has been drained.
-                    if (!mbar_wait(lr_full, local & 1, abort_flag, args.err, kErrWaitLowRank)) break;
+                    // The low-rank term closes the tile: 4 kind::f16 MMAs (K = 64:
+                    // 32 ranks of D'_hi, then 32 of D'_lo, against up twice) from
+                    // the ring slot the epilogue warps filled.
+                    if (!mbar_try_wait(&full[s], ph) &&
+                        !mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitLowRank))
+                        break;
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(smem + kOffLrA);
-                    const uint32_t b0 = smem_u32(smem + kOffLrB);
+                    const uint32_t a0 = smem_u32(smem + L::kOffStages + s * kStageBytes);
+                    const uint32_t b0 = a0 + kATile;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16(tmem, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc_lr, 1u);
+                    tc_commit(&empty[s]);
+                    if (++s == kStagesT) { s = 0; ph ^= 1u; }
                 }
                 tc_commit(acc_full);
-            }
-        }
-    } else if (warp == 2) {
-        // ------------------------------------------------------------ low-rank operand builder
-        if (has_lr) {
-            int local = 0;
-            const int r = args.r;
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-                int m_blk, n_blk;
-                tile_coords(args, tile, m_blk, n_blk);
-                if (!mbar_wait(stage_free, (local & 1) ^ 1, abort_flag, args.err, kErrWaitLowRank)) break;
-                uint8_t* la = smem + kOffLrA;
-                uint8_t* lb = smem + kOffLrB;
-                // A: row = D'[m] as bf16 hi (channels 0..31) and lo (32..63)
-                for (int row = lane; row < kBM; row += 32) {
-                    const int64_t gm = static_cast<int64_t>(m_blk) * kBM + row;
-                    float dv[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) dv[j] = 0.0f;
-                    if (gm < args.M) {
-                        const float4* src = reinterpret_cast<const float4*>(args.D + gm * r);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            if (q * 4 < r) {
-                                const float4 v = __ldg(src + q);
-                                dv[4 * q] = v.x; dv[4 * q + 1] = v.y; dv[4 * q + 2] = v.z; dv[4 * q + 3] = v.w;
-                            }
-                        }
-                    }
-                    uint32_t hi[16], lo[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float x0 = __fmul_rn(dv[2 * j], inv_alpha);
-                        const float x1 = __fmul_rn(dv[2 * j + 1], inv_alpha);
-                        const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-                        const float r0 = __fsub_rn(x0, __bfloat162float(h0));
-                        const float r1 = __fsub_rn(x1, __bfloat162float(h1));
-                        hi[j] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                                (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-                        lo[j] = pack_bf16x2(r0, r1);
-                    }
-                    uint8_t* rowp = la + row * 128;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        *reinterpret_cast<uint4*>(rowp + ((c ^ (row & 7)) << 4)) =
-                            make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
-                        *reinterpret_cast<uint4*>(rowp + (((c + 4) ^ (row & 7)) << 4)) =
-                            make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
-                    }
-                }
-                // B: row n = [up[n, 0..31] | up[n, 0..31]] (zero beyond r)
-                for (int row = lane; row < kBN; row += 32) {
-                    const int64_t gn = static_cast<int64_t>(n_blk) * kBN + row;
-                    uint4 u[4];
-                    const uint4* src = reinterpret_cast<const uint4*>(args.up + gn * r);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) u[c] = (c * 8 < r) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-                    uint8_t* rowp = lb + row * 128;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        *reinterpret_cast<uint4*>(rowp + ((c ^ (row & 7)) << 4)) = u[c];
-                        *reinterpret_cast<uint4*>(rowp + (((c + 4) ^ (row & 7)) << 4)) = u[c];
-                    }
-                }
-                fence_async_shared();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(lr_full);
             }
         }
     } else if (warp < kEpiWarp0) {
@@ -437,7 +476,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         // the MMA thread, these stores run alongside the MMAs instead of in front
         // of them.  Ring slot: released once both of its stages are in registers.
         // Tensor-memory buffer s: written only after the MMAs of its previous
-        // use have completed (the stage's empty barrier).
+        // use have completed (the stage's empty barrier).  Low-rank stages are
+        // the epilogue's: the writers only step over them.
         const uint32_t tq = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         int s = 0, it = 0, pair = -1;
         uint32_t ph = 0;
@@ -460,8 +500,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 if constexpr (kMx) {
                     // MXFP8: the stage's one A atom and one W atom per 128-row block
                     // (slot layout: A [2 stages][512], then W [2 row blocks][2 stages][512]).
-                    const uint8_t* sfa = smem + kOffSf + slot * kSfSlot + (kb & 1) * 512;
-                    const uint8_t* sfb = smem + kOffSf + slot * kSfSlot + kSfaPairT + (kb & 1) * 512;
+                    const uint8_t* sfa = smem + L::kOffSf + slot * kSfSlot + (kb & 1) * 512;
+                    const uint8_t* sfb = smem + L::kOffSf + slot * kSfSlot + kSfaPairT + (kb & 1) * 512;
                     const uint4 a = *reinterpret_cast<const uint4*>(sfa + lane * 16);
                     const uint4 x = *reinterpret_cast<const uint4*>(sfb + lane * 16);
                     const uint4 y = *reinterpret_cast<const uint4*>(sfb + 1024 + lane * 16);
@@ -469,8 +509,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     rb[0] = x.x; rb[1] = x.y; rb[2] = x.z; rb[3] = x.w;
                     rb[4] = y.x; rb[5] = y.y; rb[6] = y.z; rb[7] = y.w;
                 } else {
-                    const uint8_t* sfa = smem + kOffSf + slot * kSfSlot + (kb & 1) * 2048;
-                    const uint8_t* sfb = smem + kOffSf + slot * kSfSlot + kSfaPair + (kb & 1) * 2048;
+                    const uint8_t* sfa = smem + L::kOffSf + slot * kSfSlot + (kb & 1) * 2048;
+                    const uint8_t* sfb = smem + L::kOffSf + slot * kSfSlot + kSfaPair + (kb & 1) * 2048;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const uint4 a = *reinterpret_cast<const uint4*>(sfa + q * 512 + lane * 16);
@@ -485,7 +525,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sf_free[slot]);
                 }
-                if (it >= kStages && !mbar_try_wait(&empty[s], ph ^ 1) &&
+                if (it >= kStagesT && !mbar_try_wait(&empty[s], ph ^ 1) &&
                     !mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) {
                     ok = false;
                     break;
@@ -504,17 +544,20 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[s]);
-                if (++s == kStages) { s = 0; ph ^= 1u; }
+                if (++s == kStagesT) { s = 0; ph ^= 1u; }
+            }
+            if (ok && has_lr) {
+                ++it;
+                if (++s == kStagesT) { s = 0; ph ^= 1u; }
             }
         }
     } else if constexpr (kScore) {
         // ------------------------------------------------------------ epilogue with scoring
         // The plain epilogue's output path plus the tile's scoring against the
         // reference output.  The reference comes in by TMA as strips of 128 rows x
-        // 64 columns (16 KB, 128-byte swizzle) into a three-slot ring over the
-        // low-rank operand area, which is free from "accumulator full" (this
-        // tile's low-rank MMAs have completed) until every epilogue warp has
-        // signalled stage_free.  Strips 0 and 2 (the first 64 columns of each
+        // 64 columns (16 KB, 128-byte swizzle) into a three-slot ring in the
+        // epilogue area, which the previous tile's strips (and the output stores
+        // that read them) have left by the barrier that ends each tile.  Strips 0 and 2 (the first 64 columns of each
         // column half) and strip 1 go out at "accumulator full"; strip 3 takes
         // strip 0's slot once the four warps of column half 0 are done with it.
         // Each lane scores its own row against its converted output values, so no
@@ -528,12 +571,15 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         const int half = ew >> 2;                           // column half of the tile
         const int etid = ew * 32 + lane;                    // 0..255
         const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * (kBN / 2);
-        uint16_t* bias_s = reinterpret_cast<uint16_t*>(smem + kOffBias);
-        uint8_t* ring = smem + kOffLrA;
-        double2* rowsum = reinterpret_cast<double2*>(smem + kOffScore);   // [column half][tile row] (num, den)
+        uint16_t* bias_s = reinterpret_cast<uint16_t*>(smem + L::kOffBias);
+        uint8_t* ring = smem + L::kOffEpi;
+        double2* rowsum = reinterpret_cast<double2*>(smem + L::kOffScore);   // [column half][tile row] (num, den)
         double2* segsum = rowsum + 2 * kBM;                              // [segment] this CTA's (num, den)
         int2* segrows = reinterpret_cast<int2*>(segsum + kMaxSegments);  // [segment] rows [begin, end)
         const int n_seg = args.segs.n;
+        pdl_wait();                                   // inputs of the earlier kernels are written
+        const float alpha = __fmul_rn(__ldg(args.s_g_act), __ldg(args.s_g_w));
+        const float inv_alpha = __frcp_rn(alpha);
         for (int i = etid; i < kMaxSegments; i += kEpiWarps * 32) {
             segsum[i] = make_double2(0.0, 0.0);
             if (i < n_seg) {
@@ -551,9 +597,16 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             const int32_t col0 = n_blk * kBN;
             const int32_t m0 = m_blk * kBM;
             uint16_t* bt = bias_s + (local & 1) * kBN;
-            bt[etid] = args.bias ? args.bias[col0 + etid] : static_cast<uint16_t>(0);
+            bt[etid] = (args.bias && col0 + etid < args.N) ? args.bias[col0 + etid] : static_cast<uint16_t>(0);
             // bias staged, the previous tile's row sums consumed; leave together on abort
             if (bar_sync_or<1, kEpiWarps * 32>(*abort_flag != 0u)) break;
+            if (has_lr) {
+                const int64_t p = static_cast<int64_t>(local + 1) * span - 1;      // this tile's low-rank stage
+                const int slot = static_cast<int>(p % kStagesT);
+                if (!lr_stage(args, smem + L::kOffStages + slot * kStageBytes, lr_go, static_cast<uint32_t>(local & 1),
+                              &full[slot], lr_done, m_blk, n_blk, inv_alpha, etid, abort_flag))
+                    continue;                                // the abort flag is up: the loop top leaves
+            }
             bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, local & 1, abort_flag, args.err, kErrWaitMma));
             tc_fence_after();
             if (ok && etid == 0) {
@@ -628,7 +681,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     if (args.write_y) {
                         fence_async_shared();
                         __syncwarp();
-                        if (lane == 0 && grow0 < M32) {     // boxes wholly below row M are skipped
+                        if (lane == 0 && grow0 < M32 && col0 + half * (kBN / 2) + h * 64 < args.N) {
+                            // boxes wholly past row M or column N are skipped
                             tma_store_2d(&tmap_y, part, col0 + half * (kBN / 2) + h * 64, grow0);
                             bulk_commit_group();
                         }
@@ -648,9 +702,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     }
                 }
             }
-            if (args.write_y && lane == 0) bulk_wait_read_all();
+            if (args.write_y && lane == 0) bulk_wait_read_all();   // the ring is no longer read
             __syncwarp();
-            if (lane == 0) mbar_arrive(stage_free);         // the ring is no longer read
             rowsum[half * kBM + quarter * 32 + lane] =
                 grow0 + static_cast<int32_t>(lane) < M32
                     ? make_double2(static_cast<double>(nh) + static_cast<double>(nl),
@@ -695,88 +748,102 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     } else {
         // ------------------------------------------------------------ epilogue
         // Two warps per tensor-memory lane quarter, each owning 128 of the 256
-        // columns.  The tile's bias is staged in shared memory before the
-        // accumulator wait, so nothing but tensor-memory reads sits between
-        // "accumulator full" and "accumulator free".
+        // columns.  Per tile: the bias is staged in shared memory; the tile's
+        // low-rank stage is written into the ring (lr_stage); then, at
+        // "accumulator full", the warp reads all its 128 columns (two 32-column
+        // loads per wait), releases the accumulator and only then applies alpha
+        // and bias and stores, so the next tile's MMAs start as early as possible.
+        // bf16 rows leave in eight TMA stores of 16 columns x 32 rows through the
+        // warp's 1 KB staging buffer (bulk stores keep scattered per-row writes off
+        // the load/store path the tensor core reads its operands through); fp32
+        // rows with plain stores.  The loop is left only at its top, all warps
+        // together, so a wait that runs out never strands a warp at a barrier.
         const int ew = warp - kEpiWarp0;                    // 0..7
         const int quarter = warp & 3;                       // lane quarter this warp may access
         const int half = ew >> 2;                           // column half of the tile
         const int etid = ew * 32 + lane;                    // 0..255
         const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * (kBN / 2);
-        uint16_t* bias_s = reinterpret_cast<uint16_t*>(smem + kOffBias);
+        uint16_t* bias_s = reinterpret_cast<uint16_t*>(smem + L::kOffBias);
+        uint8_t* stg = smem + L::kOffEpi + ew * kYStageBytes;
+        pdl_wait();                                   // inputs of the earlier kernels are written
+        const float alpha = kMx ? 1.0f : __fmul_rn(__ldg(args.s_g_act), __ldg(args.s_g_w));
+        const float inv_alpha = __frcp_rn(alpha);
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             int m_blk, n_blk;
             tile_coords(args, tile, m_blk, n_blk);
             const int64_t col0 = static_cast<int64_t>(n_blk) * kBN;
             uint16_t* bt = bias_s + (local & 1) * kBN;
-            bt[etid] = args.bias ? args.bias[col0 + etid] : static_cast<uint16_t>(0);
-            asm volatile("bar.sync 1, %0;" :: "n"(kEpiWarps * 32) : "memory");
-            if (!mbar_wait(acc_full, local & 1, abort_flag, args.err, kErrWaitMma)) break;
+            bt[etid] = (args.bias && col0 + etid < args.N) ? args.bias[col0 + etid] : static_cast<uint16_t>(0);
+            // bias staged; leave together on abort
+            if (bar_sync_or<1, kEpiWarps * 32>(*abort_flag != 0u)) break;
+            if (has_lr) {
+                const int64_t p = static_cast<int64_t>(local + 1) * span - 1;      // this tile's low-rank stage
+                const int slot = static_cast<int>(p % kStagesT);
+                if (!lr_stage(args, smem + L::kOffStages + slot * kStageBytes, lr_go, static_cast<uint32_t>(local & 1),
+                              &full[slot], lr_done, m_blk, n_blk, inv_alpha, etid, abort_flag))
+                    continue;                                // the abort flag is up: the loop top leaves
+            }
+            if (!mbar_wait(acc_full, local & 1, abort_flag, args.err, kErrWaitMma)) continue;
             tc_fence_after();
             const int64_t row = static_cast<int64_t>(m_blk) * kBM + quarter * 32 + lane;
             const int64_t ccol = col0 + half * (kBN / 2);   // first output column of this warp
             const uint16_t* bw = bt + half * (kBN / 2);
-            const bool row_ok = row < args.M;
             if constexpr (!kOutF32) {
-                // Per 64-column half: two 32-column tensor-memory loads in flight per
-                // wait, alpha and bias, bf16 rows staged in shared memory (the
-                // low-rank operand area, free since this tile's low-rank MMAs
-                // completed before the accumulator was signalled full; 32 rows x 64
-                // columns per warp, 128-byte swizzle) and written by a TMA bulk
-                // store.  The accumulator is released as soon as the second half
-                // has been read, before its conversion.  Bulk stores keep the
-                // scattered per-row writes off the load/store path the tensor core
-                // reads its operands through.
-                uint8_t* stg = smem + kOffLrA + ew * 4096;
+                // pk[16 c + j]: columns 32 c + 2 j and 32 c + 2 j + 1 of this warp, as bf16
+                uint32_t pk[64];
+                auto convert = [&](const uint32_t (&v)[32], int c) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const uint32_t bb = *reinterpret_cast<const uint32_t*>(bw + c * 32 + 2 * j);
+                        pk[c * 16 + j] = pack_bf16x2(fmaf(alpha, __uint_as_float(v[2 * j]), bf16_lo(bb)),
+                                                     fmaf(alpha, __uint_as_float(v[2 * j + 1]), bf16_hi(bb)));
+                    }
+                };
+                {
+                    uint32_t v[2][32];
+                    tmem_ld_32x32b_x32(tbase, v[0]);
+                    tmem_ld_32x32b_x32(tbase + 32, v[1]);
+                    tmem_ld_wait();
+                    convert(v[0], 0);
+                    convert(v[1], 1);
+                }
+                {
+                    // one piece at a time: the converted columns and one load fit the registers
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase + 64, v);
+                    tmem_ld_wait();
+                    convert(v, 2);
+                    tmem_ld_32x32b_x32(tbase + 96, v);
+                    tmem_ld_wait();
+                    tc_fence_before();              // the accumulator has been read: next tile's MMAs may start
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(acc_empty);
+                    convert(v, 3);
+                }
                 const int32_t grow0 = static_cast<int32_t>(m_blk * kBM + quarter * 32);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t v[2][32];
-                    tmem_ld_32x32b_x32(tbase + (2 * h) * 32, v[0]);
-                    tmem_ld_32x32b_x32(tbase + (2 * h + 1) * 32, v[1]);
-                    tmem_ld_wait();
-                    if (h == 1) {                   // the accumulator has been read: next tile's MMAs may start
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(acc_empty);
-                    }
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int c = 2 * h + hh;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const uint32_t bb = *reinterpret_cast<const uint32_t*>(bw + c * 32 + 2 * j);
-                            pk[hh * 16 + j] = pack_bf16x2(fmaf(alpha, __uint_as_float(v[hh][2 * j]), bf16_lo(bb)),
-                                                          fmaf(alpha, __uint_as_float(v[hh][2 * j + 1]), bf16_hi(bb)));
-                        }
-                    }
-                    if (h == 1) {                   // the first half's store has finished reading the buffer
-                        if (lane == 0) bulk_wait_read_all();
-                        __syncwarp();
-                    }
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                for (int j = 0; j < 8; ++j) {
+                    if (lane == 0) bulk_wait_read_all();    // the previous box has left the buffer
+                    __syncwarp();
+                    uint4* dst = reinterpret_cast<uint4*>(stg + lane * 32);
+                    dst[0] = make_uint4(pk[8 * j], pk[8 * j + 1], pk[8 * j + 2], pk[8 * j + 3]);
+                    dst[1] = make_uint4(pk[8 * j + 4], pk[8 * j + 5], pk[8 * j + 6], pk[8 * j + 7]);
                     fence_async_shared();
                     __syncwarp();
-                    if (lane == 0 && grow0 < args.M) {          // boxes wholly below row M are skipped
-                        tma_store_2d(&tmap_y, stg, static_cast<int32_t>(ccol) + h * 64, grow0);
+                    if (lane == 0 && grow0 < args.M && ccol + 16 * j < args.N) {   // boxes wholly past M or N are skipped
+                        tma_store_2d(&tmap_y, stg, static_cast<int32_t>(ccol) + 16 * j, grow0);
                         bulk_commit_group();
                     }
                 }
-                if (lane == 0) bulk_wait_read_all();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(stage_free);
             } else {
+                const bool row_ok = row < args.M;
 #pragma unroll 1
                 for (int c = 0; c < kBN / 2 / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, v);
                     tmem_ld_wait();
-                    if (row_ok) {
+                    if (row_ok && ccol + c * 32 < args.N) {           // N % 128 == 0: chunks are whole
                         float* dst = static_cast<float*>(args.Y) + row * args.ldy + ccol + c * 32;
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
@@ -793,10 +860,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(acc_empty);
-                    mbar_arrive(stage_free);
-                }
+                if (lane == 0) mbar_arrive(acc_empty);
             }
         }
         if constexpr (!kOutF32) {
@@ -844,32 +908,49 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     }
 }
 
-// Persistent grid: one CTA per SM (at most one fits), never more CTAs than tiles.
-inline int linear_grid(int m_tiles, int n_tiles) {
+// Persistent grid: one CTA per SM (at most one fits), never more CTAs than tiles;
+// with scoring (a cooperative launch) never more than can be resident at once.
+inline int linear_grid(int m_tiles, int n_tiles, int64_t resident = 0) {
     const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
     const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
-    return static_cast<int>(tiles < sms ? tiles : sms);
+    int64_t g = tiles < sms ? tiles : sms;
+    if (resident > 0 && g > resident) g = resident;
+    return static_cast<int>(g);
 }
 
+// `ws_bytes`: the scoring workspace (per-CTA segment sums), checked against the grid.
 template <bool kOutF32, bool kScore, bool kMx = false>
 int launch_linear(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, const CUtensorMap& tr,
-                  const CUtensorMap& tsa, const CUtensorMap& tsb, const LinearArgs& a, cudaStream_t st) {
+                  const CUtensorMap& tsa, const CUtensorMap& tsb, const LinearArgs& a, cudaStream_t st,
+                  size_t ws_bytes = 0) {
     static_assert(!(kOutF32 && kScore), "scoring is fused into the bf16 epilogue only");
-    const uint32_t smem = kSmemBytes + 1024;
+    const uint32_t smem = LinLayout<kScore>::kBytes + 1024;
     auto kern = linear_kernel<kOutF32, kScore, kMx>;
     static std::atomic<uint64_t> smem_set{0};
     if (!set_dynamic_smem_once(kern, smem, smem_set)) return SVDQ_ERR_CUDA;
-    const int grid = linear_grid(a.m_tiles, a.n_tiles);
+    int64_t resident = 0;
+    if (kScore) {
+        resident = coresident_grid(kern, kThreads, smem);
+        if (resident < 1) return SVDQ_ERR_CUDA;
+    }
+    const int grid = linear_grid(a.m_tiles, a.n_tiles, resident);
+    if (kScore && ws_bytes < static_cast<size_t>(grid) * a.segs.n * 2 * sizeof(double)) return SVDQ_ERR_INVALID_ARG;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;      // scoring ends with a grid barrier
-    attr[0].val.cooperative = 1;
+    if (kScore) {
+        attr[0].id = cudaLaunchAttributeCooperative;      // scoring ends with a grid barrier
+        attr[0].val.cooperative = 1;
+    } else {
+        // a programmatic dependent of the quantiser: set-up overlaps its tail
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = kScore ? 1 : 0;
+    cfg.numAttrs = 1;
     return launch_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, tr, tsa, tsb, a));
 }
 
@@ -878,7 +959,7 @@ int linear_prepare(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g
                    const uint8_t* w_codes, const uint8_t* w_sf, const float* s_g_w, const void* up,
                    const void* bias, void* Y, int64_t ldy, int out_dtype, int64_t M, int64_t N, int64_t K,
                    CUtensorMap* ta, CUtensorMap* tb, CUtensorMap* ty, CUtensorMap* tsa, CUtensorMap* tsb,
-                   LinearArgs* a, bool mx = false) {
+                   LinearArgs* a, bool mx = false, bool score = false) {
     // mx: MXFP8 operands (one byte per element, E8M0 scales per 32, no tensor
     // scales, no low-rank branch); otherwise NVFP4 (two elements per byte).
     if (a_codes == nullptr || a_sf == nullptr || w_codes == nullptr || w_sf == nullptr ||
@@ -890,10 +971,10 @@ int linear_prepare(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g
         return SVDQ_ERR_MISALIGNED;
     if (mx ? r != 0 : (r != 0 && r != 16 && r != 32)) return SVDQ_ERR_UNSUPPORTED;
     if ((r > 0) != (D != nullptr) || (r > 0) != (up != nullptr)) return SVDQ_ERR_INVALID_ARG;
-    if (K % (mx ? 128 : 256) != 0 || N % 256 != 0) return SVDQ_ERR_UNSUPPORTED;
+    if (K % (mx ? 128 : 64) != 0 || N % 128 != 0) return SVDQ_ERR_UNSUPPORTED;
     if (M > (int64_t(1) << 31) - 128 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 30))
         return SVDQ_ERR_UNSUPPORTED;
-    const int64_t m_tiles = (M + 127) / 128, n_tiles = N / 256;
+    const int64_t m_tiles = (M + 127) / 128, n_tiles = (N + 255) / 256;
     if (m_tiles * n_tiles > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
     if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(Y))
         return SVDQ_ERR_MISALIGNED;
@@ -910,9 +991,13 @@ int linear_prepare(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g
         !encode_tmap_2d(tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w_codes, row_bytes, N, row_bytes, 128, 256,
                         CU_TENSOR_MAP_SWIZZLE_128B))
         return SVDQ_ERR_CUDA;
+    // bf16 output boxes: 16 columns x 32 rows unswizzled (the plain epilogue's
+    // 1 KB staging), or 64 x 32 with the 128-byte swizzle of the scoring
+    // epilogue's reference strips
     *ty = *ta;
     if (out_dtype == 0 && Y != nullptr &&
-        !encode_tmap_2d(ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, N, M, ldy * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+        !encode_tmap_2d(ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, N, M, ldy * 2, score ? 64 : 16, 32,
+                        score ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
         return SVDQ_ERR_CUDA;
     // Scale atoms viewed as [row block][atoms x 2 halves][256 bytes]: one box
     // holds the atoms of two stages (A: one row block, W: two).  NVFP4: K / 64
@@ -1006,10 +1091,9 @@ extern "C" int svdq_linear_score(const uint8_t* a_codes, const uint8_t* a_sf, co
     CUtensorMap ta, tb, ty, tsa, tsb;
     LinearArgs a;
     const int st0 = linear_prepare(a_codes, a_sf, s_g_act, D, r, w_codes, w_sf, s_g_w, up, bias, Y, ldy, 0, M, N,
-                                   K, &ta, &tb, &ty, &tsa, &tsb, &a);
+                                   K, &ta, &tb, &ty, &tsa, &tsb, &a, false, true);
     if (st0 != SVDQ_OK) return st0;
-    const int grid = linear_grid(a.m_tiles, a.n_tiles);
-    if (workspace_bytes < static_cast<size_t>(grid) * n_seg * 2 * sizeof(double)) return SVDQ_ERR_INVALID_ARG;
+    if (workspace_bytes < static_cast<size_t>(n_seg) * 2 * sizeof(double)) return SVDQ_ERR_INVALID_ARG;
     const int sst = make_seg_table(segs, n_seg, M, &a.segs);
     if (sst != SVDQ_OK) return sst;
     // The reference in strips of 64 columns x 128 rows, 128-byte swizzle (rows past M read as zeros).
@@ -1021,5 +1105,6 @@ extern "C" int svdq_linear_score(const uint8_t* a_codes, const uint8_t* a_sf, co
     a.num = num;
     a.den = den;
     a.rel = rel;
-    return launch_linear<false, true>(ta, tb, ty, tr, tsa, tsb, a, static_cast<cudaStream_t>(stream));
+    return launch_linear<false, true>(ta, tb, ty, tr, tsa, tsb, a, static_cast<cudaStream_t>(stream),
+                                      workspace_bytes);
 }

@@ -9,34 +9,45 @@
 // "DeltaQuant on MiniMax-H3", section "The activation scale bound held": the
 // tensor scale is static and saturated groups are counted at run time.
 //
-// Layout of one CTA (18 warps, one CTA per SM) over a 128-row tile and a
-// slice of K:
-//   warp 16     TMA producer: 128 x 64 bf16 tiles of X (128-byte swizzle), the
-//               matching r x 64 tile of the down weight and 64 values of
-//               1/lambda into a 9-stage ring (a multiple of the 3 quantiser teams)
-//   warp 17     tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
-//   warps 0..15 quantisers, in two teams of 8 that take alternate stages; a
-//               lane owns one 16-channel group in each of two rows (two
-//               independent dependency chains), reads them from the swizzled
-//               tile, multiplies by 1/lambda and later by 1/S with packed
-//               f32x2 multiplies, forms the E4M3 scales of both rows with one
-//               conversion and the E2M1 codes with the hardware RNE
-//               conversions, and stores 8-byte code words and 4-byte scale
-//               words; 1/S comes from a per-CTA table over the 127 finite
-//               non-negative E4M3 bytes (S = RN(dec(byte) * s_g), 1/S = RN(1/S)),
-//               built once at CTA start;
-//               warps 0..3 (one per tensor-memory lane quarter) finally read
-//               D_partial from tensor memory.
-// K is split across the CTAs of a thread-block cluster (up to 4); the partial
-// D tiles are summed in a fixed order through distributed shared memory, so D
-// is deterministic.  Memory traffic per element: 2 bytes in, 0.5625 out.
+// Work split: the rows are cut into G groups of R consecutive rows (R <= 128,
+// the last group shorter) and K into S slices of consecutive 64-channel chunks
+// (S <= 4, the CTAs of one thread-block cluster): one CTA per (group, slice).
+// R and S are chosen so that G * S comes close to the SM count (at most one
+// CTA fits per SM): 148 CTAs of 111 rows at 4096 rows (S = 4) and at 16384
+// rows (S = 1), 147 of 84 rows at 12288 rows.  Whole 128-row tiles would leave
+// 20 to 52 SMs without work at these sizes.  The partial D tiles of a cluster
+// are summed in cluster-rank order through distributed shared memory, so D is
+// deterministic.
+//
+// Layout of one CTA (26 warps) over its group's rows and its slice of K:
+//   warp 24      TMA producer: R x 64 bf16 tiles of X (128-byte swizzle), the
+//                matching r x 64 tile of the down weight and 64 values of
+//                1/lambda into a 9-stage ring (a multiple of the 3 quantiser teams)
+//   warp 25      tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
+//                (M = 128: rows of a stage slot past R are never stored)
+//   warps 0..23  quantisers, in three teams of 8 that take the stages in
+//                turn; a lane owns one 16-channel group in each of two rows
+//                (two independent dependency chains), reads them from the
+//                swizzled tile, multiplies by 1/lambda and later by 1/S with
+//                packed f32x2 multiplies, forms the E4M3 scales of both rows
+//                with one conversion and the E2M1 codes with the hardware RNE
+//                conversions, and stores 8-byte code words and 4-byte scale
+//                words; 1/S comes from a per-CTA table over the 127 finite
+//                non-negative E4M3 bytes (S = RN(dec(byte) * s_g), 1/S = RN(1/S)),
+//                built once at CTA start;
+//                warps 0..3 (one per tensor-memory lane quarter) finally read
+//                D_partial from tensor memory.
+// The kernel is a programmatic dependent of the one before it in the stream:
+// barrier set-up, tensor-memory allocation and the tensor-map prefetch run
+// before griddepcontrol.wait, and it lets its own dependent (the linear) start
+// launching at once.  Memory traffic per element: 2 bytes in, 0.5625 out.
 #include "common.cuh"
 #include "sm100.cuh"
 
 namespace svdq {
 namespace {
 
-constexpr int kBM = 128;               // rows per CTA tile
+constexpr int kBM = 128;               // rows of a stage slot (the MMA's M); a group holds at most this many
 constexpr int kBK = 64;                // channels per stage (128 bytes of bf16)
 constexpr int kStages = 9;
 constexpr int kTeams = 3;             // teams of quantiser warps take stages in turn
@@ -77,6 +88,7 @@ struct QuantArgs {
     uint32_t* err;
     int n_chunks;      // K / 64
     int split;         // CTAs along K (cluster size when R > 0)
+    int rows;          // rows per group (the TMA box height), <= 128
 };
 
 __device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t local_addr, uint32_t rank) {
@@ -88,8 +100,7 @@ __device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t local_addr, uint32_t r
     return v;
 }
 
-// E4M3 scale byte and saturation (t > 448) of t = RN(a / d), a >= 0, d > 0,
-// for two groups.  With y = RN(1 / d): |a y - a / d| <= 2^-24 a / d < 1 ulp,
+// E4M3 scale byte and saturation (t > 448) of t = RN(a / d), a >= 0, d > 0.  With y = RN(1 / d): |a y - a / d| <= 2^-24 a / d < 1 ulp,
 // rounding a y to q adds at most 1/2 ulp and t is within 1/2 ulp of a / d, so
 // |q - t| < 2 ulp (a power-of-two boundary between them only widens the
 // bit-pattern steps used below).  E4M3 rounding and the test t > 448 are
@@ -111,10 +122,6 @@ __device__ __forceinline__ uint32_t scale_byte_checked(float a, float d, float r
     return cvt_e4m3x2(t, 0.0f) & 0xFFu;
 }
 
-__device__ __forceinline__ uint32_t scale_bytes2(float a0, float a1, float d, float rd, uint32_t& sat) {
-    return scale_byte_checked(a0, d, rd, sat) | (scale_byte_checked(a1, d, rd, sat) << 8);
-}
-
 template <int R>
 __global__ void __launch_bounds__(kThreads)
 quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_down,
@@ -130,7 +137,12 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
 
     const int warp = threadIdx.x >> 5;
     const uint32_t lane = threadIdx.x & 31;
-    const int m_blk = blockIdx.x;
+    const int64_t row_base = static_cast<int64_t>(blockIdx.x) * args.rows;   // first row of this group
+    // Box rows that are real rows or zero fill inside the scale array's 128-row
+    // padding (their scale bytes are written); rows of the box at or past M are
+    // zero-filled by TMA.
+    const int64_t m_pad = (args.M + 127) / 128 * 128;
+    const int box_rows = static_cast<int>(min(static_cast<int64_t>(args.rows), m_pad - row_base));
     const int ky = blockIdx.y;
     const int c_begin = static_cast<int>(static_cast<int64_t>(ky) * args.n_chunks / args.split);
     const int c_end = static_cast<int>(static_cast<int64_t>(ky + 1) * args.n_chunks / args.split);
@@ -149,32 +161,29 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         tmem_alloc(tmem_slot, 32);
         tmem_relinquish();
     }
-    if (threadIdx.x < 128) {
-        // 1/S for every scale byte the RNE-satfinite conversion can produce (0x00..0x7E).
-        const float s_g = __ldg(args.s_g);
-        const float S = __fmul_rn(e4m3_to_f32(threadIdx.x), s_g);
-        reinterpret_cast<float*>(smem + L::kTabOff)[threadIdx.x] =
-            (threadIdx.x == 0x7F || S == 0.0f) ? 0.0f : __frcp_rn(S);
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_d = (R > 0) ? *tmem_slot : 0u;
+    pdl_launch_dependents();                  // the next kernel's set-up may overlap this one
 
     if (warp == kProducerWarp) {
         if (lane == 0) {
             prefetch_tmap(&tmap_x);
             if (R > 0) prefetch_tmap(&tmap_down);
+            pdl_wait();                           // X, 1/lambda and the tensor scale are written
+            const uint32_t x_bytes = static_cast<uint32_t>(args.rows) * kBK * 2;
             int issued = 0;
             for (int i = 0; i < n_local; ++i) {
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
                 if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) break;
                 const int col = (c_begin + i) * kBK;
-                mbar_arrive_expect_tx(&full[s], kXTileBytes + L::kDownTileBytes + (args.inv_lambda ? kBK * 4 : 0));
+                mbar_arrive_expect_tx(&full[s], x_bytes + L::kDownTileBytes + (args.inv_lambda ? kBK * 4 : 0));
                 if (args.inv_lambda)
                     bulk_load(smem + L::kIlamOff + s * kBK * 4, args.inv_lambda + col, kBK * 4, &full[s]);
-                tma_load_2d(smem + L::kXOff + s * kXTileBytes, &tmap_x, &full[s], col, m_blk * kBM);
+                tma_load_2d(smem + L::kXOff + s * kXTileBytes, &tmap_x, &full[s], col,
+                            static_cast<int32_t>(row_base));
                 if (R > 0)
                     tma_load_2d(smem + L::kDownOff + s * L::kDownTileBytes, &tmap_down, &full[s], col, 0);
                 ++issued;
@@ -205,6 +214,15 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         }
     } else {
         // ------------------------------------------------------------ quantisers
+        pdl_wait();                               // the tensor scale is written
+        if (threadIdx.x < 128) {
+            // 1/S for every scale byte the RNE-satfinite conversion can produce (0x00..0x7E).
+            const float s_g0 = __ldg(args.s_g);
+            const float S = __fmul_rn(e4m3_to_f32(threadIdx.x), s_g0);
+            reinterpret_cast<float*>(smem + L::kTabOff)[threadIdx.x] =
+                (threadIdx.x == 0x7F || S == 0.0f) ? 0.0f : __frcp_rn(S);
+        }
+        asm volatile("bar.sync 1, %0;" :: "n"(kQuantWarps * 32) : "memory");
         const float s_g = __ldg(args.s_g);
         const float d = __fmul_rn(6.0f, s_g);
         const float rd = __frcp_rn(d);
@@ -222,15 +240,28 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         const int rw = lane >> 2;
         const int b = lane & 3;
         const int r0 = (warp % kTeamWarps) * 16 + rw;
-        const int64_t grow0 = static_cast<int64_t>(m_blk) * kBM + r0;
+        const int r1 = r0 + 8;
+        const int64_t grow0 = row_base + r0;
         const int64_t grow1 = grow0 + 8;
+        // rows past the box hold stale shared memory: nothing of them is stored or counted
+        const bool box0 = r0 < box_rows, box1 = r1 < box_rows;
+        const bool code0 = box0 && grow0 < M, code1 = box1 && grow1 < M;
         const int ph0 = ((2 * b) ^ (r0 & 7)) << 4;
         const int ph1 = ((2 * b + 1) ^ (r0 & 7)) << 4;
         const uint64_t one2 = pack_f32x2(1.0f, 1.0f);
+        // A warp whose 16 rows all lie past this group's box has nothing to
+        // quantise: it only keeps the ring's protocol (wait for each of its
+        // team's stages, release it), so the work per stage follows the rows.
+        const bool idle = (warp % kTeamWarps) * 16 >= box_rows;
         for (int i = team; i < n_local; i += kTeams) {
             const int s = i % kStages;
             const uint32_t ph = (i / kStages) & 1;
             if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
+            if (idle) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                continue;
+            }
             const int chunk = c_begin + i;
             const uint8_t* tile = smem + L::kXOff + s * kXTileBytes;
             const uint4 u0 = *reinterpret_cast<const uint4*>(tile + r0 * 128 + ph0);
@@ -262,8 +293,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             const float aa = absmax16(xa), ab = absmax16(xb);
             // Scale bytes and saturation of both rows from t = RN(a / d), through
             // the product with 1/d where that is provably the same (see scale_from_amax).
-            uint32_t sat2 = 0;
-            const uint32_t sf2 = scale_bytes2(aa, ab, d, rd, sat2);   // byte 0: row r0, byte 1: row r0 + 8
+            uint32_t sat_a = 0, sat_b = 0;
+            const uint32_t sf2 = scale_byte_checked(aa, d, rd, sat_a) |
+                                 (scale_byte_checked(ab, d, rd, sat_b) << 8);   // byte 0: row r0, byte 1: row r0 + 8
             const float rsa = rs_tab[sf2 & 0xFFu], rsb = rs_tab[sf2 >> 8];
             const uint64_t ra = pack_f32x2(rsa, rsa), rb = pack_f32x2(rsb, rsb);
             uint64_t qa[8], qb[8];
@@ -276,7 +308,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                                         cvt_e2m1x8_pairs(qa[4], qa[5], qa[6], qa[7]));
             const uint2 cb = make_uint2(cvt_e2m1x8_pairs(qb[0], qb[1], qb[2], qb[3]),
                                         cvt_e2m1x8_pairs(qb[4], qb[5], qb[6], qb[7]));
-            sat += sat2;
+            sat += (box0 ? sat_a : 0u) + (box1 ? sat_b : 0u);
             // scale words of both rows: bytes of lanes 4 rw .. 4 rw + 3 (groups b = 0..3)
             const uint32_t n1 = __shfl_down_sync(0xffffffffu, sf2, 1);
             const uint32_t n2 = __shfl_down_sync(0xffffffffu, sf2, 2);
@@ -286,13 +318,30 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);        // shared memory of this stage no longer read
             uint8_t* cbase = args.codes + chunk * (kBK / 2) + b * 8;
-            if (grow0 < M) *reinterpret_cast<uint2*>(cbase + grow0 * half_k) = ca;
-            if (grow1 < M) *reinterpret_cast<uint2*>(cbase + grow1 * half_k) = cb;
+            if (code0) *reinterpret_cast<uint2*>(cbase + grow0 * half_k) = ca;
+            if (code1) *reinterpret_cast<uint2*>(cbase + grow1 * half_k) = cb;
             if (b == 0) {
-                uint8_t* atom = args.sf + (static_cast<int64_t>(m_blk) * atoms_k + chunk) * 512;
-                const int r1 = r0 + 8;
-                *reinterpret_cast<uint32_t*>(atom + (r0 & 31) * 16 + ((r0 >> 5) & 3) * 4) = __byte_perm(x01, x23, 0x5410);
-                *reinterpret_cast<uint32_t*>(atom + (r1 & 31) * 16 + ((r1 >> 5) & 3) * 4) = __byte_perm(x01, x23, 0x7632);
+                // a row's word in its 128-row block's 512-byte atom of this chunk
+                if (box0)
+                    *reinterpret_cast<uint32_t*>(args.sf + ((grow0 >> 7) * atoms_k + chunk) * 512 +
+                                                 (grow0 & 31) * 16 + ((grow0 >> 5) & 3) * 4) =
+                        __byte_perm(x01, x23, 0x5410);
+                if (box1)
+                    *reinterpret_cast<uint32_t*>(args.sf + ((grow1 >> 7) * atoms_k + chunk) * 512 +
+                                                 (grow1 & 31) * 16 + ((grow1 >> 5) & 3) * 4) =
+                        __byte_perm(x01, x23, 0x7632);
+            }
+        }
+        // Padding rows of the scale array past the last group's box (the box ends
+        // before the 128-row boundary): zero scale words for this CTA's chunks.
+        if (row_base + args.rows < m_pad && row_base + args.rows >= M) {
+            const int64_t pad0 = row_base + args.rows;
+            const int64_t n_pad = (m_pad - pad0) * n_local;
+            for (int64_t t = threadIdx.x; t < n_pad; t += kQuantWarps * 32) {
+                const int64_t row = pad0 + t / n_local;
+                const int64_t chunk = c_begin + t % n_local;
+                *reinterpret_cast<uint32_t*>(args.sf + ((row >> 7) * atoms_k + chunk) * 512 + (row & 31) * 16 +
+                                             ((row >> 5) & 3) * 4) = 0u;
             }
         }
         // saturation count: one atomic per warp
@@ -345,10 +394,11 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             const int cr = static_cast<int>(cluster_ctarank());
             const int q0 = cr * kNq / split, q1 = (cr + 1) * kNq / split;
             const int row = warp * 32 + lane;
-            const int64_t grow = static_cast<int64_t>(m_blk) * kBM + row;
+            const int64_t grow = row_base + row;
+            const bool row_ok = row < args.rows && grow < args.M;
             const uint32_t base = smem_u32(smem + L::kPartOff) + row * L::kPartStride * 4;
             if (split == 1) {
-                if (grow < args.M) {
+                if (row_ok) {
                     const float4* src = reinterpret_cast<const float4*>(smem + L::kPartOff) + row * (L::kPartStride / 4);
                     float4* dst = reinterpret_cast<float4*>(args.D + grow * R);
 #pragma unroll
@@ -364,7 +414,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                         for (int c = 0; c < kMaxSplit; ++c)
                             if (q0 + t0 + t < q1 && c < split)
                                 got[t][c] = ld_dsmem_f32x4(base + (q0 + t0 + t) * 16, c);
-                    if (grow < args.M) {
+                    if (row_ok) {
                         float4* dst = reinterpret_cast<float4*>(args.D + grow * R);
 #pragma unroll
                         for (int t = 0; t < 2; ++t) {
@@ -392,12 +442,70 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     }
 }
 
+// Work split of an M x K problem over `sms` SMs (one CTA fits per SM): K slices
+// per row group (a cluster, at most 4, only when whole 128-row tiles leave SMs
+// for it) and rows per group (at most 128, at least 16 where M allows) so that
+// groups x slices comes as close to the SM count as the rows allow.
+struct QuantPlan {
+    int split;
+    int rows;
+    int64_t groups;
+};
+
+inline QuantPlan plan_quantize(int64_t M, int n_chunks, int64_t sms, int64_t max_clusters) {
+    QuantPlan p{};
+    const int64_t m_tiles = (M + kBM - 1) / kBM;
+    const int64_t per_tile = sms / m_tiles;
+    p.split = static_cast<int>(per_tile < 1 ? 1 : (per_tile > kMaxSplit ? kMaxSplit : per_tile));
+    if (p.split > n_chunks) p.split = n_chunks;
+    int64_t groups_max = sms / p.split > 0 ? sms / p.split : 1;
+    // clusters are placed whole inside a GPC: never more than fit at once
+    if (p.split > 1 && max_clusters > 0 && groups_max > max_clusters) groups_max = max_clusters;
+    int64_t rows = (M + groups_max - 1) / groups_max;
+    rows = (rows + 7) / 8 * 8;                    // whole 8-row swizzle groups
+    if (rows > kBM) rows = kBM;                   // more rows than one wave holds: whole 128-row groups
+    if (rows > M) rows = M;
+    p.rows = static_cast<int>(rows);
+    p.groups = (M + rows - 1) / rows;
+    return p;
+}
+
 template <int R>
 int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const QuantArgs& base, const void* down,
                     cudaStream_t st) {
+    QuantArgs a = base;
+    a.n_chunks = static_cast<int>(K / kBK);
+    const int64_t sms = device_sm_count() > 0 ? device_sm_count() : 148;
+    const uint32_t smem = QSmem<R>::kBytes + 1024;
+    auto kern = quantize_act_kernel<R>;
+    static std::atomic<uint64_t> smem_set{0};
+    if (!set_dynamic_smem_once(kern, smem, smem_set)) return SVDQ_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    // clusters of 4 along K that fit on the device at once (0: unknown)
+    int max_clusters = 0;
+    if (R > 0) {
+        cfg.gridDim = dim3(1, kMaxSplit, 1);
+        attr[0].val.clusterDim.y = kMaxSplit;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess) max_clusters = 0;
+    }
+    const QuantPlan plan = plan_quantize(M, a.n_chunks, sms, max_clusters);
+    if (plan.groups > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
+    a.split = plan.split;
+    a.rows = plan.rows;
     CUtensorMap tx, td;
-    if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, K, M, ldx * 2, kBK, kBM,
-                        CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, K, M, ldx * 2, kBK,
+                        static_cast<uint32_t>(plan.rows), CU_TENSOR_MAP_SWIZZLE_128B))
         return SVDQ_ERR_CUDA;
     if (R > 0) {
         if (!encode_tmap_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, down, K, R, K * 2, kBK, R,
@@ -406,35 +514,10 @@ int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const Quan
     } else {
         td = tx;
     }
-    QuantArgs a = base;
-    a.n_chunks = static_cast<int>(K / kBK);
-    const int64_t m_tiles = (M + kBM - 1) / kBM;
-    // Split K across up to 4 CTAs of a cluster, only as far as the grid still runs in one
-    // wave (one CTA fits per SM): a second wave costs more than the split saves (measured
-    // on B200: 12288 x 5120 takes 54 us unsplit, 60 us split in two or four).
-    const int64_t sms = device_sm_count() > 0 ? device_sm_count() : 148;
-    int64_t per_tile = sms / m_tiles;
-    int split = static_cast<int>(per_tile < 1 ? 1 : (per_tile > kMaxSplit ? kMaxSplit : per_tile));
-    if (split > a.n_chunks) split = a.n_chunks;
-    a.split = split;
-    if (m_tiles > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
 
-    const uint32_t smem = QSmem<R>::kBytes + 1024;
-    auto kern = quantize_act_kernel<R>;
-    static std::atomic<uint64_t> smem_set{0};
-    if (!set_dynamic_smem_once(kern, smem, smem_set)) return SVDQ_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(m_tiles), static_cast<unsigned>(split), 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = (R > 0) ? split : 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(plan.groups), static_cast<unsigned>(plan.split), 1);
+    attr[0].val.clusterDim.y = (R > 0) ? plan.split : 1;
+    cfg.numAttrs = 2;
     return launch_status(cudaLaunchKernelEx(&cfg, kern, tx, td, a));
 }
 

@@ -305,8 +305,12 @@ int score_lambda_launch(const void* Yq, const void* Yref, int64_t M, int64_t N, 
         if (!set_dynamic_smem_once(score_stream_kernel, kStreamSmem, smem_set)) return SVDQ_ERR_CUDA;
         uint32_t* err = device_error_word();
         if (err == nullptr) return SVDQ_ERR_CUDA;
+        // cooperative: never more CTAs than can be resident together
+        const int64_t resident = coresident_grid(score_stream_kernel, kStreamThreads, kStreamSmem);
+        if (resident < 1) return SVDQ_ERR_CUDA;
         const int64_t sms = device_sm_count() > 0 ? device_sm_count() : 148;
-        const int64_t grid = chunks < sms ? chunks : sms;
+        int64_t grid = chunks < sms ? chunks : sms;
+        if (grid > resident) grid = resident;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
         cfg.blockDim = dim3(kStreamThreads, 1, 1);

@@ -77,22 +77,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity to complete.  On timeout
-// it records `code` in the device error word, raises the CTA-wide abort flag
-// (so the other roles stop waiting too) and returns false.  It also returns
-// false at once when another role already raised the abort flag.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                          uint32_t* err_word, uint32_t code) {
+// (`limit` cycles) it records `code` in the device error word, raises the
+// CTA-wide abort flag (so the other roles stop waiting too) and returns false.
+// It also returns false at once when another role already raised the abort flag.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                                uint32_t* err_word, uint32_t code, long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long start = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (clock64() - start > kWaitLimitCycles) {
+        if (clock64() - start > limit) {
             *abort_flag = 1u;
             atomicCAS(err_word, 0u, code);
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                          uint32_t* err_word, uint32_t code) {
+    return mbar_wait_limit(bar, parity, abort_flag, err_word, code, kWaitLimitCycles);
 }
 
 // ---------------------------------------------------------------------------

@@ -117,6 +117,26 @@ def svdq_calib_lambda(x: torch.Tensor, segs: Segs = None, w: Optional[torch.Tens
 
 
 @_on_tensor_device
+def svdq_calib_lambda_stored_w(x: torch.Tensor, segs: Segs, amax_w: torch.Tensor, stream=None) -> dict:
+    """svdq_calib_lambda against a stored weight absmax (fp32 [K] device tensor): reads only x."""
+    lib = _lib.load()
+    _check_bf16(x, "x")
+    m, k = x.shape
+    ldx = _row_stride(x, "x")
+    if amax_w.dtype != torch.float32 or amax_w.numel() != k or not amax_w.is_contiguous():
+        raise ValueError("amax_w must be a contiguous float32 tensor of K values")
+    dev = x.device
+    ax = torch.empty(k, dtype=torch.float32, device=dev)
+    lam = torch.empty(k, dtype=torch.float32, device=dev)
+    inv = torch.empty(k, dtype=torch.float32, device=dev)
+    s_g = torch.empty(1, dtype=torch.float32, device=dev)
+    arr, n_seg = _lib.seg_array(segs)
+    _lib.check("svdq_calib_lambda_stored_w", lib.svdq_calib_lambda_stored_w(
+        _ptr(x), m, k, ldx, arr, n_seg, _ptr(amax_w), _ptr(ax), _ptr(lam), _ptr(inv), _ptr(s_g), _stream(stream)))
+    return dict(amax_x=ax, amax_w=amax_w, lam=lam, inv_lam=inv, s_g=s_g)
+
+
+@_on_tensor_device
 def svdq_quantize_act(x: torch.Tensor, inv_lambda: Optional[torch.Tensor], s_g: torch.Tensor,
                       down: Optional[torch.Tensor] = None, sat_count: Optional[torch.Tensor] = None,
                       out: Optional[dict] = None, stream=None) -> dict:

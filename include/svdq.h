@@ -123,6 +123,20 @@ int svdq_calib_lambda(const void* X, int64_t M, int64_t K, int64_t ldx,
                       float* s_g, void* stream);
 
 /*
+ * svdq_calib_lambda_stored_w -- svdq_calib_lambda against a weight absmax that
+ * was reduced before (the same passages).  The weight of a converted layer does
+ * not change, so its absmax amax_w[j] = max over n of |W[n, j]| (device fp32
+ * [K], an input here, e.g. the amax_w output of one svdq_calib_lambda call over
+ * W) is kept, and each calibration reads only the selected rows of X.  Outputs
+ * amax_x, lambda, inv_lambda and s_g are bit for bit those of svdq_calib_lambda
+ * with that W.  Errors as svdq_calib_lambda; SVDQ_ERR_INVALID_ARG if amax_w is
+ * NULL.
+ */
+int svdq_calib_lambda_stored_w(const void* X, int64_t M, int64_t K, int64_t ldx,
+                               const svdq_seg* segs, int n_seg, const float* amax_w,
+                               float* amax_x, float* lambda, float* inv_lambda, float* s_g, void* stream);
+
+/*
  * svdq_quantize_act -- smooth and quantise activations per token to NVFP4 and
  * produce the low-rank down-projection ("MiniMax-H3 NVFP4 ...", section "Why";
  * "MiniMax-H3 . SVDQuant W4A4", opening section).
@@ -172,8 +186,11 @@ int svdq_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx,
  * D: device fp32 [M, r] (row stride r), NULL iff r == 0; up: device bf16 [N, r]
  * (row stride r), NULL iff r == 0; bias: device bf16 [N] or NULL.
  * Y: device [M, N] with row stride ldy; out_dtype 0 = bf16 (round to nearest
- * even), 1 = fp32.  Requirements: K % 256 == 0, N % 256 == 0, M >= 1,
- * r in {0, 16, 32}; otherwise SVDQ_ERR_UNSUPPORTED.
+ * even), 1 = fp32.  Requirements: K % 64 == 0 (one scale atom of 4 groups),
+ * N % 128 == 0 (one 128-row scale block), M >= 1, r in {0, 16, 32}; otherwise
+ * SVDQ_ERR_UNSUPPORTED.  The tensor cores take 256 channels and 256 columns per
+ * step: a ragged last step reads zero codes and zero scales (it adds nothing)
+ * and columns past N are not written.
  */
 int svdq_linear(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g_act,
                 const float* D, int r,
@@ -314,7 +331,7 @@ int svdq_residual(const void* W, int64_t N, int64_t K, int64_t ldw, const float*
  * (tcgen05 kind::mxf8f6f4 with E8M0 block scales).  A from svdq_quantize_mxfp8 of
  * X [M, K], W from it on the weight [N, K]; bias bf16 [N] or NULL; Y bf16 [M, N]
  * (device, row stride ldy >= N, ldy * 2 a multiple of 16, 16-byte aligned).
- * K % 128 == 0, N % 256 == 0, M >= 1.  Asynchronous on `stream`.
+ * K % 128 == 0, N % 128 == 0, M >= 1.  Asynchronous on `stream`.
  */
 size_t svdq_mxfp8_sf_bytes(int64_t rows, int64_t K);
 int svdq_quantize_mxfp8(const void* X, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* sf,
@@ -373,6 +390,23 @@ int svdq_bits_lost(const float* amax_x, int64_t ld_amax, int n_mod, const float*
  * synchronisation itself failed).
  */
 int svdq_device_error(void* stream, uint32_t* code);
+
+/*
+ * svdq_debug_arm_calib_timeout -- test hook for the bounded waits (no page has
+ * a counterpart).  Arms the next svdq_calib_lambda call in this process, on
+ * whichever device it runs: in that call the first CTA's loader leaves its
+ * ring unit number `unit` (0-based, within that CTA's range of 32-row x
+ * 256-channel units) unloaded, and the CTA's waits give up after
+ * `wait_limit_cycles` SM cycles instead of the usual ~2 s.  The consumer wait
+ * for the missing unit therefore runs out: the kernel records code 1 ("a
+ * consumer waited too long for a TMA stage") in the error word, stops its
+ * other roles, waits for its own copies in flight and returns.  Nothing is
+ * faulted and the context stays usable; that call's outputs are not valid.
+ * One-shot: the following calls run normally.  Returns SVDQ_ERR_INVALID_ARG
+ * for unit < 0 or a limit below 100000 cycles.  A unit at or past the CTA's
+ * range arms nothing that call.
+ */
+int svdq_debug_arm_calib_timeout(int64_t unit, int64_t wait_limit_cycles);
 
 #ifdef __cplusplus
 }

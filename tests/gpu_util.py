@@ -96,3 +96,24 @@ def d_tolerance(x_bits: np.ndarray, down_bits: np.ndarray) -> np.ndarray:
     ax = np.abs(O.bf16_to_f64(x_bits))
     ad = np.abs(O.bf16_to_f64(down_bits))
     return n * 2.0 ** -24 * (ax @ ad.T) + 1e-30
+
+
+def check_d(d_gpu: np.ndarray, d64: np.ndarray, x_bits: np.ndarray, down_bits: np.ndarray) -> float:
+    """D against the fp64 value: every element within the worst-case bound of
+    d_tolerance, and the whole array norm-wise within ((K/16)/2 + 4) * 2^-24.
+
+    The recursive-summation bound gives each element an error of at most
+    n 2^-24 sum|x down| for n = K/16 MMA steps.  The tensor core does not round
+    like n sequential fp32 additions, so the typical error is not a random walk
+    of roundings either: norm-wise it came out at 0.64 n 2^-24 relative on the
+    16384 x 20480 FFN down-projection input (n = 1280) and lower on the smaller
+    K.  Half of the factor n, applied to the norm, still fails an accumulation
+    that went wrong on average -- a dropped or doubled partial, a lost split-K
+    term, a partial rounded to bf16 -- although each element may still fit the
+    worst case."""
+    k = x_bits.shape[1]
+    assert np.all(np.abs(d_gpu - d64) <= d_tolerance(x_bits, down_bits))
+    rel = rel_l2(d_gpu.astype(np.float64), d64)
+    bound = ((k / 16) / 2 + 4) * 2.0 ** -24          # + 4 units: the roundings of a single MMA step
+    assert rel <= bound, f"D rel-L2 {rel:.3e} above {bound:.3e}"
+    return rel

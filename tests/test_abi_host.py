@@ -105,8 +105,10 @@ def test_linear_rejects_bad_arguments():
         return lib.svdq_linear(a["a"], a["asf"], a["sga"], a["d"], a["r"], a["w"], a["wsf"], a["sgw"], a["up"],
                                a["bias"], a["y"], a["ldy"], a["dt"], a["m"], a["n"], a["k"], None)
 
-    assert call(k=320) == _lib.SVDQ_ERR_UNSUPPORTED          # K % 256
-    assert call(n=384, ldy=384) == _lib.SVDQ_ERR_UNSUPPORTED  # N % 256
+    assert call(k=288) == _lib.SVDQ_ERR_UNSUPPORTED          # K % 64
+    assert call(n=320, ldy=320) == _lib.SVDQ_ERR_UNSUPPORTED  # N % 128
+    # K % 64 and N % 128 pass validation; with no GPU the call stops at the device check
+    assert call(k=320, n=384, ldy=384) == _lib.SVDQ_ERR_NO_DEVICE
     assert call(r=16) == _lib.SVDQ_ERR_INVALID_ARG           # rank without D / up
     assert call(r=24, d=p, up=p) == _lib.SVDQ_ERR_UNSUPPORTED
     assert call(dt=2) == _lib.SVDQ_ERR_INVALID_ARG

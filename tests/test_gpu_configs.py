@@ -16,7 +16,7 @@ import torch
 
 import synthetic as S
 from oracle import svdq_oracle as O
-from gpu_util import (check_codes, check_linear_bf16, check_linear_f32, d_tolerance, dev_bits, dev_f32,
+from gpu_util import (check_codes, check_d, check_linear_bf16, check_linear_f32, dev_bits, dev_f32,
                       host_bits, requires_cuda)
 
 pytestmark = [pytest.mark.gpu, requires_cuda]
@@ -77,7 +77,7 @@ def _check_layer(lib, L, c, wt, rows, cols):
     got_sf = O.sf_from_mma_layout(q["sf"].cpu().numpy(), L.m, L.k)[rows]
     assert np.array_equal(got_sf, sf), "activation scale bytes"
     d64 = O.lowrank_down(L.x[rows], wt["down"])
-    assert np.all(np.abs(q["d"].cpu().numpy()[rows] - d64) <= d_tolerance(L.x[rows], wt["down"]))
+    check_d(q["d"].cpu().numpy()[rows], d64, L.x[rows], wt["down"])
     wcodes, wsf, _ = O.quantize_blocks(wt["r"][cols], None, wt["s_g"])
     check_codes(wt["wq"]["codes"], wcodes, rows=cols)
     args = (q["codes"], q["sf"], s_ga, q["d"], wt["wq"]["codes"], wt["wq"]["sf"], wt["wsg"], dev_bits(wt["up"]),

@@ -54,6 +54,9 @@ CASES = [
     (2048, 5120, 256, 32, [(0, 1000), (1000, 2048)]),
     (4000, 5120, 256, 16, [(0, 4000), (17, 3001), (3001, 3001), (3500, 4000)]),
     (1536, 4096, 1024, 0, [(0, 1536)]),
+    # ragged: N % 256 == 128 (the last tile's second column half lies past N) and
+    # K % 256 == 64 (a last partial channel stage)
+    (700, 1152, 1344, 32, [(0, 350), (350, 700)]),
 ]
 
 

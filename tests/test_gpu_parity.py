@@ -10,7 +10,7 @@ import torch
 
 import synthetic as S
 from oracle import svdq_oracle as O
-from gpu_util import (check_codes, check_linear_bf16, check_linear_f32, check_sf, d_tolerance, dev_bits, dev_f32,
+from gpu_util import (check_codes, check_d, check_linear_bf16, check_linear_f32, check_sf, dev_bits, dev_f32,
                       host_bits, requires_cuda, rel_l2)
 
 pytestmark = [pytest.mark.gpu, requires_cuda]
@@ -54,6 +54,24 @@ def test_calib_row_segments(lib, segs):
     assert g["s_g"].item() == float(c["s_g"])
 
 
+@pytest.mark.parametrize("segs", [None, [(0, 0), (5, 9), (100, 1000)], [(999, 1000)]])
+def test_calib_stored_weight_absmax_equals_reading_the_weight(lib, segs):
+    """The weight's absmax kept from one call over W gives the same lambda, 1/lambda
+    and s_g as reading W again, bit for bit, and as the oracle."""
+    x = S.random_bf16((1000, 1280), 31, 2.0)
+    w = S.random_bf16((300, 1280), 32, 0.02)
+    w_bits = w.copy()
+    w_bits[:, 5] = 0                                   # a zero weight channel: lambda = 1 there
+    c = O.calib(x, segs, w_bits)
+    xd, wd = dev_bits(x), dev_bits(w_bits)
+    full = lib.svdq_calib_lambda(xd, segs, wd)
+    stored = lib.svdq_calib_lambda_stored_w(xd, segs, full["amax_w"])
+    for key, gk in (("ax", "amax_x"), ("lam", "lam"), ("inv_lam", "inv_lam")):
+        assert np.array_equal(stored[gk].cpu().numpy(), c[key]), key
+        assert torch.equal(stored[gk], full[gk]), key
+    assert stored["s_g"].item() == float(c["s_g"]) == full["s_g"].item()
+
+
 @pytest.mark.parametrize("m,k", [(1, 8), (3, 72), (1000, 264)])
 def test_calib_ragged_and_without_weight(lib, m, k):
     x = S.random_bf16((m, k), 21, 1.0)
@@ -89,10 +107,6 @@ def test_calib_wide_k_many_strips_and_repeated_calls(lib):
         del g
 
 
-def _d_tolerance(x_bits, down_bits):
-    return d_tolerance(x_bits, down_bits)
-
-
 def test_quantize_cfg0_bit_exact(lib, cfg0):
     L, segs, c, conv = cfg0
     codes, sf, n_sat = O.quantize_blocks(L.x, c["inv_lam"], c["s_g"])
@@ -103,7 +117,7 @@ def test_quantize_cfg0_bit_exact(lib, cfg0):
     check_sf(q["sf"], sf, L.m, L.k)
     assert int(sat.item()) == n_sat
     d64 = O.lowrank_down(L.x, conv["down"])
-    assert np.all(np.abs(q["d"].cpu().numpy() - d64) <= _d_tolerance(L.x, conv["down"]))
+    check_d(q["d"].cpu().numpy(), d64, L.x, conv["down"])
 
 
 def _outlier_x(m, k, seed):
@@ -131,7 +145,7 @@ def test_quantize_shapes(lib, m, k, r):
     assert int(sat.item()) == n_sat
     if r:
         d64 = O.lowrank_down(x, down)
-        assert np.all(np.abs(q["d"].cpu().numpy() - d64) <= _d_tolerance(x, down))
+        check_d(q["d"].cpu().numpy(), d64, x, down)
 
 
 def test_quantize_ties_saturation_and_signed_zero(lib):
@@ -279,7 +293,14 @@ def test_linear_cfg0(lib, cfg0):
 @pytest.mark.parametrize("m,n,k,r,bias", [
     (128, 256, 256, 0, True), (1, 256, 512, 16, True), (200, 512, 768, 32, False), (384, 256, 1024, 32, True),
     (300, 768, 512, 16, True), (129, 512, 2048, 0, False),
-    (3200, 1024, 256, 32, True)])     # 100 whole tiles: a last wave too full to split into half tiles
+    (3200, 1024, 256, 32, True),      # 100 whole tiles: a last wave too full to split into half tiles
+    # several tiles per CTA, each closed by its low-rank stage in the operand ring:
+    # 2, 3, 4 and 12 ring positions per tile against the ring's 4 slots, and an odd
+    # number of K stages (the last scale batch half past K)
+    (8192, 2048, 256, 32, True), (2048, 4608, 512, 16, True), (1536, 6144, 768, 32, False),
+    (2560, 4096, 2816, 32, True),
+    # ragged N (a multiple of 128, not of 256) and K (a multiple of 64, not of 256)
+    (300, 384, 320, 32, True), (129, 640, 576, 16, True), (2048, 1152, 1344, 32, False)])
 def test_linear_shapes(lib, m, n, k, r, bias):
     x = _outlier_x(m, k, 3 * m + k)
     w = S.random_bf16((n, k), n + k, 0.02)
@@ -368,7 +389,7 @@ def test_config1_calib_quantize_full(lib, cfg1):
     assert int(sat.item()) == n_sat
     rows = np.arange(0, L.m, 61)
     d64 = O.lowrank_down(L.x[rows], conv["down"])
-    assert np.all(np.abs(q["d"].cpu().numpy()[rows] - d64) <= _d_tolerance(L.x[rows], conv["down"]))
+    check_d(q["d"].cpu().numpy()[rows], d64, L.x[rows], conv["down"])
 
 
 def test_config1_residual_and_linear_sampled(lib, cfg1):
