@@ -183,10 +183,13 @@ __device__ __forceinline__ void tile_coords(const LinearArgs& a, int tile, int& 
     }
 }
 
+// Two fp32 values rounded to nearest-even bf16 in one packed conversion
+// (cvt.rn.bf16x2.f32), `lo` in the low half: the same bits as two scalar
+// conversions, in half the conversion-pipe instructions.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-    const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-    return l | (h << 16);
+    uint32_t out;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(hi), "f"(lo));
+    return out;
 }
 
 // The tile's low-rank operands, written by the epilogue warps into the ring
@@ -221,20 +224,17 @@ __device__ __forceinline__ bool lr_stage(const LinearArgs& a, uint8_t* slot, uin
     const uint4* usrc = reinterpret_cast<const uint4*>(a.up + gn * r);
 #pragma unroll
     for (int c = 0; c < 4; ++c) u[c] = (c * 8 < r && gn < a.N) ? __ldg(usrc + c) : make_uint4(0, 0, 0, 0);
+    // D' = D / alpha as bf16 hi + lo pairs, formed before the wait
+    uint32_t hi[8], lo[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float x0 = __fmul_rn(dv[2 * j], inv_alpha);
+        const float x1 = __fmul_rn(dv[2 * j + 1], inv_alpha);
+        hi[j] = pack_bf16x2(x0, x1);
+        lo[j] = pack_bf16x2(__fsub_rn(x0, bf16_lo(hi[j])), __fsub_rn(x1, bf16_hi(hi[j])));
+    }
     const bool ok = mbar_wait(go_bar, parity, abort_flag, a.err, kErrWaitLowRank);
     if (ok) {
-        uint32_t hi[8], lo[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float x0 = __fmul_rn(dv[2 * j], inv_alpha);
-            const float x1 = __fmul_rn(dv[2 * j + 1], inv_alpha);
-            const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-            const float r0 = __fsub_rn(x0, __bfloat162float(h0));
-            const float r1 = __fsub_rn(x1, __bfloat162float(h1));
-            hi[j] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                    (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-            lo[j] = pack_bf16x2(r0, r1);
-        }
         uint8_t* rowp = slot + arow * 128;
         const int sw = arow & 7;
         *reinterpret_cast<uint4*>(rowp + (((2 * h) ^ sw) << 4)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -295,7 +295,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     // a last partial stage reads zero codes and zero scales past K (TMA fill): it adds nothing
     const int k_stages = static_cast<int>((args.K + kStageK - 1) / kStageK);
     const bool has_lr = args.r > 0;
-    // Ring positions per tile: the K stages, then the low-rank stage.
+    // Ring positions per tile: the low-rank stage, then the K stages.
     const int span = k_stages + (has_lr ? 1 : 0);
 
     if (threadIdx.x == 0) {
@@ -366,24 +366,15 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 int m_blk, n_blk;
                 tile_coords(args, tile, m_blk, n_blk);
-                for (int kb = 0; kb < k_stages; ++kb, ++it) {
-                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) { ok = false; break; }
-                    uint8_t* st = smem + L::kOffStages + s * kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], kStageBytes);
-                    tma_load_2d(st, &tmap_a, &full[s], kb * kBKBytes, m_blk * kBM);
-                    tma_load_2d(st + kATile, &tmap_b, &full[s], kb * kBKBytes, n_blk * kBN);
-                    if ((kb & 1) == 0 && !issue_scales()) { ok = false; break; }
-                    if (++s == kStagesT) { s = 0; ph ^= 1u; }
-                }
-                if (ok && has_lr) {
-                    // The low-rank stage: the epilogue warps fill this slot.  The
-                    // producer walks the ring in order, so its wait for the slot's
-                    // previous MMAs is the safe one (a parity wait tells only one
-                    // phase from the next); it hands the free slot to the epilogue
-                    // through lr_go, once the epilogue has written the previous
-                    // tile's stage (lr_done), so neither barrier ever runs two
-                    // phases ahead of its waiter.  Its arrival on full stands for
-                    // the copies.
+                if (has_lr) {
+                    // The low-rank stage opens the tile: the epilogue warps fill this
+                    // slot.  The producer walks the ring in order, so its wait for
+                    // the slot's previous MMAs is the safe one (a parity wait tells
+                    // only one phase from the next); it hands the free slot to the
+                    // epilogue through lr_go, once the epilogue has written the
+                    // previous tile's stage (lr_done), so neither barrier ever runs
+                    // two phases ahead of its waiter.  Its arrival on full stands
+                    // for the copies.
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) { ok = false; break; }
                     if (lr_tiles > 0 &&
                         !mbar_wait(lr_done, (lr_tiles - 1) & 1, abort_flag, args.err, kErrWaitLowRank)) {
@@ -394,6 +385,15 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     mbar_arrive(lr_go);
                     ++lr_tiles;
                     ++it;
+                    if (++s == kStagesT) { s = 0; ph ^= 1u; }
+                }
+                for (int kb = 0; kb < k_stages; ++kb, ++it) {
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) { ok = false; break; }
+                    uint8_t* st = smem + L::kOffStages + s * kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], kStageBytes);
+                    tma_load_2d(st, &tmap_a, &full[s], kb * kBKBytes, m_blk * kBM);
+                    tma_load_2d(st + kATile, &tmap_b, &full[s], kb * kBKBytes, n_blk * kBN);
+                    if ((kb & 1) == 0 && !issue_scales()) { ok = false; break; }
                     if (++s == kStagesT) { s = 0; ph ^= 1u; }
                 }
             }
@@ -424,6 +424,25 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
                 if (!mbar_wait(acc_empty, (local & 1) ^ 1, abort_flag, args.err, kErrWaitAccum)) break;
                 tc_fence_after();
+                if (has_lr) {
+                    // The low-rank term opens the tile and initialises the
+                    // accumulator: 4 kind::f16 MMAs (K = 64: 32 ranks of D'_hi, then
+                    // 32 of D'_lo, against up twice) from the ring slot the epilogue
+                    // warps filled while the previous tile was finishing.
+                    if (!mbar_try_wait(&full[s], ph) &&
+                        !mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitLowRank))
+                        break;
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + L::kOffStages + s * kStageBytes);
+                    const uint32_t b0 = a0 + kATile;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc_lr,
+                                 kk == 0 ? 0u : 1u);
+                    tc_commit(&empty[s]);
+                    if (++s == kStagesT) { s = 0; ph ^= 1u; }
+                }
+                const uint32_t acc0 = has_lr ? 1u : 0u;            // the first K stage starts the sum without it
                 for (int kb = 0; kb < k_stages; ++kb) {
                     if (!mbar_try_wait(&full[s], ph) &&
                         !mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) {
@@ -433,13 +452,14 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     tc_fence_after();
                     const uint64_t da = da0 + kStageDesc * s, db = db0 + kStageDesc * s;
                     const uint32_t sf = tmem + kTmemSf0 + s * kTmemSfStrideT;
+                    const uint32_t acc = kb == 0 ? acc0 : 1u;
                     if constexpr (kMx) {
-                        mma_mxf8(tmem, da, db, idesc_mxf8(kBM, kBN, 0), sf, sf + kTmemSfbOffT, kb == 0 ? 0u : 1u);
+                        mma_mxf8(tmem, da, db, idesc_mxf8(kBM, kBN, 0), sf, sf + kTmemSfbOffT, acc);
                         mma_mxf8(tmem, da + 2, db + 2, idesc_mxf8(kBM, kBN, 1), sf, sf + kTmemSfbOffT, 1u);
                         mma_mxf8(tmem, da + 4, db + 4, idesc_mxf8(kBM, kBN, 2), sf, sf + kTmemSfbOffT, 1u);
                         mma_mxf8(tmem, da + 6, db + 6, idesc_mxf8(kBM, kBN, 3), sf, sf + kTmemSfbOffT, 1u);
                     } else {
-                        mma_nvf4(tmem, da, db, idesc_f4, sf, sf + kTmemSfbOff, kb == 0 ? 0u : 1u);
+                        mma_nvf4(tmem, da, db, idesc_f4, sf, sf + kTmemSfbOff, acc);
                         mma_nvf4(tmem, da + 2, db + 2, idesc_f4, sf + 4, sf + kTmemSfbOff + 8, 1u);
                         mma_nvf4(tmem, da + 4, db + 4, idesc_f4, sf + 8, sf + kTmemSfbOff + 16, 1u);
                         mma_nvf4(tmem, da + 6, db + 6, idesc_f4, sf + 12, sf + kTmemSfbOff + 24, 1u);
@@ -448,22 +468,6 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     if (++s == kStagesT) { s = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
-                if (has_lr) {
-                    // The low-rank term closes the tile: 4 kind::f16 MMAs (K = 64:
-                    // 32 ranks of D'_hi, then 32 of D'_lo, against up twice) from
-                    // the ring slot the epilogue warps filled.
-                    if (!mbar_try_wait(&full[s], ph) &&
-                        !mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitLowRank))
-                        break;
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(smem + L::kOffStages + s * kStageBytes);
-                    const uint32_t b0 = a0 + kATile;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc_lr, 1u);
-                    tc_commit(&empty[s]);
-                    if (++s == kStagesT) { s = 0; ph ^= 1u; }
-                }
                 tc_commit(acc_full);
             }
         }
@@ -483,6 +487,10 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         uint32_t ph = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            if (has_lr) {                                   // the tile's low-rank stage is the epilogue's
+                ++it;
+                if (++s == kStagesT) { s = 0; ph ^= 1u; }
+            }
             for (int kb = 0; kb < k_stages; ++kb, ++it) {
                 if ((kb & 1) == 0) ++pair;
                 const int slot = pair & 1;
@@ -546,10 +554,6 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 if (lane == 0) mbar_arrive(&full[s]);
                 if (++s == kStagesT) { s = 0; ph ^= 1u; }
             }
-            if (ok && has_lr) {
-                ++it;
-                if (++s == kStagesT) { s = 0; ph ^= 1u; }
-            }
         }
     } else if constexpr (kScore) {
         // ------------------------------------------------------------ epilogue with scoring
@@ -590,6 +594,13 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         }
         if (etid == 0) prefetch_tmap(&tmap_r);
         const int32_t M32 = static_cast<int32_t>(args.M);
+        // the first tile's low-rank stage (ring position 0); a failure raises the
+        // abort flag, which the loop top reads
+        if (has_lr && static_cast<int>(blockIdx.x) < num_tiles) {
+            int m_0, n_0;
+            tile_coords(args, blockIdx.x, m_0, n_0);
+            lr_stage(args, smem + L::kOffStages, lr_go, 0u, &full[0], lr_done, m_0, n_0, inv_alpha, etid, abort_flag);
+        }
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             int m_blk, n_blk;
@@ -600,11 +611,16 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             bt[etid] = (args.bias && col0 + etid < args.N) ? args.bias[col0 + etid] : static_cast<uint16_t>(0);
             // bias staged, the previous tile's row sums consumed; leave together on abort
             if (bar_sync_or<1, kEpiWarps * 32>(*abort_flag != 0u)) break;
-            if (has_lr) {
-                const int64_t p = static_cast<int64_t>(local + 1) * span - 1;      // this tile's low-rank stage
+            if (has_lr && tile + static_cast<int>(gridDim.x) < num_tiles) {
+                // the next tile's low-rank stage (its first ring position), written
+                // while this tile's last K stages run
+                const int64_t p = static_cast<int64_t>(local + 1) * span;
                 const int slot = static_cast<int>(p % kStagesT);
-                if (!lr_stage(args, smem + L::kOffStages + slot * kStageBytes, lr_go, static_cast<uint32_t>(local & 1),
-                              &full[slot], lr_done, m_blk, n_blk, inv_alpha, etid, abort_flag))
+                int m_nx, n_nx;
+                tile_coords(args, tile + static_cast<int>(gridDim.x), m_nx, n_nx);
+                if (!lr_stage(args, smem + L::kOffStages + slot * kStageBytes, lr_go,
+                              static_cast<uint32_t>((local + 1) & 1), &full[slot], lr_done, m_nx, n_nx, inv_alpha,
+                              etid, abort_flag))
                     continue;                                // the abort flag is up: the loop top leaves
             }
             bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, local & 1, abort_flag, args.err, kErrWaitMma));
@@ -768,6 +784,13 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         pdl_wait();                                   // inputs of the earlier kernels are written
         const float alpha = kMx ? 1.0f : __fmul_rn(__ldg(args.s_g_act), __ldg(args.s_g_w));
         const float inv_alpha = __frcp_rn(alpha);
+        // the first tile's low-rank stage (ring position 0); a failure raises the
+        // abort flag, which the loop top reads
+        if (has_lr && static_cast<int>(blockIdx.x) < num_tiles) {
+            int m_0, n_0;
+            tile_coords(args, blockIdx.x, m_0, n_0);
+            lr_stage(args, smem + L::kOffStages, lr_go, 0u, &full[0], lr_done, m_0, n_0, inv_alpha, etid, abort_flag);
+        }
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             int m_blk, n_blk;
@@ -777,11 +800,16 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             bt[etid] = (args.bias && col0 + etid < args.N) ? args.bias[col0 + etid] : static_cast<uint16_t>(0);
             // bias staged; leave together on abort
             if (bar_sync_or<1, kEpiWarps * 32>(*abort_flag != 0u)) break;
-            if (has_lr) {
-                const int64_t p = static_cast<int64_t>(local + 1) * span - 1;      // this tile's low-rank stage
+            if (has_lr && tile + static_cast<int>(gridDim.x) < num_tiles) {
+                // the next tile's low-rank stage (its first ring position), written
+                // while this tile's last K stages run
+                const int64_t p = static_cast<int64_t>(local + 1) * span;
                 const int slot = static_cast<int>(p % kStagesT);
-                if (!lr_stage(args, smem + L::kOffStages + slot * kStageBytes, lr_go, static_cast<uint32_t>(local & 1),
-                              &full[slot], lr_done, m_blk, n_blk, inv_alpha, etid, abort_flag))
+                int m_nx, n_nx;
+                tile_coords(args, tile + static_cast<int>(gridDim.x), m_nx, n_nx);
+                if (!lr_stage(args, smem + L::kOffStages + slot * kStageBytes, lr_go,
+                              static_cast<uint32_t>((local + 1) & 1), &full[slot], lr_done, m_nx, n_nx, inv_alpha,
+                              etid, abort_flag))
                     continue;                                // the abort flag is up: the loop top leaves
             }
             if (!mbar_wait(acc_full, local & 1, abort_flag, args.err, kErrWaitMma)) continue;
