@@ -127,6 +127,7 @@ struct LinearArgs {
     int r;
     int m_tiles, n_tiles;
     int n_fastest;            // tile order: 1 = N fastest (the weight stays in L2), 0 = M fastest
+    int band;                 // blocks of the fastest-walked operand per band (see tile_coords)
     uint32_t* err;
     // Scoring fused into the epilogue (bf16 output only; the reference comes by tensor map).
     int write_y;              // 0: the output itself is not written
@@ -171,21 +172,32 @@ __device__ __forceinline__ void pair_add(float& hi, float& lo, float x) {
 }
 
 // Output tile -> (M block, N block).  The order decides what the CTAs working
-// at the same time share: walking the smaller operand's blocks fastest keeps
-// that operand resident in L2 while the other streams through once.
+// at the same time share: the smaller operand's blocks are walked fastest, so
+// each block of the other operand is read once while the smaller one is re-read
+// from L2.  When the smaller operand itself is larger than what the L2 keeps for
+// the SMs that read it (the 52 MB weight of the 16384 x 20480 -> 5120 layer was
+// read from DRAM again on every pass of the persistent grid), it is walked in
+// bands of `band` blocks: every block of the other operand passes under one band
+// before the next band starts, so the band stays resident and the larger operand
+// is read once per band.
 __device__ __forceinline__ void tile_coords(const LinearArgs& a, int tile, int& m_blk, int& n_blk) {
+    const int fast_tiles = a.n_fastest ? a.n_tiles : a.m_tiles;
+    const int slow_tiles = a.n_fastest ? a.m_tiles : a.n_tiles;
+    const int per_band = a.band * slow_tiles;                // tiles of one full band
+    const int b = tile / per_band;
+    const int r = tile - b * per_band;
+    const int f0 = b * a.band;
+    const int width = min(a.band, fast_tiles - f0);          // the last band may be narrower
+    const int fast = f0 + r % width, slow = r / width;
     if (a.n_fastest) {
-        n_blk = tile % a.n_tiles;
-        m_blk = tile / a.n_tiles;
+        n_blk = fast;
+        m_blk = slow;
     } else {
-        m_blk = tile % a.m_tiles;
-        n_blk = tile / a.m_tiles;
+        m_blk = fast;
+        n_blk = slow;
     }
 }
 
-// Two fp32 values rounded to nearest-even bf16 in one packed conversion
-// (cvt.rn.bf16x2.f32), `lo` in the low half: the same bits as two scalar
-// conversions, in half the conversion-pipe instructions.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t out;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(hi), "f"(lo));
@@ -336,6 +348,12 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             prefetch_tmap(&tmap_sfa);
             prefetch_tmap(&tmap_sfb);
             pdl_wait();                               // the activation codes and scales are written
+            // L2 policies: the operand walked fastest over the tiles (the smaller
+            // one) is re-read by every block row (or column) of the other, so it
+            // is kept; the other streams through once.
+            const uint64_t pol_keep = l2_evict_last_policy(), pol_once = l2_evict_first_policy();
+            const uint64_t pol_a = args.n_fastest ? pol_once : pol_keep;
+            const uint64_t pol_b = args.n_fastest ? pol_keep : pol_once;
             // Scale batches run one batch (two stages) ahead of the operands: the
             // batch a stage needs has landed by the time its operands do.
             int sf_tile = blockIdx.x, sf_kb = 0, issued = 0;
@@ -350,8 +368,9 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 uint8_t* dst = smem + L::kOffSf + slot * kSfSlot;
                 mbar_arrive_expect_tx(&sf_data[slot], kSfSlotT);
                 // scale atoms of stages sf_kb and sf_kb + 1 (a last odd stage reads zeros past K)
-                tma_load_3d(dst, &tmap_sfa, &sf_data[slot], 0, sf_kb * kSfHalvesPerStage, m_blk);
-                tma_load_3d(dst + kSfaPairT, &tmap_sfb, &sf_data[slot], 0, sf_kb * kSfHalvesPerStage, 2 * n_blk);
+                tma_load_3d_hint(dst, &tmap_sfa, &sf_data[slot], 0, sf_kb * kSfHalvesPerStage, m_blk, pol_a);
+                tma_load_3d_hint(dst + kSfaPairT, &tmap_sfb, &sf_data[slot], 0, sf_kb * kSfHalvesPerStage, 2 * n_blk,
+                                 pol_b);
                 ++issued;
                 sf_kb += 2;
                 if (sf_kb >= k_stages) {
@@ -391,8 +410,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) { ok = false; break; }
                     uint8_t* st = smem + L::kOffStages + s * kStageBytes;
                     mbar_arrive_expect_tx(&full[s], kStageBytes);
-                    tma_load_2d(st, &tmap_a, &full[s], kb * kBKBytes, m_blk * kBM);
-                    tma_load_2d(st + kATile, &tmap_b, &full[s], kb * kBKBytes, n_blk * kBN);
+                    tma_load_2d_hint(st, &tmap_a, &full[s], kb * kBKBytes, m_blk * kBM, pol_a);
+                    tma_load_2d_hint(st + kATile, &tmap_b, &full[s], kb * kBKBytes, n_blk * kBN, pol_b);
                     if ((kb & 1) == 0 && !issue_scales()) { ok = false; break; }
                     if (++s == kStagesT) { s = 0; ph ^= 1u; }
                 }
@@ -781,6 +800,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * (kBN / 2);
         uint16_t* bias_s = reinterpret_cast<uint16_t*>(smem + L::kOffBias);
         uint8_t* stg = smem + L::kOffEpi + ew * kYStageBytes;
+        const uint64_t pol_y = l2_evict_first_policy();
         pdl_wait();                                   // inputs of the earlier kernels are written
         const float alpha = kMx ? 1.0f : __fmul_rn(__ldg(args.s_g_act), __ldg(args.s_g_w));
         const float inv_alpha = __frcp_rn(alpha);
@@ -860,7 +880,9 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     fence_async_shared();
                     __syncwarp();
                     if (lane == 0 && grow0 < args.M && ccol + 16 * j < args.N) {   // boxes wholly past M or N are skipped
-                        tma_store_2d(&tmap_y, stg, static_cast<int32_t>(ccol) + 16 * j, grow0);
+                        // the output is not read again here: first out of L2, so it does
+                        // not push out the operands other tiles still read
+                        tma_store_2d_hint(&tmap_y, stg, static_cast<int32_t>(ccol) + 16 * j, grow0, pol_y);
                         bulk_commit_group();
                     }
                 }
@@ -1054,6 +1076,16 @@ int linear_prepare(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g
     a->m_tiles = static_cast<int>(m_tiles);
     a->n_tiles = static_cast<int>(n_tiles);
     a->n_fastest = N <= M ? 1 : 0;                       // the weight is the smaller operand
+    {
+        // Bands of the fastest-walked operand no larger than kBandBytes (the
+        // whole operand when it is smaller): each die's L2 half (~63 MB) must
+        // hold the band and the other operand's blocks in flight.
+        constexpr int64_t kBandBytes = int64_t(40) << 20;
+        const int64_t fast_tiles = a->n_fastest ? n_tiles : m_tiles;
+        const int64_t block_bytes = (a->n_fastest ? int64_t(kBN) : int64_t(kBM)) * row_bytes;
+        const int64_t bands = (fast_tiles * block_bytes + kBandBytes - 1) / kBandBytes;
+        a->band = static_cast<int>((fast_tiles + bands - 1) / bands);
+    }
     a->err = err;
     a->write_y = Y != nullptr ? 1 : 0;
     return SVDQ_OK;
