@@ -543,6 +543,10 @@ def run_gpu(args):
     per_config = None
     if world == 1 and args.all_configs:
         per_config = all_configs(P, S, dev, fp4_peak, peaks["hbm"], flush, flush_read)
+    if world == 1 and (args.all_configs or args.sweep_layers):
+        per_config = dict(per_config or {})
+        per_config.update(sweep(P, S, dev, fp4_peak, peaks["hbm"], flush, flush_read,
+                                n_layers=args.sweep_layers or None))
 
     line = None
     if rank == 0:
@@ -684,6 +688,91 @@ def all_configs(P, S, dev, fp4_peak, hbm_peak, flush, flush_read):
     return out
 
 
+SWEEP_CANDIDATES = ("1", "all", "video", "text")
+
+
+def sweep(P, S, dev, fp4_peak, hbm_peak, flush, flush_read, n_layers=None):
+    """The whole lambda scoring sweep: every layer (K 5120, N cycling 5120 x 4 /
+    15360 / 20480, 3 x 4096 rows) x every candidate {1, all, video, text}.
+
+    Per candidate: the calibration (one graph) and the candidate's pass -- the
+    activation quantiser and the linear with the per-modality rel-L2 scoring in its
+    epilogue, output not written (one graph) -- each timed from a cold L2 and summed
+    over the sweep.  The weight conversion of each candidate (randomized rank-32
+    factorisation with library QR/SVD, residual, weight quantisation) and the bf16
+    reference output of each layer (a cuBLAS GEMM, shared by the candidates) are
+    the sweep's preparation and are reported as wall times beside it.  The host
+    builds the next layers' inputs on worker threads while the device runs."""
+    import torch
+    from concurrent.futures import ThreadPoolExecutor
+
+    layers = S.CONFIGS[4]["layers"] if n_layers is None else n_layers
+    t_calib = t_pass = 0.0
+    flop = q_bytes = s_bytes = c_bytes = 0.0
+    conv_s = ref_s = 0.0
+    rel_sum = {c: None for c in SWEEP_CANDIDATES}
+    names = None
+    wall0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=3) as pool:
+        pending = [pool.submit(S.make_layer, 4, None, None, None, l) for l in range(min(3, layers))]
+        for l in range(layers):
+            L = pending.pop(0).result()
+            if l + 3 < layers:
+                pending.append(pool.submit(S.make_layer, 4, None, None, None, l + 3))
+            x, w, bias = _to_dev(L.x, dev), _to_dev(L.w, dev), _to_dev(L.bias, dev)
+            segs_mod = [(sg.begin, sg.end) for sg in L.segments]
+            names = [sg.name for sg in L.segments]
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            yref = torch.matmul(x.view(torch.bfloat16), w.view(torch.bfloat16).t()) + bias.view(torch.bfloat16)
+            torch.cuda.synchronize()
+            ref_s += time.perf_counter() - t0
+            wf = torch.empty(P.linear_score_workspace_bytes(len(segs_mod)), dtype=torch.uint8, device=dev)
+            for cand in SWEEP_CANDIDATES:
+                segs_cal = L.seg_ranges(L.calib_sets["all" if cand == "1" else cand])
+                w_cal = None if cand == "1" else w
+                t_calib += _graph_ms(lambda: P.svdq_calib_lambda(x, segs_cal, w_cal), flush, flush_read,
+                                     reps=3, warmup=3)
+                c_bytes += 2.0 * sum(e - b for b, e in segs_cal) * L.k + (2.0 * L.n * L.k if w_cal is not None
+                                                                          else 0.0)
+                cal = P.svdq_calib_lambda(x, segs_cal, w_cal)
+                torch.cuda.synchronize()
+                t0 = time.perf_counter()
+                lin = P.SVDQW4A4Linear.convert(w, bias, cal, L.rank)
+                torch.cuda.synchronize()
+                conv_s += time.perf_counter() - t0
+                q = P.svdq_quantize_act(x, cal["inv_lam"], lin.s_g_act, lin.down)
+
+                def candidate_pass():
+                    P.svdq_quantize_act(x, cal["inv_lam"], lin.s_g_act, lin.down, out=q)
+                    return P.svdq_linear_score(q["codes"], q["sf"], lin.s_g_act, q["d"], lin.w_codes, lin.w_sf,
+                                               lin.s_g_w, lin.up, lin.bias, yref=yref, segs=segs_mod, out=None,
+                                               write_out=False, workspace=wf)
+                t_pass += _graph_ms(candidate_pass, flush, flush_read, reps=3, warmup=3)
+                rel = candidate_pass()[3].cpu().numpy()
+                rel_sum[cand] = rel if rel_sum[cand] is None else rel_sum[cand] + rel
+                flop += 2.0 * L.m * L.n * L.k
+                q_bytes += (2 + 0.5 + 0.0625) * L.m * L.k + 4.0 * L.m * L.rank
+                s_bytes += 2.0 * L.m * L.n * 2          # what a separate scoring pass reads: Yq and Yref
+                del cal, lin, q
+            del x, w, bias, yref, wf, L
+            torch.cuda.empty_cache()
+    wall = time.perf_counter() - wall0
+    dev_ms = t_calib + t_pass
+    return {f"config4_sweep_{layers}_layers_x_{len(SWEEP_CANDIDATES)}_candidates": {
+        "layers": layers, "candidates": list(SWEEP_CANDIDATES),
+        "gemm_flop": flop, "quantize_bytes": q_bytes, "score_bytes_separate_pass": s_bytes,
+        "calib_bytes": c_bytes,
+        "device_ms": dev_ms, "calib_ms": t_calib, "quantize_linear_score_ms": t_pass,
+        "TFLOP/s_device": flop / (dev_ms * 1e-3) / 1e12,
+        "TFLOP/s_quantize_linear_score": flop / (t_pass * 1e-3) / 1e12,
+        "frac_fp4_quantize_linear_score": flop / (t_pass * 1e-3) / 1e12 / fp4_peak,
+        "calib_GB/s": c_bytes / (t_calib * 1e-3) / 1e9, "calib_frac_hbm": c_bytes / (t_calib * 1e-3) / 1e9 / hbm_peak,
+        "weight_conversion_wall_s": conv_s, "bf16_reference_wall_s": ref_s, "wall_s_incl_host_inputs": wall,
+        "mean_rel_l2_vs_bf16": {c: dict(zip(names, (rel_sum[c] / layers).tolist())) for c in SWEEP_CANDIDATES},
+        "timing": "each call one CUDA graph from a cold L2, median of 3 replays after 3, summed over the sweep"}}
+
+
 def lambda_search(P, S, dev, flush, flush_read):
     """The 39-candidate lambda search on one sweep layer (rank 32, three modalities):
     wall time of the whole search (host-driven; the randomized rank-32 factorisation of
@@ -786,7 +875,10 @@ def main():
     ap.add_argument("--profile-case", default=None, choices=PROFILE_CASES,
                     help="only launch one call five times on the --config workload (for ncu)")
     ap.add_argument("--all-configs", action="store_true",
-                    help="also time every call on every configured workload (adds a few minutes)")
+                    help="also time every call on every configured workload and the whole lambda "
+                         "scoring sweep (adds several minutes)")
+    ap.add_argument("--sweep-layers", type=int, default=0,
+                    help="also time the lambda scoring sweep over its first N layers")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "svdq":
         args.warmup = 3

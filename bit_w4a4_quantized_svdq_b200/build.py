@@ -1,8 +1,11 @@
-"""Build step for the CUDA library ``libsvdq.so`` (sm_100a, in-tree).
+"""Build step for the CUDA libraries (sm_100a, in-tree).
 
 ``python -m bit_w4a4_quantized_svdq_b200.build`` compiles every ``csrc/*.cu``
-with nvcc for ``sm_100a`` into ``bit_w4a4_quantized_svdq_b200/libsvdq.so``.
-nvcc cross-compiles, so this runs on machines without a GPU.
+with nvcc for ``sm_100a`` into ``bit_w4a4_quantized_svdq_b200/libsvdq.so``
+(release) and ``libsvdq_debug.so`` (the same source with SVDQ_DEBUG_CHECKS=1:
+pointer checks on the host, store bounds checks in the kernels).  The two are
+compiled concurrently.  nvcc cross-compiles, so this runs on machines without
+a GPU.
 """
 from __future__ import annotations
 
@@ -14,6 +17,8 @@ import sys
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_PATH = os.path.join(PKG_DIR, "libsvdq.so")
+DEBUG_LIB_PATH = os.path.join(PKG_DIR, "libsvdq_debug.so")
+VARIANT_FLAGS = {LIB_PATH: [], DEBUG_LIB_PATH: ["-DSVDQ_DEBUG_CHECKS=1"]}
 INCLUDE = os.path.join(os.path.dirname(PKG_DIR), "include")
 
 SOURCES = ["abi.cu", "calib.cu", "quantize.cu", "linear.cu", "score.cu", "residual.cu", "proxy.cu", "grid.cu", "mxfp8.cu"]
@@ -31,26 +36,34 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found: the sm_100a library cannot be built")
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB_PATH):
+def needs_build(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return True
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "svdq.h")]
     return any(os.path.getmtime(p) > t for p in deps if os.path.exists(p))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile the library if a source is newer than it (or ``force``); return its path."""
-    if not force and not needs_build():
-        return LIB_PATH
-    tmp = LIB_PATH + ".tmp"
-    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
-    os.replace(tmp, LIB_PATH)
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
+    """Compile the release library (and, with ``debug``, the debug one) where a
+    source is newer than it (or ``force``); return the release library's path."""
+    targets = [p for p in ([LIB_PATH, DEBUG_LIB_PATH] if debug else [LIB_PATH]) if force or needs_build(p)]
+    procs = []
+    for path in targets:
+        cmd = [nvcc_path(), *NVCC_FLAGS, *VARIANT_FLAGS[path], "-I", INCLUDE, "-o", path + ".tmp"] + \
+              [os.path.join(CSRC, s) for s in SOURCES]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        procs.append((path, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)))
+    failed = []
+    for path, proc in procs:
+        out, err = proc.communicate()
+        if proc.returncode != 0:
+            failed.append(f"{os.path.basename(path)}: nvcc failed ({proc.returncode}):\n{out}\n{err}")
+        else:
+            os.replace(path + ".tmp", path)
+    if failed:
+        raise RuntimeError("\n".join(failed))
     return LIB_PATH
 
 

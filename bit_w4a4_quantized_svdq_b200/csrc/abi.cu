@@ -4,6 +4,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace svdq {
 
@@ -30,6 +31,41 @@ EncodeTiledFn g_encode = nullptr;
 }  // namespace
 
 int current_device_index() { return current_device(); }
+
+// Armed extent limits + 1 per store site (0: none armed).
+std::atomic<int64_t> g_extent_limit[kSiteCount] = {};
+
+int64_t debug_extent(uint32_t site, int64_t extent) {
+#if SVDQ_DEBUG_CHECKS
+    if (site < kSiteCount) {
+        const int64_t lim = g_extent_limit[site].exchange(0, std::memory_order_acq_rel) - 1;
+        if (lim >= 0 && lim < extent) return lim;
+    }
+#else
+    (void)site;
+#endif
+    return extent;
+}
+
+bool debug_ptrs_ok(std::initializer_list<const void*> ptrs) {
+#if SVDQ_DEBUG_CHECKS
+    const int dev = current_device();
+    if (dev < 0) return false;
+    for (const void* p : ptrs) {
+        if (p == nullptr) continue;
+        cudaPointerAttributes at{};
+        if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return false;
+        }
+        const bool on_device = at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+        if (!on_device || at.device != dev) return false;
+    }
+#else
+    (void)ptrs;
+#endif
+    return true;
+}
 
 uint32_t* device_error_word() {
     const int dev = current_device();
@@ -122,6 +158,7 @@ const char* svdq_status_string(int status) {
         case SVDQ_ERR_TIMEOUT: return "device wait timed out";
         case SVDQ_ERR_NO_DEVICE: return "no sm_100 device";
         case SVDQ_ERR_SCRATCH_TOO_SMALL: return "problem exceeds the library's static scratch array";
+        case SVDQ_ERR_BOUNDS: return "a device store fell outside its output (debug library)";
         default: return "unknown status";
     }
 }
@@ -147,7 +184,22 @@ int svdq_device_error(void* stream, uint32_t* code) {
         if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return SVDQ_ERR_CUDA;
     }
     *code = v;
-    return v ? SVDQ_ERR_TIMEOUT : SVDQ_OK;
+    if (v == 0) return SVDQ_OK;
+    return v >= svdq::kErrBounds ? SVDQ_ERR_BOUNDS : SVDQ_ERR_TIMEOUT;
+}
+
+int svdq_debug_build(void) { return SVDQ_DEBUG_CHECKS ? 1 : 0; }
+
+int svdq_debug_limit_extent(int site, int64_t extent) {
+#if SVDQ_DEBUG_CHECKS
+    if (site < 1 || site >= static_cast<int>(svdq::kSiteCount) || extent < 0) return SVDQ_ERR_INVALID_ARG;
+    svdq::g_extent_limit[site].store(extent + 1, std::memory_order_release);
+    return SVDQ_OK;
+#else
+    (void)site;
+    (void)extent;
+    return SVDQ_ERR_UNSUPPORTED;
+#endif
 }
 
 }  // extern "C"

@@ -63,6 +63,7 @@ struct CalibArgs {
     float* inv_lambda;
     float* s_g;                               // holds max(strip maxima) until the last strip writes the scale
     uint32_t* err;
+    int64_t ext_amax, ext_lambda;             // store-check extents (debug library): K each
     // Time-out test (armed from the host, one call): CTA 0's producer leaves its
     // ring unit `skip_unit` unloaded, so a consumer's wait for it runs out after
     // `wait_limit` cycles; -1 = off.  Every other CTA and call runs normally.
@@ -71,10 +72,11 @@ struct CalibArgs {
 };
 
 __global__ void __launch_bounds__(256)
-calib_zero_kernel(float* ax, float* aw, int64_t K, float* lambda, float* s_g) {
+calib_zero_kernel(float* ax, float* aw, int64_t K, float* lambda, float* s_g, int64_t ext, uint32_t* err) {
     pdl_launch_dependents();                  // the reduction may start streaming at once
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < K; j += stride) {
+        if (!store_ok(j, 1, ext, err, kSiteCalibZero)) continue;
         ax[j] = 0.0f;
         if (aw) aw[j] = 0.0f;
         if (j % kStripCols == 0 || j == 1) lambda[j] = 0.0f;   // strip counters, strips-done counter
@@ -103,8 +105,10 @@ __device__ void strip_lambda(const CalibArgs& a, int64_t strip) {
         const float x = __ldcg(a.ax + j);
         const float lam = lambda_of(x, a.aw, j);
         const float il = __frcp_rn(lam);
-        if (j != 1) a.lambda[j] = lam;          // lambda[1] is the strips-done counter until the end
-        if (a.inv_lambda) a.inv_lambda[j] = il;
+        if (store_ok(j, 1, a.ext_lambda, a.err, kSiteCalibLambda)) {
+            if (j != 1) a.lambda[j] = lam;      // lambda[1] is the strips-done counter until the end
+            if (a.inv_lambda) a.inv_lambda[j] = il;
+        }
         v = __fmul_rn(x, il);
     }
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -248,13 +252,17 @@ calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) m = max(m, (red[w][src_lane][word] >> (16 * hi)) & 0xFFFFu);
             const int64_t col = strip * kStripCols + t;
-            if (m != 0 && col < a.K) atomicMax(a.out_bits[job] + col, m << 16);   // bf16 -> fp32 bits
+            if (m != 0 && col < a.K && store_ok(col, 1, a.ext_amax, a.err, kSiteCalibAmax))
+                atomicMax(a.out_bits[job] + col, m << 16);   // bf16 -> fp32 bits
         }
         __threadfence();
         consumers_sync();
         if (threadIdx.x == 0) {
-            const uint32_t prev = atomicAdd(reinterpret_cast<uint32_t*>(a.lambda + strip * kStripCols), 1u);
-            is_last = (static_cast<int64_t>(prev) == strip_merges(a, strip, G) - 1) ? 1u : 0u;
+            is_last = 0u;
+            if (store_ok(strip * kStripCols, 1, a.ext_lambda, a.err, kSiteCalibLambda)) {
+                const uint32_t prev = atomicAdd(reinterpret_cast<uint32_t*>(a.lambda + strip * kStripCols), 1u);
+                is_last = (static_cast<int64_t>(prev) == strip_merges(a, strip, G) - 1) ? 1u : 0u;
+            }
         }
         consumers_sync();
         if (is_last) {
@@ -328,6 +336,7 @@ int calib_launch(const void* X, int64_t M, int64_t K, int64_t ldx, const svdq_se
     int st = make_seg_table(segs, n_seg, M, &a.segs);
     if (st != SVDQ_OK) return st;
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    if (!debug_ptrs_ok({X, W, aw_in, amax_x, amax_w, lambda, inv_lambda, s_g})) return SVDQ_ERR_INVALID_ARG;
     uint32_t* err = device_error_word();
     if (err == nullptr) return SVDQ_ERR_CUDA;
     const int64_t sms = device_sm_count() > 0 ? device_sm_count() : 148;
@@ -353,6 +362,8 @@ int calib_launch(const void* X, int64_t M, int64_t K, int64_t ldx, const svdq_se
     a.inv_lambda = inv_lambda;
     a.s_g = s_g;
     a.err = err;
+    a.ext_amax = debug_extent(kSiteCalibAmax, K);
+    a.ext_lambda = debug_extent(kSiteCalibLambda, K);
     a.skip_unit = g_arm_skip.exchange(-1);       // armed by the time-out test for this one call
     a.wait_limit = a.skip_unit >= 0 ? g_arm_limit.load() : kWaitLimitCycles;
     if (a.strips >= (int64_t(1) << 24)) return SVDQ_ERR_UNSUPPORTED;
@@ -371,7 +382,7 @@ int calib_launch(const void* X, int64_t M, int64_t K, int64_t ldx, const svdq_se
     const int64_t zb = (K + 255) / 256;
     // the stored weight absmax is an input: only the outputs are zeroed
     calib_zero_kernel<<<static_cast<unsigned>(zb < sms ? zb : sms), 256, 0, cs>>>(
-        amax_x, W != nullptr ? amax_w : nullptr, K, lambda, s_g);
+        amax_x, W != nullptr ? amax_w : nullptr, K, lambda, s_g, debug_extent(kSiteCalibZero, K), err);
     st = launch_status(cudaGetLastError());
     if (st != SVDQ_OK) return st;
     const uint32_t smem = kSmemBytes + 1024;

@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cstddef>
 #include <cstdint>
+#include <initializer_list>
 
 #include "svdq.h"   // include/ is on the include path (see build.py)
 
@@ -65,6 +66,16 @@ bool encode_tmap_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t
 
 // Current device ordinal, or -1.
 int current_device_index();
+
+// Debug library only (SVDQ_DEBUG_CHECKS=1), identity otherwise: the extent a
+// kernel checks its stores of output `site` against -- `extent`, or the
+// smaller value a test armed with svdq_debug_limit_extent (consumed here).
+int64_t debug_extent(uint32_t site, int64_t extent);
+
+// Debug library only, true otherwise: every non-null pointer is device (or
+// managed) memory of the current device.  Entry points return
+// SVDQ_ERR_INVALID_ARG when it fails.
+bool debug_ptrs_ok(std::initializer_list<const void*> ptrs);
 
 // Raise a kernel's dynamic shared memory limit to `bytes`, once per device
 // (`done` is a per-kernel bit set over device ordinals 0..63).

@@ -24,7 +24,8 @@ constexpr int kGridThreads = 256;
 
 __global__ void __launch_bounds__(kGridThreads)
 lambda_grid_kernel(const float* __restrict__ ax, const float* __restrict__ aw, const float* __restrict__ alpha,
-                   int64_t K, float* __restrict__ lam, float* __restrict__ inv, float* __restrict__ s_g) {
+                   int64_t K, float* __restrict__ lam, float* __restrict__ inv, float* __restrict__ s_g,
+                   int64_t ext, int64_t ext_sg, uint32_t* err) {
     __shared__ float s_top[kGridThreads / 32];
     const int c = blockIdx.x;
     const double a = static_cast<double>(__ldg(alpha + c));
@@ -40,8 +41,10 @@ lambda_grid_kernel(const float* __restrict__ ax, const float* __restrict__ aw, c
             l = __double2float_rn(exp2(t));
         }
         const float il = __frcp_rn(l);
-        lam[static_cast<int64_t>(c) * K + j] = l;
-        inv[static_cast<int64_t>(c) * K + j] = il;
+        if (store_ok(static_cast<int64_t>(c) * K + j, 1, ext, err, kSiteGrid)) {
+            lam[static_cast<int64_t>(c) * K + j] = l;
+            inv[static_cast<int64_t>(c) * K + j] = il;
+        }
         top = fmaxf(top, __fmul_rn(x, il));
     }
 #pragma unroll
@@ -51,7 +54,7 @@ lambda_grid_kernel(const float* __restrict__ ax, const float* __restrict__ aw, c
     if (threadIdx.x == 0) {
         float m = 0.0f;
         for (int i = 0; i < kGridThreads / 32; ++i) m = fmaxf(m, s_top[i]);
-        s_g[c] = m > 0.0f ? __fdiv_rn(m, 2688.0f) : 1.0f;
+        if (store_ok(c, 1, ext_sg, err, kSiteGrid)) s_g[c] = m > 0.0f ? __fdiv_rn(m, 2688.0f) : 1.0f;
     }
 }
 
@@ -70,7 +73,10 @@ extern "C" int svdq_lambda_grid(const float* amax_x, const float* amax_w, int64_
                           reinterpret_cast<uintptr_t>(inv_lambda) | reinterpret_cast<uintptr_t>(s_g);
     if (any & 3u) return SVDQ_ERR_MISALIGNED;
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    if (!debug_ptrs_ok({amax_x, amax_w, alpha, lambda, inv_lambda, s_g})) return SVDQ_ERR_INVALID_ARG;
+    uint32_t* err = device_error_word();
+    if (err == nullptr) return SVDQ_ERR_CUDA;
     lambda_grid_kernel<<<static_cast<unsigned>(n_alpha), kGridThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        amax_x, amax_w, alpha, K, lambda, inv_lambda, s_g);
+        amax_x, amax_w, alpha, K, lambda, inv_lambda, s_g, debug_extent(kSiteGrid, K * n_alpha), n_alpha, err);
     return launch_status(cudaGetLastError());
 }

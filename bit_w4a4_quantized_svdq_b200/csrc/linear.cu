@@ -136,6 +136,9 @@ struct LinearArgs {
     double* den;
     double* rel;
     SegTable segs;
+    // Store-check extents (debug library): Y's columns and rows for TMA box
+    // origins, fp32 Y elements ((M - 1) ldy + N), workspace doubles, segments.
+    int64_t ext_box_x, ext_box_y, ext_y32, ext_part, ext_seg;
 };
 
 // Scoring of eight output elements against the reference: the fp32 8-term
@@ -716,9 +719,11 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     if (args.write_y) {
                         fence_async_shared();
                         __syncwarp();
-                        if (lane == 0 && grow0 < M32 && col0 + half * (kBN / 2) + h * 64 < args.N) {
+                        const int32_t bx = col0 + half * (kBN / 2) + h * 64;
+                        if (lane == 0 && grow0 < M32 && bx < args.N &&
+                            box_ok(bx, grow0, args.ext_box_x, args.ext_box_y, args.err, kSiteLinearBox)) {
                             // boxes wholly past row M or column N are skipped
-                            tma_store_2d(&tmap_y, part, col0 + half * (kBN / 2) + h * 64, grow0);
+                            tma_store_2d(&tmap_y, part, bx, grow0);
                             bulk_commit_group();
                         }
                     }
@@ -775,9 +780,10 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
             __syncwarp();
         }
         for (int sg = ew; sg < n_seg; sg += kEpiWarps) {
-            if (lane == 0) {
-                args.seg_part[(static_cast<int64_t>(blockIdx.x) * n_seg + sg) * 2] = segsum[sg].x;
-                args.seg_part[(static_cast<int64_t>(blockIdx.x) * n_seg + sg) * 2 + 1] = segsum[sg].y;
+            const int64_t off = (static_cast<int64_t>(blockIdx.x) * n_seg + sg) * 2;
+            if (lane == 0 && store_ok(off, 2, args.ext_part, args.err, kSiteLinearScore)) {
+                args.seg_part[off] = segsum[sg].x;
+                args.seg_part[off + 1] = segsum[sg].y;
             }
         }
     } else {
@@ -879,7 +885,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     dst[1] = make_uint4(pk[8 * j + 4], pk[8 * j + 5], pk[8 * j + 6], pk[8 * j + 7]);
                     fence_async_shared();
                     __syncwarp();
-                    if (lane == 0 && grow0 < args.M && ccol + 16 * j < args.N) {   // boxes wholly past M or N are skipped
+                    if (lane == 0 && grow0 < args.M && ccol + 16 * j < args.N &&   // boxes wholly past M or N are skipped
+                        box_ok(ccol + 16 * j, grow0, args.ext_box_x, args.ext_box_y, args.err, kSiteLinearBox)) {
                         // the output is not read again here: first out of L2, so it does
                         // not push out the operands other tiles still read
                         tma_store_2d_hint(&tmap_y, stg, static_cast<int32_t>(ccol) + 16 * j, grow0, pol_y);
@@ -894,9 +901,11 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     tmem_ld_32x32b_x32(tbase + c * 32, v);
                     tmem_ld_wait();
                     if (row_ok && ccol + c * 32 < args.N) {           // N % 128 == 0: chunks are whole
-                        float* dst = static_cast<float*>(args.Y) + row * args.ldy + ccol + c * 32;
+                        const int64_t off = row * args.ldy + ccol + c * 32;
+                        float* dst = static_cast<float*>(args.Y) + off;
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
+                            if (!store_ok(off + 4 * q, 4, args.ext_y32, args.err, kSiteLinearF32)) continue;
                             float y[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
@@ -944,7 +953,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                         num += __shfl_xor_sync(0xffffffffu, num, o);
                         den += __shfl_xor_sync(0xffffffffu, den, o);
                     }
-                    if (lane == 0) {
+                    if (lane == 0 && store_ok(sg, 1, args.ext_seg, args.err, kSiteLinearScore)) {
                         args.num[sg] = num;
                         args.den[sg] = den;
                         double rel;
@@ -1032,6 +1041,7 @@ int linear_prepare(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g
     if (r > 0 && (!aligned16(D) || !aligned16(up))) return SVDQ_ERR_MISALIGNED;
     if (bias && !aligned16(bias)) return SVDQ_ERR_MISALIGNED;
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    if (!debug_ptrs_ok({a_codes, a_sf, s_g_act, D, w_codes, w_sf, s_g_w, up, bias, Y})) return SVDQ_ERR_INVALID_ARG;
     uint32_t* err = device_error_word();
     if (err == nullptr) return SVDQ_ERR_CUDA;
 
@@ -1088,6 +1098,9 @@ int linear_prepare(const uint8_t* a_codes, const uint8_t* a_sf, const float* s_g
     }
     a->err = err;
     a->write_y = Y != nullptr ? 1 : 0;
+    a->ext_box_x = debug_extent(kSiteLinearBox, N);
+    a->ext_box_y = M;
+    a->ext_y32 = debug_extent(kSiteLinearF32, (M - 1) * ldy + N);
     return SVDQ_OK;
 }
 
@@ -1161,10 +1174,13 @@ extern "C" int svdq_linear_score(const uint8_t* a_codes, const uint8_t* a_sf, co
     if (!encode_tmap_2d(&tr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Yref, N, M, ldr * 2, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B))
         return SVDQ_ERR_CUDA;
+    if (!debug_ptrs_ok({Yref, num, den, rel, workspace})) return SVDQ_ERR_INVALID_ARG;
     a.seg_part = static_cast<double*>(workspace);
     a.num = num;
     a.den = den;
     a.rel = rel;
+    a.ext_part = debug_extent(kSiteLinearScore, static_cast<int64_t>(workspace_bytes / sizeof(double)));
+    a.ext_seg = n_seg;
     return launch_linear<false, true>(ta, tb, ty, tr, tsa, tsb, a, static_cast<cudaStream_t>(stream),
                                       workspace_bytes);
 }

@@ -40,7 +40,8 @@ __device__ __forceinline__ int64_t mx_sf_offset(int64_t row, int64_t blk, int64_
 
 __global__ void __launch_bounds__(kMxThreads)
 mx_quantize_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int64_t ldx, uint32_t n_units,
-                   uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+                   uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, int64_t ext_codes, int64_t ext_sf,
+                   uint32_t* err) {
     const int lane = threadIdx.x & 31;
     const uint32_t segs_per_row = static_cast<uint32_t>((K + 255) / 256);
     const uint32_t warps = gridDim.x * (kMxThreads / 32);
@@ -93,7 +94,7 @@ mx_quantize_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int64_t
                 unpack_f32x2(mul_f32x2(bf16x2_to_f32x2(w[2 * j + 1]), inv2), p2, p3);
                 q[j] = cvt_e4m3x2(p0, p1) | (cvt_e4m3x2(p2, p3) << 16);
             }
-            if (row < M && col < K)
+            if (row < M && col < K && store_ok(row * K + col, 8, ext_codes, err, kSiteMxCodes))
                 *reinterpret_cast<uint2*>(codes + row * K + col) = make_uint2(q[0], q[1]);
             // scale bytes of blocks 4g .. 4g + 3 of this segment: lanes 16 g, 16 g + 4, + 8, + 12
             const uint32_t sb = static_cast<uint32_t>(e + 127);
@@ -101,9 +102,9 @@ mx_quantize_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int64_t
             const uint32_t s2 = __shfl_down_sync(0xffffffffu, sb, 8);
             const uint32_t s3 = __shfl_down_sync(0xffffffffu, sb, 12);
             if ((lane & 15) == 0 && col < K) {
-                const int64_t blk = col / 32;
-                *reinterpret_cast<uint32_t*>(sf + mx_sf_offset(row, blk, blocks_per_row)) =
-                    sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+                const int64_t off = mx_sf_offset(row, col / 32, blocks_per_row);
+                if (store_ok(off, 4, ext_sf, err, kSiteMxSf))
+                    *reinterpret_cast<uint32_t*>(sf + off) = sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
             }
         }
     }
@@ -127,6 +128,9 @@ extern "C" int svdq_quantize_mxfp8(const void* X, int64_t M, int64_t K, int64_t 
     if (!aligned16(X) || (ldx * 2) % 16 != 0 || !aligned16(codes) || (reinterpret_cast<uintptr_t>(sf) & 3u))
         return SVDQ_ERR_MISALIGNED;
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    if (!debug_ptrs_ok({X, codes, sf})) return SVDQ_ERR_INVALID_ARG;
+    uint32_t* err = device_error_word();
+    if (err == nullptr) return SVDQ_ERR_CUDA;
     const int64_t rows_pad = (M + 127) / 128 * 128;
     const int64_t units = rows_pad * ((K + 255) / 256);            // 256-element row segments
     if (units > 0x7FFFFFFFLL) return SVDQ_ERR_UNSUPPORTED;
@@ -134,6 +138,8 @@ extern "C" int svdq_quantize_mxfp8(const void* X, int64_t M, int64_t K, int64_t 
     const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
     const int64_t blocks = std::min<int64_t>((warps_needed + 7) / 8, static_cast<int64_t>(sms) * 8);
     mx_quantize_kernel<<<static_cast<unsigned>(blocks), kMxThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint16_t*>(X), M, K, ldx, static_cast<uint32_t>(units), codes, sf);
+        static_cast<const uint16_t*>(X), M, K, ldx, static_cast<uint32_t>(units), codes, sf,
+        debug_extent(kSiteMxCodes, M * K), debug_extent(kSiteMxSf, static_cast<int64_t>(svdq_mxfp8_sf_bytes(M, K))),
+        err);
     return launch_status(cudaGetLastError());
 }

@@ -29,7 +29,7 @@ constexpr int kGroup = 16;
 
 __global__ void __launch_bounds__(kProxyThreads)
 bits_lost_kernel(const float* __restrict__ ax, int64_t ld_ax, const float* __restrict__ inv_lam, int64_t ld_lam,
-                 int64_t K, int n_mod, double* __restrict__ bits) {
+                 int64_t K, int n_mod, double* __restrict__ bits, int64_t ext, uint32_t* err) {
     __shared__ double s_sum[kProxyThreads / 32];
     __shared__ unsigned long long s_cnt[kProxyThreads / 32];
     const int mod = blockIdx.x;
@@ -73,7 +73,8 @@ bits_lost_kernel(const float* __restrict__ ax, int64_t ld_ax, const float* __res
             total += s_sum[w];
             n += s_cnt[w];
         }
-        bits[static_cast<int64_t>(cand) * n_mod + mod] = n > 0 ? total / static_cast<double>(n) : 0.0;
+        const int64_t off = static_cast<int64_t>(cand) * n_mod + mod;
+        if (store_ok(off, 1, ext, err, kSiteBits)) bits[off] = n > 0 ? total / static_cast<double>(n) : 0.0;
     }
 }
 
@@ -91,7 +92,11 @@ extern "C" int svdq_bits_lost(const float* amax_x, int64_t ld_amax, int n_mod, c
         (reinterpret_cast<uintptr_t>(bits) & 7u))
         return SVDQ_ERR_MISALIGNED;
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    if (!debug_ptrs_ok({amax_x, inv_lambda, bits})) return SVDQ_ERR_INVALID_ARG;
+    uint32_t* err = device_error_word();
+    if (err == nullptr) return SVDQ_ERR_CUDA;
     bits_lost_kernel<<<dim3(static_cast<unsigned>(n_mod), static_cast<unsigned>(n_cand)), kProxyThreads, 0,
-                       static_cast<cudaStream_t>(stream)>>>(amax_x, ld_amax, inv_lambda, ld_lam, K, n_mod, bits);
+                       static_cast<cudaStream_t>(stream)>>>(amax_x, ld_amax, inv_lambda, ld_lam, K, n_mod, bits,
+                                                       debug_extent(kSiteBits, int64_t(n_mod) * n_cand), err);
     return launch_status(cudaGetLastError());
 }

@@ -86,6 +86,7 @@ struct QuantArgs {
     float* D;
     uint32_t* sat_count;
     uint32_t* err;
+    int64_t ext_codes, ext_sf, ext_d;   // store-check extents (debug library): M K / 2 bytes, the scale bytes, M R floats
     int n_chunks;      // K / 64
     int split;         // CTAs along K (cluster size when R > 0)
     int rows;          // rows per group (the TMA box height), <= 128
@@ -317,19 +318,19 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             const uint32_t x23 = __byte_perm(n2, n3, 0x5140);    // c0 d0 c1 d1
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);        // shared memory of this stage no longer read
-            uint8_t* cbase = args.codes + chunk * (kBK / 2) + b * 8;
-            if (code0) *reinterpret_cast<uint2*>(cbase + grow0 * half_k) = ca;
-            if (code1) *reinterpret_cast<uint2*>(cbase + grow1 * half_k) = cb;
+            const int64_t coff = chunk * (kBK / 2) + b * 8;
+            if (code0 && store_ok(coff + grow0 * half_k, 8, args.ext_codes, args.err, kSiteQuantCodes))
+                *reinterpret_cast<uint2*>(args.codes + coff + grow0 * half_k) = ca;
+            if (code1 && store_ok(coff + grow1 * half_k, 8, args.ext_codes, args.err, kSiteQuantCodes))
+                *reinterpret_cast<uint2*>(args.codes + coff + grow1 * half_k) = cb;
             if (b == 0) {
                 // a row's word in its 128-row block's 512-byte atom of this chunk
-                if (box0)
-                    *reinterpret_cast<uint32_t*>(args.sf + ((grow0 >> 7) * atoms_k + chunk) * 512 +
-                                                 (grow0 & 31) * 16 + ((grow0 >> 5) & 3) * 4) =
-                        __byte_perm(x01, x23, 0x5410);
-                if (box1)
-                    *reinterpret_cast<uint32_t*>(args.sf + ((grow1 >> 7) * atoms_k + chunk) * 512 +
-                                                 (grow1 & 31) * 16 + ((grow1 >> 5) & 3) * 4) =
-                        __byte_perm(x01, x23, 0x7632);
+                const int64_t o0 = ((grow0 >> 7) * atoms_k + chunk) * 512 + (grow0 & 31) * 16 + ((grow0 >> 5) & 3) * 4;
+                const int64_t o1 = ((grow1 >> 7) * atoms_k + chunk) * 512 + (grow1 & 31) * 16 + ((grow1 >> 5) & 3) * 4;
+                if (box0 && store_ok(o0, 4, args.ext_sf, args.err, kSiteQuantSf))
+                    *reinterpret_cast<uint32_t*>(args.sf + o0) = __byte_perm(x01, x23, 0x5410);
+                if (box1 && store_ok(o1, 4, args.ext_sf, args.err, kSiteQuantSf))
+                    *reinterpret_cast<uint32_t*>(args.sf + o1) = __byte_perm(x01, x23, 0x7632);
             }
         }
         // Padding rows of the scale array past the last group's box (the box ends
@@ -340,8 +341,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             for (int64_t t = threadIdx.x; t < n_pad; t += kQuantWarps * 32) {
                 const int64_t row = pad0 + t / n_local;
                 const int64_t chunk = c_begin + t % n_local;
-                *reinterpret_cast<uint32_t*>(args.sf + ((row >> 7) * atoms_k + chunk) * 512 + (row & 31) * 16 +
-                                             ((row >> 5) & 3) * 4) = 0u;
+                const int64_t off = ((row >> 7) * atoms_k + chunk) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
+                if (store_ok(off, 4, args.ext_sf, args.err, kSiteQuantSf))
+                    *reinterpret_cast<uint32_t*>(args.sf + off) = 0u;
             }
         }
         // saturation count: one atomic per warp
@@ -402,7 +404,8 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                     const float4* src = reinterpret_cast<const float4*>(smem + L::kPartOff) + row * (L::kPartStride / 4);
                     float4* dst = reinterpret_cast<float4*>(args.D + grow * R);
 #pragma unroll
-                    for (int q = 0; q < kNq; ++q) dst[q] = src[q];
+                    for (int q = 0; q < kNq; ++q)
+                        if (store_ok(grow * R + 4 * q, 4, args.ext_d, args.err, kSiteQuantD)) dst[q] = src[q];
                 }
             } else {
                 // two groups at a time: at most 8 remote 16-byte loads in flight per thread
@@ -427,7 +430,8 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                                         acc.z += got[t][c].z; acc.w += got[t][c].w;
                                     }
                                 }
-                                dst[q0 + t0 + t] = acc;
+                                if (store_ok(grow * R + 4 * (q0 + t0 + t), 4, args.ext_d, args.err, kSiteQuantD))
+                                    dst[q0 + t0 + t] = acc;
                             }
                         }
                     }
@@ -542,6 +546,7 @@ extern "C" int svdq_quantize_act(const void* X, int64_t M, int64_t K, int64_t ld
     if (r > 0 && (!aligned16(down) || !aligned16(D))) return SVDQ_ERR_MISALIGNED;
     if (sat_count && (reinterpret_cast<uintptr_t>(sat_count) & 3u)) return SVDQ_ERR_MISALIGNED;
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    if (!debug_ptrs_ok({X, inv_lambda, s_g, down, codes, sf, D, sat_count})) return SVDQ_ERR_INVALID_ARG;
     uint32_t* err = device_error_word();
     if (err == nullptr) return SVDQ_ERR_CUDA;
     QuantArgs a{};
@@ -554,6 +559,9 @@ extern "C" int svdq_quantize_act(const void* X, int64_t M, int64_t K, int64_t ld
     a.D = D;
     a.sat_count = sat_count;
     a.err = err;
+    a.ext_codes = debug_extent(kSiteQuantCodes, M * (K / 2));
+    a.ext_sf = debug_extent(kSiteQuantSf, static_cast<int64_t>(svdq_sf_bytes(M, K)));
+    a.ext_d = debug_extent(kSiteQuantD, M * r);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // Rows of the last 128-row block beyond M hold zero scale bytes: the kernel
     // writes every row of every tile (zero-filled by TMA), so no memset is needed.

@@ -21,7 +21,8 @@ constexpr int kTileK = 256;     // one thread per k, one block row of up values 
 __global__ void __launch_bounds__(kTileK)
 residual_kernel(const uint16_t* __restrict__ W, int64_t N, int64_t K, int64_t ldw,
                 const float* __restrict__ lambda, const uint16_t* __restrict__ down,
-                const uint16_t* __restrict__ up, int r, uint16_t* __restrict__ R, int rows_per_block) {
+                const uint16_t* __restrict__ up, int r, uint16_t* __restrict__ R, int rows_per_block,
+                int64_t ext, uint32_t* err) {
     __shared__ double up_s[kMaxRank];
     const int64_t k = static_cast<int64_t>(blockIdx.x) * kTileK + threadIdx.x;
     const int64_t n0 = static_cast<int64_t>(blockIdx.y) * rows_per_block;
@@ -47,7 +48,8 @@ residual_kernel(const uint16_t* __restrict__ W, int64_t N, int64_t K, int64_t ld
             const double w = static_cast<double>(__uint_as_float(static_cast<uint32_t>(W[n * ldw + k]) << 16));
             const double v = __dsub_rn(__dmul_rn(w, lam), __dmul_rn(lam, acc));
             const float f = __double2float_rn(v);
-            R[n * K + k] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+            if (store_ok(n * K + k, 1, ext, err, kSiteResidual))
+                R[n * K + k] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
         }
     }
 }
@@ -62,12 +64,16 @@ extern "C" int svdq_residual(const void* W, int64_t N, int64_t K, int64_t ldw, c
     if (r < 0 || r > kMaxRank) return SVDQ_ERR_UNSUPPORTED;
     if (r > 0 && (down == nullptr || up == nullptr)) return SVDQ_ERR_INVALID_ARG;
     if (!device_is_sm100()) return SVDQ_ERR_NO_DEVICE;
+    if (!debug_ptrs_ok({W, lambda, down, up, R})) return SVDQ_ERR_INVALID_ARG;
+    uint32_t* err = device_error_word();
+    if (err == nullptr) return SVDQ_ERR_CUDA;
     const int rows_per_block = 16;
     const int64_t gy = (N + rows_per_block - 1) / rows_per_block;
     if (gy > 65535) return SVDQ_ERR_UNSUPPORTED;
     dim3 grid(static_cast<unsigned>((K + kTileK - 1) / kTileK), static_cast<unsigned>(gy));
     residual_kernel<<<grid, kTileK, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint16_t*>(W), N, K, ldw, lambda, static_cast<const uint16_t*>(down),
-        static_cast<const uint16_t*>(up), r, static_cast<uint16_t*>(R), rows_per_block);
+        static_cast<const uint16_t*>(up), r, static_cast<uint16_t*>(R), rows_per_block,
+        debug_extent(kSiteResidual, N * K), err);
     return launch_status(cudaGetLastError());
 }

@@ -78,7 +78,7 @@ __device__ __forceinline__ void accum8(const uint4& qa, const uint4& qb, double&
 
 __global__ void __launch_bounds__(kThreads)
 score_partial_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict__ yr, int64_t N, int64_t ld,
-                     ChunkPlan plan, double* __restrict__ partial) {
+                     ChunkPlan plan, double* __restrict__ partial, int64_t ext_part, uint32_t* err) {
     __shared__ double sh[kThreads / 32];
     const int64_t chunk = blockIdx.x;
     int s = 0;
@@ -116,7 +116,7 @@ score_partial_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict
     }
     num = block_sum(num, sh);
     den = block_sum(den, sh);
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && store_ok(2 * chunk, 2, ext_part, err, kSiteScorePart)) {
         partial[2 * chunk] = num;
         partial[2 * chunk + 1] = den;
     }
@@ -124,7 +124,7 @@ score_partial_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict
 
 __global__ void __launch_bounds__(kThreads)
 score_finalize_kernel(ChunkPlan plan, const double* __restrict__ partial, double* __restrict__ num_out,
-                      double* __restrict__ den_out, double* __restrict__ rel_out) {
+                      double* __restrict__ den_out, double* __restrict__ rel_out, int64_t ext_out, uint32_t* err) {
     __shared__ double sh[kThreads / 32];
     const int s = blockIdx.x;
     double num = 0.0, den = 0.0;
@@ -134,7 +134,7 @@ score_finalize_kernel(ChunkPlan plan, const double* __restrict__ partial, double
     }
     num = block_sum(num, sh);
     den = block_sum(den, sh);
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && store_ok(s, 1, ext_out, err, kSiteScoreOut)) {
         num_out[s] = num;
         den_out[s] = den;
         double rel;
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict__ yr, int64_t N,
                     const __grid_constant__ ChunkPlan plan, int64_t n_chunks, double* __restrict__ partial,
                     double* __restrict__ num_out, double* __restrict__ den_out, double* __restrict__ rel_out,
-                    uint32_t* err) {
+                    uint32_t* err, int64_t ext_part, int64_t ext_out) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStreamSlots * 2 * kChunkBytes);
     uint64_t* empty = full + kStreamSlots;
@@ -256,7 +256,7 @@ score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict_
             for (int v = 0; v < kVecPerThread; ++v) accum8(va[v], vb[v], num, den);
             num = consumer_sum(num, sh);
             den = consumer_sum(den, sh);
-            if (threadIdx.x == 0) {
+            if (threadIdx.x == 0 && store_ok(2 * c, 2, ext_part, err, kSiteScorePart)) {
                 partial[2 * c] = num;
                 partial[2 * c + 1] = den;
             }
@@ -276,7 +276,7 @@ score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict_
             }
             num = consumer_sum(num, sh);
             den = consumer_sum(den, sh);
-            if (threadIdx.x == 0) {
+            if (threadIdx.x == 0 && store_ok(s, 1, ext_out, err, kSiteScoreOut)) {
                 num_out[s] = num;
                 den_out[s] = den;
                 double rel;
@@ -300,11 +300,14 @@ int score_lambda_launch(const void* Yq, const void* Yref, int64_t M, int64_t N, 
     const int64_t chunks = plan.chunk_prefix[n_seg];
     if (partial_bytes < static_cast<size_t>(chunks) * 2 * sizeof(double)) return SVDQ_ERR_INVALID_ARG;
     if (chunks > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
+    if (!debug_ptrs_ok({Yq, Yref, num, den, rel, partial})) return SVDQ_ERR_INVALID_ARG;
+    uint32_t* err = device_error_word();
+    if (err == nullptr) return SVDQ_ERR_CUDA;
+    const int64_t ext_part = debug_extent(kSiteScorePart, static_cast<int64_t>(partial_bytes / sizeof(double)));
+    const int64_t ext_out = debug_extent(kSiteScoreOut, n_seg);
     if (ld == N && N % 8 == 0) {
         static std::atomic<uint64_t> smem_set{0};
         if (!set_dynamic_smem_once(score_stream_kernel, kStreamSmem, smem_set)) return SVDQ_ERR_CUDA;
-        uint32_t* err = device_error_word();
-        if (err == nullptr) return SVDQ_ERR_CUDA;
         // cooperative: never more CTAs than can be resident together
         const int64_t resident = coresident_grid(score_stream_kernel, kStreamThreads, kStreamSmem);
         if (resident < 1) return SVDQ_ERR_CUDA;
@@ -323,13 +326,13 @@ int score_lambda_launch(const void* Yq, const void* Yref, int64_t M, int64_t N, 
         cfg.numAttrs = 1;
         return launch_status(cudaLaunchKernelEx(&cfg, score_stream_kernel, static_cast<const uint16_t*>(Yq),
                                                 static_cast<const uint16_t*>(Yref), N, plan, chunks, partial, num,
-                                                den, rel, err));
+                                                den, rel, err, ext_part, ext_out));
     } else {
         score_partial_kernel<<<static_cast<unsigned>(chunks), kThreads, 0, cs>>>(
-            static_cast<const uint16_t*>(Yq), static_cast<const uint16_t*>(Yref), N, ld, plan, partial);
+            static_cast<const uint16_t*>(Yq), static_cast<const uint16_t*>(Yref), N, ld, plan, partial, ext_part, err);
     }
     if (cudaGetLastError() != cudaSuccess) return SVDQ_ERR_CUDA;
-    score_finalize_kernel<<<n_seg, kThreads, 0, cs>>>(plan, partial, num, den, rel);
+    score_finalize_kernel<<<n_seg, kThreads, 0, cs>>>(plan, partial, num, den, rel, ext_out, err);
     return launch_status(cudaGetLastError());
 }
 

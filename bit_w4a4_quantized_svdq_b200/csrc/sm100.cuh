@@ -27,6 +27,68 @@ enum DevErr : uint32_t {
 // legitimate wait, short enough to return control on a lost arrival.
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
+// ---------------------------------------------------------------------------
+// Store checks of the debug library (compiled with SVDQ_DEBUG_CHECKS=1)
+// ---------------------------------------------------------------------------
+// Every plain global store of an output goes through store_ok(), and every TMA
+// store's box origin through box_ok().  The extent is the output's documented
+// size, computed on the host apart from the kernel's index arithmetic.  In the
+// debug library a store outside it is skipped and kErrBounds + site goes into
+// the error word (the first error wins), so the kernel runs on and the host
+// reads SVDQ_ERR_BOUNDS.  In the release library both return true and compile
+// away.
+#ifndef SVDQ_DEBUG_CHECKS
+#define SVDQ_DEBUG_CHECKS 0
+#endif
+constexpr uint32_t kErrBounds = 0x100u;
+enum StoreSite : uint32_t {
+    kSiteCalibZero = 1,       // calibration: zeroing of absmax, counters, scale
+    kSiteCalibAmax = 2,       // calibration: per-channel absmax merge
+    kSiteCalibLambda = 3,     // calibration: lambda, 1/lambda, strip counters, scale
+    kSiteQuantCodes = 4,      // NVFP4 quantiser: packed codes
+    kSiteQuantSf = 5,         // NVFP4 quantiser: swizzled scale bytes
+    kSiteQuantD = 6,          // NVFP4 quantiser: low-rank down-projection D
+    kSiteLinearBox = 7,       // linear: TMA store box origin of Y
+    kSiteLinearF32 = 8,       // linear: fp32 output
+    kSiteLinearScore = 9,     // fused scoring: per-CTA partials and the result
+    kSiteScorePart = 10,      // scoring: per-CTA partial sums
+    kSiteScoreOut = 11,       // scoring: num, den, rel
+    kSiteResidual = 12,       // residual weight
+    kSiteGrid = 13,           // lambda grid: lambda, 1/lambda, scale
+    kSiteBits = 14,           // bits lost
+    kSiteMxCodes = 15,        // MXFP8 quantiser: codes
+    kSiteMxSf = 16,           // MXFP8 quantiser: scale bytes
+    kSiteCount = 17
+};
+
+// A store of `width` elements at element offset `off` into an output of
+// `extent` elements.
+__device__ __forceinline__ bool store_ok(int64_t off, int64_t width, int64_t extent, uint32_t* err,
+                                         uint32_t site) {
+#if SVDQ_DEBUG_CHECKS
+    if (off >= 0 && off + width <= extent) return true;
+    atomicCAS(err, 0u, kErrBounds + site);
+    return false;
+#else
+    (void)off; (void)width; (void)extent; (void)err; (void)site;
+    return true;
+#endif
+}
+
+// A TMA store box starting at (x, y) of a tensor of dims {dx, dy}: the origin
+// must lie inside (the copy clips the far edges; a negative origin is not allowed).
+__device__ __forceinline__ bool box_ok(int64_t x, int64_t y, int64_t dx, int64_t dy, uint32_t* err,
+                                       uint32_t site) {
+#if SVDQ_DEBUG_CHECKS
+    if (x >= 0 && y >= 0 && x < dx && y < dy) return true;
+    atomicCAS(err, 0u, kErrBounds + site);
+    return false;
+#else
+    (void)x; (void)y; (void)dx; (void)dy; (void)err; (void)site;
+    return true;
+#endif
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -99,11 +99,11 @@ def svdq_calib_lambda(x: torch.Tensor, segs: Segs = None, w: Optional[torch.Tens
     m, k = x.shape
     ldx = _row_stride(x, "x")
     dev = x.device
-    ax = torch.empty(k, dtype=torch.float32, device=dev)
-    aw = torch.empty(k, dtype=torch.float32, device=dev) if w is not None else None
-    lam = torch.empty(k, dtype=torch.float32, device=dev)
-    inv = torch.empty(k, dtype=torch.float32, device=dev)
-    s_g = torch.empty(1, dtype=torch.float32, device=dev)
+    ax = _lib.out_empty(k, torch.float32, dev)
+    aw = _lib.out_empty(k, torch.float32, dev) if w is not None else None
+    lam = _lib.out_empty(k, torch.float32, dev)
+    inv = _lib.out_empty(k, torch.float32, dev)
+    s_g = _lib.out_empty(1, torch.float32, dev)
     if w is not None:
         _check_bf16(w, "w")
         n, ldw = w.shape[0], _row_stride(w, "w")
@@ -126,10 +126,10 @@ def svdq_calib_lambda_stored_w(x: torch.Tensor, segs: Segs, amax_w: torch.Tensor
     if amax_w.dtype != torch.float32 or amax_w.numel() != k or not amax_w.is_contiguous():
         raise ValueError("amax_w must be a contiguous float32 tensor of K values")
     dev = x.device
-    ax = torch.empty(k, dtype=torch.float32, device=dev)
-    lam = torch.empty(k, dtype=torch.float32, device=dev)
-    inv = torch.empty(k, dtype=torch.float32, device=dev)
-    s_g = torch.empty(1, dtype=torch.float32, device=dev)
+    ax = _lib.out_empty(k, torch.float32, dev)
+    lam = _lib.out_empty(k, torch.float32, dev)
+    inv = _lib.out_empty(k, torch.float32, dev)
+    s_g = _lib.out_empty(1, torch.float32, dev)
     arr, n_seg = _lib.seg_array(segs)
     _lib.check("svdq_calib_lambda_stored_w", lib.svdq_calib_lambda_stored_w(
         _ptr(x), m, k, ldx, arr, n_seg, _ptr(amax_w), _ptr(ax), _ptr(lam), _ptr(inv), _ptr(s_g), _stream(stream)))
@@ -148,9 +148,9 @@ def svdq_quantize_act(x: torch.Tensor, inv_lambda: Optional[torch.Tensor], s_g: 
     r = 0 if down is None else int(down.shape[0])
     dev = x.device
     if out is None:
-        out = dict(codes=torch.empty((m, k // 2), dtype=torch.uint8, device=dev),
-                   sf=torch.empty(sf_bytes(m, k), dtype=torch.uint8, device=dev),
-                   d=torch.empty((m, r), dtype=torch.float32, device=dev) if r else None)
+        out = dict(codes=_lib.out_empty((m, k // 2), torch.uint8, dev),
+                   sf=_lib.out_empty(sf_bytes(m, k), torch.uint8, dev),
+                   d=_lib.out_empty((m, r), torch.float32, dev) if r else None)
     _lib.check("svdq_quantize_act", lib.svdq_quantize_act(
         _ptr(x), m, k, ldx, _ptr(inv_lambda), _ptr(s_g), _ptr(down), r,
         _ptr(out["codes"]), _ptr(out["sf"]), _ptr(out["d"]), _ptr(sat_count), _stream(stream)))
@@ -169,7 +169,7 @@ def svdq_linear(a_codes: torch.Tensor, a_sf: torch.Tensor, s_g_act: torch.Tensor
     k = 2 * kh
     r = 0 if d is None else int(d.shape[1])
     if out is None:
-        out = torch.empty((m, n), dtype=out_dtype, device=a_codes.device)
+        out = _lib.out_empty((m, n), out_dtype, a_codes.device)
     ldy = _row_stride(out, "out")
     code = {torch.bfloat16: 0, torch.float32: 1}[out.dtype]
     _lib.check("svdq_linear", lib.svdq_linear(
@@ -200,16 +200,16 @@ def svdq_linear_score(a_codes: torch.Tensor, a_sf: torch.Tensor, s_g_act: torch.
         raise ValueError(f"yref must be [{m}, {n}], got {tuple(yref.shape)}")
     dev = a_codes.device
     if write_out and out is None:
-        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        out = _lib.out_empty((m, n), torch.bfloat16, dev)
     if not write_out:
         out = None
     ldy = _row_stride(out, "out") if out is not None else n
     arr, n_seg = _lib.seg_array(segs)
-    num = torch.empty(n_seg, dtype=torch.float64, device=dev)
-    den = torch.empty(n_seg, dtype=torch.float64, device=dev)
-    rel = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    num = _lib.out_empty(n_seg, torch.float64, dev)
+    den = _lib.out_empty(n_seg, torch.float64, dev)
+    rel = _lib.out_empty(n_seg, torch.float64, dev)
     if workspace is None:
-        workspace = torch.empty(linear_score_workspace_bytes(n_seg), dtype=torch.uint8, device=dev)
+        workspace = _lib.out_empty(linear_score_workspace_bytes(n_seg), torch.uint8, dev)
     _lib.check("svdq_linear_score", lib.svdq_linear_score(
         _ptr(a_codes), _ptr(a_sf), _ptr(s_g_act), _ptr(d), r, _ptr(w_codes), _ptr(w_sf), _ptr(s_g_w),
         _ptr(up), _ptr(bias), _ptr(out), ldy, _ptr(yref), _row_stride(yref, "yref"), arr, n_seg,
@@ -236,12 +236,12 @@ def svdq_score_lambda(yq: torch.Tensor, yref: torch.Tensor, segs: Sequence[Tuple
         raise ValueError("yq and yref must share a row stride")
     arr, n_seg = _lib.seg_array(segs)
     dev = yq.device
-    num = torch.empty(n_seg, dtype=torch.float64, device=dev)
-    den = torch.empty(n_seg, dtype=torch.float64, device=dev)
-    rel = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    num = _lib.out_empty(n_seg, torch.float64, dev)
+    den = _lib.out_empty(n_seg, torch.float64, dev)
+    rel = _lib.out_empty(n_seg, torch.float64, dev)
     need = score_workspace_bytes(segs, n)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        workspace = _lib.out_empty(need, torch.uint8, dev)
     _lib.check("svdq_score_lambda", lib.svdq_score_lambda(
         _ptr(yq), _ptr(yref), m, n, ld, arr, n_seg, _ptr(num), _ptr(den), _ptr(rel),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
@@ -260,9 +260,9 @@ def svdq_score_lambda_static(yq: torch.Tensor, yref: torch.Tensor, segs: Sequenc
         raise ValueError("yq and yref must share a row stride")
     arr, n_seg = _lib.seg_array(segs)
     dev = yq.device
-    num = torch.empty(n_seg, dtype=torch.float64, device=dev)
-    den = torch.empty(n_seg, dtype=torch.float64, device=dev)
-    rel = torch.empty(n_seg, dtype=torch.float64, device=dev)
+    num = _lib.out_empty(n_seg, torch.float64, dev)
+    den = _lib.out_empty(n_seg, torch.float64, dev)
+    rel = _lib.out_empty(n_seg, torch.float64, dev)
     _lib.check("svdq_score_lambda_static", lib.svdq_score_lambda_static(
         _ptr(yq), _ptr(yref), m, n, ld, arr, n_seg, _ptr(num), _ptr(den), _ptr(rel), _stream(stream)))
     return num, den, rel
@@ -276,7 +276,7 @@ def svdq_residual(w: torch.Tensor, lam: Optional[torch.Tensor], down: Optional[t
     _check_bf16(w, "w")
     n, k = w.shape
     r = 0 if down is None else int(down.shape[0])
-    out = torch.empty((n, k), dtype=torch.bfloat16, device=w.device)
+    out = _lib.out_empty((n, k), torch.bfloat16, w.device)
     _lib.check("svdq_residual", lib.svdq_residual(
         _ptr(w), n, k, _row_stride(w, "w"), _ptr(lam), _ptr(down), _ptr(up), r, _ptr(out), _stream(stream)))
     return out
@@ -299,7 +299,7 @@ def svdq_bits_lost(amax_x: torch.Tensor, inv_lambda: Optional[torch.Tensor] = No
         if il.dtype != torch.float32 or not il.is_cuda or il.stride(1) != 1 or il.shape[1] != k:
             raise ValueError("inv_lambda must be a CUDA float32 [n_cand, K] tensor with unit column stride")
         n_cand, ld_lam = il.shape[0], il.stride(0)
-    bits = torch.empty((n_cand, n_mod), dtype=torch.float64, device=ax.device)
+    bits = _lib.out_empty((n_cand, n_mod), torch.float64, ax.device)
     _lib.check("svdq_bits_lost", lib.svdq_bits_lost(
         _ptr(ax), ax.stride(0), n_mod, _ptr(il), ld_lam, n_cand, k, _ptr(bits), _stream(stream)))
     return bits
@@ -317,9 +317,9 @@ def svdq_lambda_grid(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: torch.Te
         raise ValueError("amax_x and amax_w differ in length")
     n = alpha.numel()
     dev = amax_x.device
-    lam = torch.empty((n, k), dtype=torch.float32, device=dev)
-    inv = torch.empty((n, k), dtype=torch.float32, device=dev)
-    s_g = torch.empty(n, dtype=torch.float32, device=dev)
+    lam = _lib.out_empty((n, k), torch.float32, dev)
+    inv = _lib.out_empty((n, k), torch.float32, dev)
+    s_g = _lib.out_empty(n, torch.float32, dev)
     _lib.check("svdq_lambda_grid", lib.svdq_lambda_grid(
         _ptr(amax_x), _ptr(amax_w), k, _ptr(alpha), n, _ptr(lam), _ptr(inv), _ptr(s_g), _stream(stream)))
     return dict(lam=lam, inv_lam=inv, s_g=s_g)
@@ -339,8 +339,8 @@ def svdq_quantize_mxfp8(x: torch.Tensor, out: Optional[dict] = None, stream=None
     if nbytes == 0:
         raise ValueError("K must be a positive multiple of 128")
     if out is None:
-        out = dict(codes=torch.empty((m, k), dtype=torch.uint8, device=x.device),
-                   sf=torch.empty(nbytes, dtype=torch.uint8, device=x.device))
+        out = dict(codes=_lib.out_empty((m, k), torch.uint8, x.device),
+                   sf=_lib.out_empty(nbytes, torch.uint8, x.device))
     _lib.check("svdq_quantize_mxfp8", lib.svdq_quantize_mxfp8(
         _ptr(x), m, k, _row_stride(x, "x"), _ptr(out["codes"]), _ptr(out["sf"]), _stream(stream)))
     return out
@@ -355,7 +355,7 @@ def svdq_linear_mxfp8(a_codes: torch.Tensor, a_sf: torch.Tensor, w_codes: torch.
     m, k = a_codes.shape
     n = w_codes.shape[0]
     if out is None:
-        out = torch.empty((m, n), dtype=torch.bfloat16, device=a_codes.device)
+        out = _lib.out_empty((m, n), torch.bfloat16, a_codes.device)
     _lib.check("svdq_linear_mxfp8", lib.svdq_linear_mxfp8(
         _ptr(a_codes), _ptr(a_sf), _ptr(w_codes), _ptr(w_sf), _ptr(bias), _ptr(out), _row_stride(out, "out"),
         m, n, k, _stream(stream)))
@@ -363,9 +363,11 @@ def svdq_linear_mxfp8(a_codes: torch.Tensor, a_sf: torch.Tensor, w_codes: torch.
 
 
 def svdq_device_error(stream=None) -> int:
-    """Synchronise and return (then clear) the device error word; 0 = no timeout."""
+    """Synchronise and return (then clear) the device error word: 0 = nothing
+    recorded, 1..6 = a bounded wait ran out, 0x100 + site = a store the debug
+    library found outside its output."""
     code = c_uint32(0)
     st = _lib.load().svdq_device_error(_stream(stream), byref(code))
-    if st not in (_lib.SVDQ_OK, _lib.SVDQ_ERR_TIMEOUT):
+    if st not in (_lib.SVDQ_OK, _lib.SVDQ_ERR_TIMEOUT, _lib.SVDQ_ERR_BOUNDS):
         _lib.check("svdq_device_error", st)
     return int(code.value)

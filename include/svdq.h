@@ -76,7 +76,8 @@ typedef enum {
     SVDQ_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, attribute) */
     SVDQ_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out */
     SVDQ_ERR_NO_DEVICE = 6,     /* no sm_100 device is current */
-    SVDQ_ERR_SCRATCH_TOO_SMALL = 7  /* problem needs more than the library's static scratch array */
+    SVDQ_ERR_SCRATCH_TOO_SMALL = 7, /* problem needs more than the library's static scratch array */
+    SVDQ_ERR_BOUNDS = 8             /* debug library: a device store fell outside its output */
 } svdq_status;
 
 /* Half-open row range [begin, end) of X; a host array of these selects rows. */
@@ -384,10 +385,12 @@ int svdq_bits_lost(const float* amax_x, int64_t ld_amax, int n_mod, const float*
 
 /*
  * svdq_device_error -- synchronise `stream`, then read and clear the current
- * device's error word.  *code receives 0 when no bounded wait ran out since
- * the last call, otherwise a nonzero code naming the wait.  Returns
- * SVDQ_ERR_TIMEOUT if *code != 0, SVDQ_OK otherwise (SVDQ_ERR_CUDA if the
- * synchronisation itself failed).
+ * device's error word.  *code receives 0 when nothing was recorded since the
+ * last call, otherwise the first code recorded: 1..6 name a bounded wait that
+ * ran out (returns SVDQ_ERR_TIMEOUT); 0x100 + site names an output whose
+ * store the debug library found outside the output's extent and skipped
+ * (returns SVDQ_ERR_BOUNDS; sites as listed at svdq_debug_limit_extent).
+ * SVDQ_OK when *code == 0; SVDQ_ERR_CUDA if the synchronisation itself failed.
  */
 int svdq_device_error(void* stream, uint32_t* code);
 
@@ -407,6 +410,36 @@ int svdq_device_error(void* stream, uint32_t* code);
  * range arms nothing that call.
  */
 int svdq_debug_arm_calib_timeout(int64_t unit, int64_t wait_limit_cycles);
+
+/*
+ * The debug library.  libsvdq_debug.so is the same source compiled with
+ * SVDQ_DEBUG_CHECKS=1 (no page has a counterpart; it stands in for a memory
+ * checker).  It adds, to every entry point above:
+ *   - host side: every non-null device-pointer argument must be device (or
+ *     managed) memory of the current device, else SVDQ_ERR_INVALID_ARG and
+ *     nothing is launched;
+ *   - device side: each plain global store of an output is checked against
+ *     the output's extent -- its size as documented above, computed on the
+ *     host apart from the kernel's index arithmetic -- and each TMA store's box
+ *     origin against the output's dims.  A store outside is skipped and
+ *     0x100 + site goes into the error word (svdq_device_error).
+ * Sites: 1 calibration zeroing, 2 calibration absmax, 3 lambda / 1/lambda /
+ * scale, 4 NVFP4 codes, 5 NVFP4 scale bytes, 6 D, 7 linear Y (TMA box
+ * origin, in 16-byte units of a row x rows), 8 linear fp32 Y, 9 fused scoring
+ * partials and results, 10 scoring partials, 11 scoring num / den / rel,
+ * 12 residual, 13 lambda grid (lambda, 1/lambda, scales), 14 bits lost,
+ * 15 MXFP8 codes, 16 MXFP8 scale bytes.
+ *
+ * svdq_debug_build -- 1 in the debug library, 0 in the release one.
+ *
+ * svdq_debug_limit_extent -- test hook of the debug library: the next launch
+ * that stores to `site` checks against min(extent, the output's extent), so a
+ * test can make the check fire without any store leaving the buffer.
+ * One-shot.  SVDQ_ERR_INVALID_ARG for an unknown site or extent < 0;
+ * SVDQ_ERR_UNSUPPORTED in the release library.
+ */
+int svdq_debug_build(void);
+int svdq_debug_limit_extent(int site, int64_t extent);
 
 #ifdef __cplusplus
 }

@@ -27,6 +27,28 @@ def test_library_exports_every_declared_symbol():
         assert name in _lib.SIGNATURES, f"binding lacks {name}"
 
 
+def test_debug_library_exports_and_reports_itself():
+    """The debug build (store bounds checks in the kernels, pointer checks on the
+    host) exports the same entry points; each build says which it is; the
+    extent hook is refused by the release build and checks its arguments in the
+    debug build (host-side only here)."""
+    from bit_w4a4_quantized_svdq_b200.build import DEBUG_LIB_PATH, LIB_PATH
+    rel = ctypes.CDLL(LIB_PATH)
+    dbg = ctypes.CDLL(DEBUG_LIB_PATH)
+    for name in _declared_functions():
+        assert hasattr(dbg, name), name
+    for lib in (rel, dbg):
+        lib.svdq_debug_limit_extent.argtypes = [ctypes.c_int, ctypes.c_int64]
+    assert rel.svdq_debug_build() == 0 and dbg.svdq_debug_build() == 1
+    assert rel.svdq_debug_limit_extent(4, 0) == _lib.SVDQ_ERR_UNSUPPORTED
+    assert dbg.svdq_debug_limit_extent(0, 10) == _lib.SVDQ_ERR_INVALID_ARG
+    assert dbg.svdq_debug_limit_extent(17, 10) == _lib.SVDQ_ERR_INVALID_ARG
+    assert dbg.svdq_debug_limit_extent(4, -1) == _lib.SVDQ_ERR_INVALID_ARG
+    assert dbg.svdq_debug_limit_extent(16, 0) == _lib.SVDQ_OK
+    dbg.svdq_status_string.restype = ctypes.c_char_p
+    assert dbg.svdq_status_string(_lib.SVDQ_ERR_BOUNDS).startswith(b"a device store fell outside")
+
+
 def test_version_and_status_strings():
     lib = _lib.load()
     assert lib.svdq_version() == 100
