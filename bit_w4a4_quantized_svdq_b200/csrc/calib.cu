@@ -294,6 +294,7 @@ calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 m3 = __vmaxu2(m3, q.w & 0x7FFF7FFFu);
             }
         }
+        consumed(m0, m1, m2, m3);                     // the unit's loads are in these maxima
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
     }

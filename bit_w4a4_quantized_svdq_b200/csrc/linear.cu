@@ -12,30 +12,29 @@
 //   Y[m, n] = alpha * (sum_k A[m,k] B[n,k] + sum_j D'[m,j] up[n,j]) + bias[n]
 //   alpha   = s_g_act * s_g_w,   D' = D / alpha (split into bf16 hi + lo)
 //
-// One persistent CTA per SM walks 128 x 256 output tiles (the smaller
-// operand's blocks fastest, so it stays in L2).  Warps:
-//   0     TMA producer: per 256-channel stage, A codes 128 x 128 B and B codes
-//         256 x 128 B (128-byte swizzle); every second stage, the scale atoms of
-//         the next two stages (A 4 KB, W 8 KB) with two 3-D tensor loads into a
-//         2-slot ring
-//   1     tcgen05 issuer and tensor-memory owner: per stage one barrier wait and
-//         4 kind::mxf4nvf4 block16 MMAs (K = 64 each) into one fp32
-//         accumulator, then per tile 4 kind::f16 MMAs for the low-rank term
-//         (K = 64: 32 ranks of D'_hi then 32 of D'_lo against up twice)
-//   2     low-rank operand builder: D' hi/lo and the duplicated up tile written
-//         into the swizzled operand layout in shared memory
-//   3..6  block-scale writers: each stage's scale atoms, shared memory ->
+// One persistent CTA per SM walks 128 x 256 output tiles (in bands of the
+// operand walked fastest, so that band stays in L2).  Warps:
+//   0     operand producer: per 256-channel stage, A codes 128 x 128 B and B
+//         codes 256 x 128 B (128-byte swizzle) into a four-stage ring; each
+//         tile's first ring position is its low-rank stage, handed to the
+//         epilogue warps to fill
+//   1     tcgen05 issuer and tensor-memory owner: per tile 4 kind::f16 MMAs for
+//         the low-rank term (K = 64: 32 ranks of D'_hi then 32 of D'_lo
+//         against up twice), which start the accumulator; then per stage one
+//         barrier wait and 4 kind::mxf4nvf4 block16 MMAs (K = 64 each)
+//   2..5  block-scale writers: each stage's scale atoms, shared memory ->
 //         registers -> tensor memory (tcgen05.st, one warp per lane quarter),
 //         into a per-stage buffer, then an arrival on the stage's barrier; this
 //         keeps the tensor pipe free for MMAs
-//   7..14 epilogue (two warps per tensor-memory lane quarter): tensor memory ->
-//         registers, alpha and bias, bf16 rows staged in shared memory and
-//         written by TMA bulk stores (fp32 rows: plain stores); the accumulator
-//         is released as soon as it has been read, so the stores overlap the
-//         next tile's main loop.
-// The low-rank MMAs close each tile, so their operand area doubles as the
-// epilogue's output staging: builder -> MMA -> epilogue -> builder.
-//
+//   6..13 epilogue (two warps per tensor-memory lane quarter): the next tile's
+//         low-rank stage (D' hi/lo and up in the swizzled operand layout), then
+//         tensor memory -> registers, alpha and bias, bf16 rows staged in shared
+//         memory and written by TMA bulk stores (fp32 rows: plain stores); the
+//         accumulator is released as soon as it has been read, so the stores
+//         overlap the next tile's main loop
+//   14    scale producer: the scale atoms of two stages at a time (A 4 KB, W
+//         8 KB, two 3-D tensor loads) into a 2-slot ring, from its own thread so
+//         the operand copies never queue behind them
 // Instantiations (linear_kernel<out fp32, score, MXFP8>):
 //   <0|1, 0, 0>  svdq_linear: the NVFP4 linear, bf16 or fp32 output
 //   <0, 1, 0>    svdq_linear_score: the same, with the tile scored against a bf16
@@ -66,14 +65,17 @@ constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBKBytes = 128;                 // packed FP4 bytes per row per stage (256 channels)
 constexpr int kBK = 256;                      // channels per stage
-constexpr int kThreads = 448;                 // 14 warps
+constexpr int kThreads = 480;                 // 15 warps
 constexpr int kSfWarp0 = 2;                   // warps 2..5 write block scales into tensor memory
 constexpr int kSfWarps = 4;
 constexpr int kEpiWarp0 = 6;                  // warps 6..13: epilogue
 constexpr int kEpiWarps = 8;
-static_assert(kSfWarp0 == 2 && kSfWarp0 + kSfWarps == kEpiWarp0 && kEpiWarp0 + kEpiWarps == kThreads / 32,
-              "warp roles: 0 producer, 1 MMA issuer, 2..5 scale writers, 6..13 epilogue; each group of four "
-              "consecutive warps covers the four tensor-memory lane quarters (warp % 4)");
+constexpr int kSfLoadWarp = 14;               // warp 14: scale-atom copies
+static_assert(kSfWarp0 == 2 && kSfWarp0 + kSfWarps == kEpiWarp0 && kEpiWarp0 + kEpiWarps == kSfLoadWarp &&
+                  kSfLoadWarp + 1 == kThreads / 32,
+              "warp roles: 0 operand producer, 1 MMA issuer, 2..5 scale writers, 6..13 epilogue, 14 scale "
+              "producer; each group of four consecutive warps covers the four tensor-memory lane quarters "
+              "(warp % 4)");
 
 constexpr uint32_t kATile = kBM * kBKBytes;          // 16 KB
 constexpr uint32_t kBTile = kBN * kBKBytes;          // 32 KB
@@ -183,7 +185,11 @@ __device__ __forceinline__ void pair_add(float& hi, float& lo, float x) {
 // bands of `band` blocks: every block of the other operand passes under one band
 // before the next band starts, so the band stays resident and the larger operand
 // is read once per band.
-__device__ __forceinline__ void tile_coords(const LinearArgs& a, int tile, int& m_blk, int& n_blk) {
+struct TileOrder {
+    int m_tiles, n_tiles, n_fastest, band;
+};
+
+__device__ __forceinline__ void tile_coords(const TileOrder& a, int tile, int& m_blk, int& n_blk) {
     const int fast_tiles = a.n_fastest ? a.n_tiles : a.m_tiles;
     const int slow_tiles = a.n_fastest ? a.m_tiles : a.n_tiles;
     const int per_band = a.band * slow_tiles;                // tiles of one full band
@@ -199,6 +205,10 @@ __device__ __forceinline__ void tile_coords(const LinearArgs& a, int tile, int& 
         m_blk = fast;
         n_blk = slow;
     }
+}
+
+__device__ __forceinline__ void tile_coords(const LinearArgs& a, int tile, int& m_blk, int& n_blk) {
+    tile_coords(TileOrder{a.m_tiles, a.n_tiles, a.n_fastest, a.band}, tile, m_blk, n_blk);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -269,6 +279,52 @@ __device__ __forceinline__ bool lr_stage(const LinearArgs& a, uint8_t* slot, uin
     if (!fail && (etid & 31) == 0 && etid < 4 * 32) mbar_arrive(full_bar);
     if (!fail && etid == 0) mbar_arrive(done_bar);
     return !fail;
+}
+
+// The scale atoms of two stages per copy pair into a 2-slot ring (`ring`,
+// kSfSlot bytes a slot), in the operand producer's tile order, as far ahead as
+// the writers free the slots.  Issued from their own thread (warp 14): TMA issue
+// from one thread is serial, so the operand copies never queue behind these.
+template <bool kMx>
+__device__ __forceinline__ void scale_producer(const CUtensorMap* tmap_sfa, const CUtensorMap* tmap_sfb,
+                                            TileOrder order, uint32_t* err, uint8_t* ring, uint64_t* sf_data,
+                                            uint64_t* sf_free, volatile uint32_t* abort_flag, int num_tiles,
+                                            int k_stages) {
+    constexpr uint32_t kSfaPairT = kMx ? 1024 : kSfaPair;          // A scale bytes of two stages
+    constexpr uint32_t kSfSlotT = kMx ? 3072 : kSfSlot;            // A + W scale bytes of two stages
+    constexpr int kSfHalvesPerStage = kMx ? 2 : 8;                  // 256-byte scale pieces per row block
+    prefetch_tmap(tmap_sfa);
+    prefetch_tmap(tmap_sfb);
+    pdl_wait();                                   // the activation scales are written
+    const uint64_t pol_keep = l2_evict_last_policy(), pol_once = l2_evict_first_policy();
+    const uint64_t pol_a = order.n_fastest ? pol_once : pol_keep;
+    const uint64_t pol_b = order.n_fastest ? pol_keep : pol_once;
+    int issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        int m_blk, n_blk;
+        tile_coords(order, tile, m_blk, n_blk);
+        for (int kb = 0; kb < k_stages; kb += 2) {
+            const int slot = issued & 1;
+            if (issued >= 2 &&
+                !mbar_wait(&sf_free[slot], ((issued >> 1) & 1) ^ 1, abort_flag, err, kErrWaitEmpty)) {
+                ok = false;
+                break;
+            }
+            uint8_t* dst = ring + slot * kSfSlot;
+            mbar_arrive_expect_tx(&sf_data[slot], kSfSlotT);
+            // scale atoms of stages kb and kb + 1 (a last odd stage reads zeros past K)
+            tma_load_3d_hint(dst, tmap_sfa, &sf_data[slot], 0, kb * kSfHalvesPerStage, m_blk, pol_a);
+            tma_load_3d_hint(dst + kSfaPairT, tmap_sfb, &sf_data[slot], 0, kb * kSfHalvesPerStage, 2 * n_blk,
+                             pol_b);
+            ++issued;
+        }
+    }
+    // Bounded drain of the copies still in flight.
+    for (int q = (issued > 2 ? issued - 2 : 0); q < issued; ++q) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&sf_data[q & 1], (q >> 1) & 1) && clock64() - t0 < kWaitLimitCycles) {}
+    }
 }
 
 template <bool kOutF32, bool kScore, bool kMx>
@@ -348,43 +404,16 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         if (lane == 0) {
             prefetch_tmap(&tmap_a);
             prefetch_tmap(&tmap_b);
-            prefetch_tmap(&tmap_sfa);
-            prefetch_tmap(&tmap_sfb);
-            pdl_wait();                               // the activation codes and scales are written
+            pdl_wait();                               // the activation codes are written
             // L2 policies: the operand walked fastest over the tiles (the smaller
             // one) is re-read by every block row (or column) of the other, so it
             // is kept; the other streams through once.
             const uint64_t pol_keep = l2_evict_last_policy(), pol_once = l2_evict_first_policy();
             const uint64_t pol_a = args.n_fastest ? pol_once : pol_keep;
             const uint64_t pol_b = args.n_fastest ? pol_keep : pol_once;
-            // Scale batches run one batch (two stages) ahead of the operands: the
-            // batch a stage needs has landed by the time its operands do.
-            int sf_tile = blockIdx.x, sf_kb = 0, issued = 0;
-            auto issue_scales = [&]() -> bool {
-                if (sf_tile >= num_tiles) return true;
-                const int slot = issued & 1;
-                if (issued >= 2 &&
-                    !mbar_wait(&sf_free[slot], ((issued >> 1) & 1) ^ 1, abort_flag, args.err, kErrWaitEmpty))
-                    return false;
-                int m_blk, n_blk;
-                tile_coords(args, sf_tile, m_blk, n_blk);
-                uint8_t* dst = smem + L::kOffSf + slot * kSfSlot;
-                mbar_arrive_expect_tx(&sf_data[slot], kSfSlotT);
-                // scale atoms of stages sf_kb and sf_kb + 1 (a last odd stage reads zeros past K)
-                tma_load_3d_hint(dst, &tmap_sfa, &sf_data[slot], 0, sf_kb * kSfHalvesPerStage, m_blk, pol_a);
-                tma_load_3d_hint(dst + kSfaPairT, &tmap_sfb, &sf_data[slot], 0, sf_kb * kSfHalvesPerStage, 2 * n_blk,
-                                 pol_b);
-                ++issued;
-                sf_kb += 2;
-                if (sf_kb >= k_stages) {
-                    sf_kb = 0;
-                    sf_tile += gridDim.x;
-                }
-                return true;
-            };
             int s = 0, it = 0, lr_tiles = 0;
             uint32_t ph = 0;
-            bool ok = issue_scales();
+            bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 int m_blk, n_blk;
                 tile_coords(args, tile, m_blk, n_blk);
@@ -415,7 +444,6 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     mbar_arrive_expect_tx(&full[s], kStageBytes);
                     tma_load_2d_hint(st, &tmap_a, &full[s], kb * kBKBytes, m_blk * kBM, pol_a);
                     tma_load_2d_hint(st + kATile, &tmap_b, &full[s], kb * kBKBytes, n_blk * kBN, pol_b);
-                    if ((kb & 1) == 0 && !issue_scales()) { ok = false; break; }
                     if (++s == kStagesT) { s = 0; ph ^= 1u; }
                 }
             }
@@ -424,11 +452,12 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 const long long t0 = clock64();
                 while (!mbar_try_wait(&full[i % kStagesT], (i / kStagesT) & 1) && clock64() - t0 < kWaitLimitCycles) {}
             }
-            for (int q = (issued > 2 ? issued - 2 : 0); q < issued; ++q) {
-                const long long t0 = clock64();
-                while (!mbar_try_wait(&sf_data[q & 1], (q >> 1) & 1) && clock64() - t0 < kWaitLimitCycles) {}
-            }
         }
+    } else if (warp == kSfLoadWarp) {
+        // ------------------------------------------------------------ scale-atom producer
+        if (lane == 0)
+            scale_producer<kMx>(&tmap_sfa, &tmap_sfb, TileOrder{args.m_tiles, args.n_tiles, args.n_fastest, args.band},
+                                args.err, smem + L::kOffSf, sf_data, sf_free, abort_flag, num_tiles, k_stages);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         // Kept to the minimum between MMAs: one wait per stage (the barrier counts
@@ -500,7 +529,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
         // holds the full set, the layout the block-scaled MMA reads), then
         // arrives on the stage's barrier.  Unlike a shared->tensor copy issued by
         // the MMA thread, these stores run alongside the MMAs instead of in front
-        // of them.  Ring slot: released once both of its stages are in registers.
+        // of them.  Ring slot: released after the stores of its last stage.
         // Tensor-memory buffer s: written only after the MMAs of its previous
         // use have completed (the stage's empty barrier).  Low-rank stages are
         // the epilogue's: the writers only step over them.
@@ -551,10 +580,6 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                         rb[8 * q + 4] = y.x; rb[8 * q + 5] = y.y; rb[8 * q + 6] = y.z; rb[8 * q + 7] = y.w;
                     }
                 }
-                if ((kb & 1) == 1 || kb == k_stages - 1) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sf_free[slot]);
-                }
                 if (it >= kStagesT && !mbar_try_wait(&empty[s], ph ^ 1) &&
                     !mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) {
                     ok = false;
@@ -574,6 +599,11 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[s]);
+                // The ring slot is released only now: the shared-memory loads above
+                // are complete once the tensor-memory stores that read their
+                // registers have been issued, and a slot released with loads still
+                // in flight could be refilled by the next copy under them.
+                if (lane == 0 && ((kb & 1) == 1 || kb == k_stages - 1)) mbar_arrive(&sf_free[slot]);
                 if (++s == kStagesT) { s = 0; ph ^= 1u; }
             }
         }
@@ -674,7 +704,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     uint32_t v[2][32];
                     tmem_ld_32x32b_x32(tbase, v[0]);
                     tmem_ld_32x32b_x32(tbase + 32, v[1]);
-                    tmem_ld_wait();
+                    tmem_ld_wait(v[0]);
+                    tmem_ld_tie(v[1]);
                     convert(v[0], 0);
                     convert(v[1], 1);
                 }
@@ -682,7 +713,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 for (int c = 2; c < 4; ++c) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, v);
-                    tmem_ld_wait();
+                    tmem_ld_wait(v);
                     if (c == 3) {                   // the accumulator has been read: next tile's MMAs may start
                         tc_fence_before();
                         __syncwarp();
@@ -858,7 +889,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     uint32_t v[2][32];
                     tmem_ld_32x32b_x32(tbase, v[0]);
                     tmem_ld_32x32b_x32(tbase + 32, v[1]);
-                    tmem_ld_wait();
+                    tmem_ld_wait(v[0]);
+                    tmem_ld_tie(v[1]);
                     convert(v[0], 0);
                     convert(v[1], 1);
                 }
@@ -866,10 +898,10 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     // one piece at a time: the converted columns and one load fit the registers
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tbase + 64, v);
-                    tmem_ld_wait();
+                    tmem_ld_wait(v);
                     convert(v, 2);
                     tmem_ld_32x32b_x32(tbase + 96, v);
-                    tmem_ld_wait();
+                    tmem_ld_wait(v);
                     tc_fence_before();              // the accumulator has been read: next tile's MMAs may start
                     __syncwarp();
                     if (lane == 0) mbar_arrive(acc_empty);
@@ -899,7 +931,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 for (int c = 0; c < kBN / 2 / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, v);
-                    tmem_ld_wait();
+                    tmem_ld_wait(v);
                     if (row_ok && ccol + c * 32 < args.N) {           // N % 128 == 0: chunks are whole
                         const int64_t off = row * args.ldy + ccol + c * 32;
                         float* dst = static_cast<float*>(args.Y) + off;

@@ -316,6 +316,8 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             const uint32_t n3 = __shfl_down_sync(0xffffffffu, sf2, 3);
             const uint32_t x01 = __byte_perm(sf2, n1, 0x5140);   // a0 b0 a1 b1
             const uint32_t x23 = __byte_perm(n2, n3, 0x5140);    // c0 d0 c1 d1
+            consumed(ca.x, ca.y, cb.x, cb.y);            // every loaded value of the stage is in these
+            consumed(x01, x23);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);        // shared memory of this stage no longer read
             const int64_t coff = chunk * (kBK / 2) + b * 8;
@@ -358,7 +360,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 if constexpr (R == 32) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr, v);
-                    tmem_ld_wait();
+                    tmem_ld_wait(v);
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4*>(part + j) = make_float4(
@@ -367,7 +369,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 } else {
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(taddr, v);
-                    tmem_ld_wait();
+                    tmem_ld_wait(v);
 #pragma unroll
                     for (int j = 0; j < 16; j += 4)
                         *reinterpret_cast<float4*>(part + j) = make_float4(

@@ -249,13 +249,15 @@ score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict_
                     vb[v] = make_uint4(0, 0, 0, 0);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);           // slot read: the producer may refill it
             double num = 0.0, den = 0.0;
 #pragma unroll
             for (int v = 0; v < kVecPerThread; ++v) accum8(va[v], vb[v], num, den);
             num = consumer_sum(num, sh);
             den = consumer_sum(den, sh);
+            // The slot is released once the loaded values have been used (the
+            // shuffles of the sums read them): a release with shared-memory loads
+            // still in flight could let the next copy land under them.
+            if (lane == 0) mbar_arrive(&empty[s]);
             if (threadIdx.x == 0 && store_ok(2 * c, 2, ext_part, err, kSiteScorePart)) {
                 partial[2 * c] = num;
                 partial[2 * c + 1] = den;

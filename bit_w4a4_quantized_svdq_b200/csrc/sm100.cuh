@@ -128,6 +128,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
+// A consumer's values computed from a shared-memory stage, tied in place
+// before it releases the stage: the compiler may not sink their computation
+// past this point, and since a warp issues in order and these instructions wait
+// for the loads they read, the release below cannot be issued while a load of
+// the stage is still in flight (the next copy into the stage could otherwise
+// land under it).
+__device__ __forceinline__ void consumed(uint32_t a, uint32_t b) { asm volatile("" :: "r"(a), "r"(b) : "memory"); }
+__device__ __forceinline__ void consumed(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("" :: "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -402,6 +413,39 @@ __device__ __forceinline__ void tmem_st_wait() {
 
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// tcgen05.ld writes its destination registers asynchronously: they hold the
+// loaded values only after tcgen05.wait::ld.  To the compiler the registers are
+// ready as soon as the load's asm statement ends, so it may move their uses
+// above a plain wait.  These waits also pass the registers through the asm
+// statement ("+r"), so every use depends on the wait.  After one wait, further
+// arrays loaded before it are tied with tmem_ld_tie (an empty asm, ordered
+// after the wait as both are volatile).
+__device__ __forceinline__ void tmem_ld_tie(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_tie(uint32_t (&r)[16]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[N]) {
+    tmem_ld_wait();
+    tmem_ld_tie(r);
 }
 
 // ---------------------------------------------------------------------------
