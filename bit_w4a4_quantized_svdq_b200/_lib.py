@@ -62,7 +62,7 @@ SIGNATURES = {
     "svdq_residual": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_int,
                               c_void_p, c_void_p]),
     "svdq_device_error": (c_int, [c_void_p, POINTER(c_uint32)]),
-    "svdq_debug_arm_calib_timeout": (c_int, [c_int64, c_int64]),
+    "svdq_debug_arm_score_timeout": (c_int, [c_int64, c_int64]),
     "svdq_debug_build": (c_int, []),
     "svdq_debug_limit_extent": (c_int, [c_int, c_int64]),
     "svdq_linear_score": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p,

@@ -11,64 +11,65 @@
 // values integer order equals value order, so two channels reduce per packed
 // 16-bit unsigned max (__vmaxu2).
 //
-// Streaming: the work is cut into units of 32 rows x 256 channels (a strip of
-// channels; rows counted from the start of each selected row segment), ordered
-// matrix, strip, segment, row box.  One persistent CTA per SM takes a
-// contiguous range of units; its producer warp brings each unit into an
-// 8-slot shared-memory ring with a TMA tensor load (a constant 128 KB in
-// flight per SM), its 8 consumer warps keep a running max per channel of the
-// current strip and merge it into the outputs (integer atomicMax on the fp32
-// bit patterns: exact, order independent) whenever the strip changes.
+// Streaming: the channels are cut into bands of 2048 and the rows of each
+// matrix (the selected rows of X, counted across its row segments, then the
+// rows of W) into chunks; one 1024-thread CTA takes one (band, chunk) item: 256
+// thread columns of 8 channels by 4 row slices, each thread reading its 16 bytes
+// of every fourth row of the chunk with streaming loads, eight rows in flight
+// (128 KB per SM).  A row's band is 4 KB of contiguous memory and the CTAs of a
+// wave together cover whole rows: the wider a row's piece, the closer plain
+// loads come to the copy bandwidth (4 KB pieces 5.6 TB/s, 1 KB pieces 4.8 TB/s
+// on the 16384 x 20480 input).  The running maxima stay in registers (four
+// packed words per thread), meet across the row slices in shared memory, and
+// are merged into the outputs once per item (integer atomicMax on the fp32 bit
+// patterns: exact and order independent).  One atomic per channel per item is
+// what sizes the items: one CTA per SM, so the chunks per band are the SMs over
+// the bands.
 //
-// Completion without scratch memory: the first lambda word of each strip
-// counts, for the duration of the call, the merges into that strip; the CTA
-// whose merge is the strip's last (the number of merges follows from the unit
-// ranges) forms lambda and 1/lambda for the strip's 256 channels.  The strip
-// maxima of RN(ax / lambda) / 2688 meet in the bits of the s_g output
-// (atomicMax; division by 2688 is monotonic, so the max of the quotients is
-// the quotient of the max), and lambda[1] counts finished strips; the last
-// strip writes the final s_g (1 when every maximum is 0) and lambda[1].  So the
-// call is two launches: a zeroing kernel and the reduction.  The reduction is a
-// programmatic dependent of the zeroing kernel: its loads of X and W start while
-// the zeroing runs, and its consumers wait for it (griddepcontrol.wait) before
-// their first write to the outputs.
+// Completion without scratch memory: the first lambda word of each band
+// counts, for the duration of the call, the items merged into that band; the
+// CTA whose merge is the band's last forms lambda and 1/lambda for its 2048
+// channels.  The band maxima of RN(ax / lambda) / 2688 meet in the bits of the
+// s_g output (atomicMax; division by 2688 is monotonic, so the max of the
+// quotients is the quotient of the max), and lambda[1] counts finished bands;
+// the last band writes the final s_g (1 when every maximum is 0) and lambda[1].
+// So the call is two launches: a zeroing kernel and the reduction.  The
+// reduction is a programmatic dependent of the zeroing kernel: its loads of X
+// and W run while the zeroing finishes, and it waits for it
+// (griddepcontrol.wait) before its first write to the outputs.
+#include <algorithm>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
 namespace svdq {
 namespace {
 
-constexpr int kStripCols = 256;               // channels per unit (512 bytes per row)
-constexpr int kBoxRows = 32;                  // rows per unit
-constexpr int kSlots = 8;                     // ring slots of 16 KB
-constexpr int kConsumerWarps = 8;             // 4 rows of each unit per warp
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;     // + producer warp
-constexpr uint32_t kUnitBytes = kBoxRows * kStripCols * 2;   // 16 KB
-constexpr uint32_t kSmemBytes = kSlots * kUnitBytes + 256;
+constexpr int kThreads = 1024;
+constexpr int kColThreads = 256;              // thread columns of a band
+constexpr int kRowSlices = kThreads / kColThreads;   // rows r, r + 4, ... per slice
+constexpr int kBandCols = kColThreads * 8;    // channels per band (16 bytes of bf16 per thread)
+constexpr int kRowsInFlight = 8;              // rows loaded per thread before they are reduced
 
 struct CalibArgs {
-    SegTable segs;                            // row selection of X
-    int64_t box_prefix[kMaxSegments + 1];     // row boxes before segment s (X)
-    int64_t boxes[2];                         // row boxes per strip: X (all segments), W
-    int64_t units[2];                         // strips * boxes
-    int64_t n_units;                          // units[0] + units[1]
-    int64_t N;                                // rows of W
+    const uint16_t* x;
+    int64_t ldx;
+    const uint16_t* w;                        // nullptr when the weight is not read here
+    int64_t ldw;
+    SegTable segs;                            // selected rows of X
     int64_t K;
-    int64_t strips;
+    int64_t bands;
+    int64_t chunk_rows;                       // rows per chunk (both matrices)
+    int64_t chunks[2];                        // chunks of X's selected rows, of W's rows
+    int64_t rows[2];                          // selected rows of X, rows of W
     uint32_t* out_bits[2];                    // absmax of X, of W (fp32 bit patterns)
     const float* ax;
-    const float* aw;                          // nullptr when there is no weight
+    const float* aw;                          // nullptr: lambda = 1
     float* lambda;
     float* inv_lambda;
-    float* s_g;                               // holds max(strip maxima) until the last strip writes the scale
+    float* s_g;                               // holds max(band maxima) until the last band writes the scale
     uint32_t* err;
     int64_t ext_amax, ext_lambda;             // store-check extents (debug library): K each
-    // Time-out test (armed from the host, one call): CTA 0's producer leaves its
-    // ring unit `skip_unit` unloaded, so a consumer's wait for it runs out after
-    // `wait_limit` cycles; -1 = off.  Every other CTA and call runs normally.
-    int64_t skip_unit;
-    long long wait_limit;
 };
 
 __global__ void __launch_bounds__(256)
@@ -79,13 +80,9 @@ calib_zero_kernel(float* ax, float* aw, int64_t K, float* lambda, float* s_g, in
         if (!store_ok(j, 1, ext, err, kSiteCalibZero)) continue;
         ax[j] = 0.0f;
         if (aw) aw[j] = 0.0f;
-        if (j % kStripCols == 0 || j == 1) lambda[j] = 0.0f;   // strip counters, strips-done counter
+        if (j % kBandCols == 0 || j == 1) lambda[j] = 0.0f;   // band counters, bands-done counter
     }
     if (blockIdx.x == 0 && threadIdx.x == 0) *reinterpret_cast<uint32_t*>(s_g) = 0u;
-}
-
-__device__ __forceinline__ void consumers_sync() {
-    asm volatile("bar.sync 1, %0;" :: "n"(kConsumers) : "memory");
 }
 
 __device__ __forceinline__ float lambda_of(float x, const float* aw, int64_t j) {
@@ -94,33 +91,39 @@ __device__ __forceinline__ float lambda_of(float x, const float* aw, int64_t j) 
     return (x > 0.0f && w > 0.0f) ? __fsqrt_rn(__fdiv_rn(x, w)) : 1.0f;
 }
 
-// By the consumer threads of the CTA that made a strip's last merge:
-// lambda_j = sqrt(ax_j / aw_j) (1 where either absmax is 0) and 1/lambda_j for
-// the strip's channels, then the strip's share of s_g = max_j(ax_j / lambda_j) / (6 * 448).
-__device__ void strip_lambda(const CalibArgs& a, int64_t strip) {
-    __shared__ float red[kConsumerWarps];
-    const int64_t j = strip * kStripCols + threadIdx.x;
+__device__ __forceinline__ float block_max(float v, float* red) {
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int w = 1; w < kThreads / 32; ++w) v = fmaxf(v, red[w]);
+    return v;                                 // valid in thread 0
+}
+
+// By the CTA that made a band's last merge: lambda_j = sqrt(ax_j / aw_j) (1
+// where either absmax is 0) and 1/lambda_j for the band's channels, then the
+// band's share of s_g = max_j(ax_j / lambda_j) / (6 * 448).
+__device__ void band_lambda(const CalibArgs& a, int64_t band) {
+    __shared__ float red[kThreads / 32];
+    const int64_t j1 = min(a.K, (band + 1) * kBandCols);
     float v = 0.0f;
-    if (j < a.K) {
+    for (int64_t j = band * kBandCols + threadIdx.x; j < j1; j += kThreads) {
         const float x = __ldcg(a.ax + j);
         const float lam = lambda_of(x, a.aw, j);
         const float il = __frcp_rn(lam);
         if (store_ok(j, 1, a.ext_lambda, a.err, kSiteCalibLambda)) {
-            if (j != 1) a.lambda[j] = lam;      // lambda[1] is the strips-done counter until the end
+            if (j != 1) a.lambda[j] = lam;          // lambda[1] is the bands-done counter until the end
             if (a.inv_lambda) a.inv_lambda[j] = il;
         }
-        v = __fmul_rn(x, il);
+        v = fmaxf(v, __fmul_rn(x, il));
     }
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    consumers_sync();
+    v = block_max(v, red);
     if (threadIdx.x == 0) {
-        for (int w = 1; w < kConsumerWarps; ++w) v = fmaxf(v, red[w]);
         const float q = __fdiv_rn(v, 2688.0f);
         if (q > 0.0f) atomicMax(reinterpret_cast<uint32_t*>(a.s_g), __float_as_uint(q));
         __threadfence();
         const uint32_t done = atomicAdd(reinterpret_cast<uint32_t*>(a.lambda + 1), 1u);
-        if (done == static_cast<uint32_t>(a.strips) - 1) {
+        if (done == static_cast<uint32_t>(a.bands) - 1) {
             __threadfence();
             const float m = __uint_as_float(atomicAdd(reinterpret_cast<uint32_t*>(a.s_g), 0u));
             const float x1 = __ldcg(a.ax + 1);
@@ -128,195 +131,114 @@ __device__ void strip_lambda(const CalibArgs& a, int64_t strip) {
             *a.s_g = m > 0.0f ? m : 1.0f;
         }
     }
-    consumers_sync();
 }
 
-// CTA that owns unit u when n units are split into g contiguous ranges
-// [i n / g, (i + 1) n / g).
-__device__ __forceinline__ int64_t unit_owner(int64_t u, int64_t g, int64_t n) {
-    return ((u + 1) * g - 1) / n;
+__device__ __forceinline__ void max_row(uint32_t (&m)[4], const uint4& q) {
+    m[0] = __vmaxu2(m[0], q.x & 0x7FFF7FFFu);
+    m[1] = __vmaxu2(m[1], q.y & 0x7FFF7FFFu);
+    m[2] = __vmaxu2(m[2], q.z & 0x7FFF7FFFu);
+    m[3] = __vmaxu2(m[3], q.w & 0x7FFF7FFFu);
 }
 
-// Merges a strip receives: one per CTA whose range meets the strip's units of a matrix.
-__device__ int64_t strip_merges(const CalibArgs& a, int64_t strip, int64_t g) {
-    int64_t m = 0;
-    int64_t base = 0;
-    for (int j = 0; j < 2; ++j) {
-        if (a.boxes[j] > 0) {
-            const int64_t first = base + strip * a.boxes[j];
-            const int64_t last = first + a.boxes[j] - 1;
-            m += unit_owner(last, g, a.n_units) - unit_owner(first, g, a.n_units) + 1;
-        }
-        base += a.units[j];
+// Keeps the compiler from interleaving the maxima with the loads (which would
+// leave one load in flight at a time): the loaded values pass through here first.
+__device__ __forceinline__ void in_flight(uint4 (&q)[kRowsInFlight]) {
+    static_assert(kRowsInFlight == 8, "one operand list per load");
+    asm volatile(""
+                 : "+r"(q[0].x), "+r"(q[0].y), "+r"(q[0].z), "+r"(q[0].w), "+r"(q[1].x), "+r"(q[1].y), "+r"(q[1].z),
+                   "+r"(q[1].w), "+r"(q[2].x), "+r"(q[2].y), "+r"(q[2].z), "+r"(q[2].w), "+r"(q[3].x), "+r"(q[3].y),
+                   "+r"(q[3].z), "+r"(q[3].w), "+r"(q[4].x), "+r"(q[4].y), "+r"(q[4].z), "+r"(q[4].w), "+r"(q[5].x),
+                   "+r"(q[5].y), "+r"(q[5].z), "+r"(q[5].w), "+r"(q[6].x), "+r"(q[6].y), "+r"(q[6].z), "+r"(q[6].w),
+                   "+r"(q[7].x), "+r"(q[7].y), "+r"(q[7].z), "+r"(q[7].w));
+}
+
+// Maxima of this thread's 8 channels (column `col`) over rows r0, r0 + step,
+// ... below r1 of a matrix with row stride ld, kRowsInFlight rows loaded before
+// they are reduced.
+__device__ __forceinline__ void max_rows(uint32_t (&m)[4], const uint16_t* base, int64_t ld, int64_t r0, int64_t r1,
+                                         int step, int64_t col) {
+    const int64_t stride = ld * step;
+    const uint16_t* p = base + r0 * ld + col;
+    int64_t r = r0;
+    for (; r + (kRowsInFlight - 1) * step < r1; r += kRowsInFlight * step, p += kRowsInFlight * stride) {
+        uint4 q[kRowsInFlight];
+#pragma unroll
+        for (int i = 0; i < kRowsInFlight; ++i) q[i] = __ldcs(reinterpret_cast<const uint4*>(p + i * stride));
+        in_flight(q);                          // all eight loads issue before the first max waits for one
+#pragma unroll
+        for (int i = 0; i < kRowsInFlight; ++i) max_row(m, q[i]);
     }
-    return m;
+    for (; r < r1; r += step, p += stride) max_row(m, __ldcs(reinterpret_cast<const uint4*>(p)));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-calib_stream_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                    const __grid_constant__ CalibArgs a) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSlots * kUnitBytes);
-    uint64_t* empty = full + kSlots;
-    uint32_t* meta = reinterpret_cast<uint32_t*>(empty + kSlots);          // per slot: strip, matrix, rows
-    volatile uint32_t* abort_flag = meta + kSlots;
-    __shared__ uint32_t red[kConsumerWarps][32][4];
+calib_rows_kernel(const __grid_constant__ CalibArgs a) {
     __shared__ uint32_t is_last;
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int64_t G = gridDim.x;
-    const int64_t g = blockIdx.x;
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kSlots; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
+    __shared__ uint4 slice_max[kRowSlices - 1][kColThreads];
+    const int64_t band = blockIdx.x % a.bands;
+    const int64_t chunk = blockIdx.x / a.bands;
+    const int job = chunk < a.chunks[0] ? 0 : 1;
+    const int64_t c = job ? chunk - a.chunks[0] : chunk;
+    const int64_t p0 = c * a.chunk_rows;
+    const int64_t p1 = min(p0 + a.chunk_rows, a.rows[job]);
+    const int tc = threadIdx.x % kColThreads, tr = threadIdx.x / kColThreads;
+    const int64_t col = band * kBandCols + tc * 8;
+    const bool active = col < a.K;             // K % 8 == 0: a thread's 8 channels are all in or all out
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
+    if (active && p0 < p1) {
+        if (job == 0) {
+            // the chunk's selected rows, segment by segment; this slice takes every
+            // kRowSlices-th of them, counted from the chunk's first
+            int s = 0;
+            while (s + 1 < a.segs.n && p0 >= a.segs.prefix[s + 1]) ++s;
+            for (int64_t p = p0; p < p1; ++s) {
+                const int64_t e = min(p1, a.segs.prefix[s + 1]);
+                const int64_t first = p + ((tr - (p - p0)) % kRowSlices + kRowSlices) % kRowSlices;
+                const int64_t row = a.segs.begin[s] + (first - a.segs.prefix[s]);
+                if (first < e) max_rows(m, a.x, a.ldx, row, row + (e - first), kRowSlices, col);
+                p = e;
+            }
+        } else {
+            max_rows(m, a.w, a.ldw, p0 + tr, p1, kRowSlices, col);
         }
-        *abort_flag = 0;
-        fence_mbar_init();
+    }
+    // the row slices meet in shared memory: slice 0 keeps the band's maxima
+    if (tr > 0) slice_max[tr - 1][tc] = make_uint4(m[0], m[1], m[2], m[3]);
+    __syncthreads();
+    if (tr == 0) {
+#pragma unroll
+        for (int i = 0; i < kRowSlices - 1; ++i) max_row(m, slice_max[i][tc]);
+    }
+    pdl_wait();                                // the zeroing kernel's writes are complete and visible
+    if (active && tr == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t v = (m[i] >> (16 * h)) & 0xFFFFu;
+                const int64_t j = col + 2 * i + h;
+                if (v != 0 && store_ok(j, 1, a.ext_amax, a.err, kSiteCalibAmax))
+                    atomicMax(a.out_bits[job] + j, v << 16);          // bf16 -> fp32 bits
+            }
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        is_last = 0u;
+        const int64_t ctr = band * kBandCols;
+        if (store_ok(ctr, 1, a.ext_lambda, a.err, kSiteCalibLambda)) {
+            const uint32_t prev = atomicAdd(reinterpret_cast<uint32_t*>(a.lambda + ctr), 1u);
+            const int64_t items = a.chunks[0] + a.chunks[1];
+            is_last = (static_cast<int64_t>(prev) == items - 1) ? 1u : 0u;
+        }
     }
     __syncthreads();
-    pdl_launch_dependents();                  // the quantiser's set-up may overlap this kernel
-
-    if (a.n_units == 0) {
-        // No rows selected and no weight: one CTA per strip forms lambda = 1.
-        pdl_wait();
-        if (warp < kConsumerWarps) strip_lambda(a, g);
-        return;
-    }
-    const int64_t u_begin = g * a.n_units / G;
-    const int64_t u_end = (g + 1) * a.n_units / G;
-    const int64_t skip = g == 0 ? a.skip_unit : -1;
-    const long long limit = skip >= 0 ? a.wait_limit : kWaitLimitCycles;
-
-    if (warp == kConsumerWarps) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            prefetch_tmap(&tmap_x);
-            if (a.units[1] > 0) prefetch_tmap(&tmap_w);
-            int i = 0;
-            for (int64_t u = u_begin; u < u_end; ++u, ++i) {
-                const int s = i % kSlots;
-                const uint32_t ph = (i / kSlots) & 1;
-                if (!mbar_wait_limit(&empty[s], ph ^ 1, abort_flag, a.err, kErrWaitEmpty, limit)) break;
-                if (i == skip) continue;              // time-out test: this unit never arrives
-                const int job = u < a.units[0] ? 0 : 1;
-                const int64_t local = job ? u - a.units[0] : u;
-                const int64_t strip = local / a.boxes[job];
-                const int64_t b = local % a.boxes[job];
-                int64_t row0, valid;
-                if (job == 0) {
-                    int seg = 0;
-                    while (seg + 1 < a.segs.n && b >= a.box_prefix[seg + 1]) ++seg;
-                    const int64_t in_seg = (b - a.box_prefix[seg]) * kBoxRows;
-                    row0 = a.segs.begin[seg] + in_seg;
-                    valid = min(static_cast<int64_t>(kBoxRows), a.segs.prefix[seg + 1] - a.segs.prefix[seg] - in_seg);
-                } else {
-                    row0 = b * kBoxRows;
-                    valid = min(static_cast<int64_t>(kBoxRows), a.N - row0);
-                }
-                meta[s] = (static_cast<uint32_t>(strip) << 8) | (static_cast<uint32_t>(job) << 7) |
-                          static_cast<uint32_t>(valid);
-                mbar_arrive_expect_tx(&full[s], kUnitBytes);
-                tma_load_2d(smem + s * kUnitBytes, job ? &tmap_w : &tmap_x, &full[s],
-                            static_cast<int32_t>(strip * kStripCols), static_cast<int32_t>(row0));
-            }
-            for (int j = (i > kSlots ? i - kSlots : 0); j < i; ++j) {   // bounded drain
-                if (j == skip) continue;
-                const long long t0 = clock64();
-                while (!mbar_try_wait(&full[j % kSlots], (j / kSlots) & 1) && clock64() - t0 < kWaitLimitCycles) {}
-            }
-        }
-        return;
-    }
-
-    // ---------------------------------------------------------------- consumers
-    pdl_wait();                               // the zeroing kernel's writes are complete and visible
-    uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
-    int64_t cur = -1;                          // (strip << 1) | matrix of the running maxima
-    auto merge = [&](int64_t key) {
-        const int job = static_cast<int>(key & 1);
-        const int64_t strip = key >> 1;
-        red[warp][lane][0] = m0;
-        red[warp][lane][1] = m1;
-        red[warp][lane][2] = m2;
-        red[warp][lane][3] = m3;
-        m0 = m1 = m2 = m3 = 0;
-        consumers_sync();
-        {
-            // thread t owns channel t of the strip
-            const int t = threadIdx.x;
-            const int src_lane = t / 8, word = (t % 8) / 2, hi = t & 1;
-            uint32_t m = 0;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) m = max(m, (red[w][src_lane][word] >> (16 * hi)) & 0xFFFFu);
-            const int64_t col = strip * kStripCols + t;
-            if (m != 0 && col < a.K && store_ok(col, 1, a.ext_amax, a.err, kSiteCalibAmax))
-                atomicMax(a.out_bits[job] + col, m << 16);   // bf16 -> fp32 bits
-        }
+    if (is_last) {
         __threadfence();
-        consumers_sync();
-        if (threadIdx.x == 0) {
-            is_last = 0u;
-            if (store_ok(strip * kStripCols, 1, a.ext_lambda, a.err, kSiteCalibLambda)) {
-                const uint32_t prev = atomicAdd(reinterpret_cast<uint32_t*>(a.lambda + strip * kStripCols), 1u);
-                is_last = (static_cast<int64_t>(prev) == strip_merges(a, strip, G) - 1) ? 1u : 0u;
-            }
-        }
-        consumers_sync();
-        if (is_last) {
-            __threadfence();
-            strip_lambda(a, strip);
-        }
-    };
-    int i = 0;
-    for (int64_t u = u_begin; u < u_end; ++u, ++i) {
-        const int s = i % kSlots;
-        const uint32_t ph = (i / kSlots) & 1;
-        if (!mbar_wait_limit(&full[s], ph, abort_flag, a.err, kErrWaitFull, limit)) break;
-        const uint32_t md = meta[s];
-        const int64_t key = (static_cast<int64_t>(md >> 8) << 1) | ((md >> 7) & 1);
-        const int valid = static_cast<int>(md & 0x7Fu);
-        if (key != cur) {                      // the same decision in every consumer warp
-            if (cur >= 0) merge(cur);
-            cur = key;
-        }
-        const uint8_t* tile = smem + s * kUnitBytes;
-#pragma unroll
-        for (int rr = 0; rr < kBoxRows / kConsumerWarps; ++rr) {
-            const int r = warp * (kBoxRows / kConsumerWarps) + rr;
-            if (r < valid) {
-                const uint4 q = *reinterpret_cast<const uint4*>(tile + r * (kStripCols * 2) + lane * 16);
-                m0 = __vmaxu2(m0, q.x & 0x7FFF7FFFu);
-                m1 = __vmaxu2(m1, q.y & 0x7FFF7FFFu);
-                m2 = __vmaxu2(m2, q.z & 0x7FFF7FFFu);
-                m3 = __vmaxu2(m3, q.w & 0x7FFF7FFFu);
-            }
-        }
-        consumed(m0, m1, m2, m3);                     // the unit's loads are in these maxima
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        band_lambda(a, band);
     }
-    if (cur >= 0) merge(cur);
 }
-
-// One-shot time-out test arming (see svdq_debug_arm_calib_timeout).
-std::atomic<long long> g_arm_skip{-1};
-std::atomic<long long> g_arm_limit{0};
-
-}  // namespace
-}  // namespace svdq
-
-extern "C" int svdq_debug_arm_calib_timeout(int64_t unit, int64_t wait_limit_cycles) {
-    if (unit < 0 || wait_limit_cycles < 100000) return SVDQ_ERR_INVALID_ARG;
-    svdq::g_arm_limit.store(wait_limit_cycles);
-    svdq::g_arm_skip.store(unit);
-    return SVDQ_OK;
-}
-
-namespace svdq {
-namespace {
 
 // Shared by both entry points.  W != NULL: the weight's absmax is reduced into
 // amax_w here.  W == NULL and aw_in != NULL: aw_in is the stored absmax of the
@@ -342,19 +264,30 @@ int calib_launch(const void* X, int64_t M, int64_t K, int64_t ldx, const svdq_se
     if (err == nullptr) return SVDQ_ERR_CUDA;
     const int64_t sms = device_sm_count() > 0 ? device_sm_count() : 148;
 
+    a.x = static_cast<const uint16_t*>(X);
+    a.ldx = ldx;
+    a.w = static_cast<const uint16_t*>(W);
+    a.ldw = ldw;
     a.K = K;
-    a.N = W != nullptr ? N : 0;
-    a.strips = (K + kStripCols - 1) / kStripCols;
-    a.box_prefix[0] = 0;
-    for (int s = 0; s < a.segs.n; ++s) {
-        const int64_t rows = a.segs.prefix[s + 1] - a.segs.prefix[s];
-        a.box_prefix[s + 1] = a.box_prefix[s] + (rows + kBoxRows - 1) / kBoxRows;
+    a.bands = (K + kBandCols - 1) / kBandCols;
+    a.rows[0] = a.segs.prefix[a.segs.n];
+    a.rows[1] = W != nullptr ? N : 0;
+    // Items (band x chunk): one wave of one CTA per SM (the chunks per band are
+    // the SMs over the bands, rounded down); chunks no shorter than the rows in
+    // flight.  With no rows at all, one empty chunk per band still forms lambda = 1.
+    const int64_t total_rows = a.rows[0] + a.rows[1];
+    const int64_t chunks_wanted = std::max<int64_t>(1, sms / a.bands);
+    // the two matrices' chunks round up separately: lengthen the chunks until
+    // their sum fits the wave
+    for (int64_t t = chunks_wanted; t >= 1; --t) {
+        a.chunk_rows = std::max<int64_t>(kRowsInFlight, (total_rows + t - 1) / t);
+        a.chunks[0] = (a.rows[0] + a.chunk_rows - 1) / a.chunk_rows;
+        a.chunks[1] = (a.rows[1] + a.chunk_rows - 1) / a.chunk_rows;
+        if (a.chunks[0] + a.chunks[1] <= chunks_wanted) break;
     }
-    a.boxes[0] = a.box_prefix[a.segs.n];
-    a.boxes[1] = (a.N + kBoxRows - 1) / kBoxRows;
-    a.units[0] = a.strips * a.boxes[0];
-    a.units[1] = a.strips * a.boxes[1];
-    a.n_units = a.units[0] + a.units[1];
+    if (a.chunks[0] + a.chunks[1] == 0) a.chunks[0] = 1;
+    const int64_t grid = a.bands * (a.chunks[0] + a.chunks[1]);
+    if (grid > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
     a.out_bits[0] = reinterpret_cast<uint32_t*>(amax_x);
     a.out_bits[1] = reinterpret_cast<uint32_t*>(amax_w);
     a.ax = amax_x;
@@ -365,19 +298,6 @@ int calib_launch(const void* X, int64_t M, int64_t K, int64_t ldx, const svdq_se
     a.err = err;
     a.ext_amax = debug_extent(kSiteCalibAmax, K);
     a.ext_lambda = debug_extent(kSiteCalibLambda, K);
-    a.skip_unit = g_arm_skip.exchange(-1);       // armed by the time-out test for this one call
-    a.wait_limit = a.skip_unit >= 0 ? g_arm_limit.load() : kWaitLimitCycles;
-    if (a.strips >= (int64_t(1) << 24)) return SVDQ_ERR_UNSUPPORTED;
-    const int64_t grid = a.n_units == 0 ? a.strips : (a.n_units < sms ? a.n_units : sms);
-
-    CUtensorMap tx, tw;
-    if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, K, M, ldx * 2, kStripCols, kBoxRows,
-                        CU_TENSOR_MAP_SWIZZLE_NONE))
-        return SVDQ_ERR_CUDA;
-    tw = tx;
-    if (W != nullptr && !encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, K, N, ldw * 2, kStripCols,
-                                        kBoxRows, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return SVDQ_ERR_CUDA;
 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const int64_t zb = (K + 255) / 256;
@@ -386,20 +306,17 @@ int calib_launch(const void* X, int64_t M, int64_t K, int64_t ldx, const svdq_se
         amax_x, W != nullptr ? amax_w : nullptr, K, lambda, s_g, debug_extent(kSiteCalibZero, K), err);
     st = launch_status(cudaGetLastError());
     if (st != SVDQ_OK) return st;
-    const uint32_t smem = kSmemBytes + 1024;
-    static std::atomic<uint64_t> smem_set{0};
-    if (!set_dynamic_smem_once(calib_stream_kernel, smem, smem_set)) return SVDQ_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = cs;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return launch_status(cudaLaunchKernelEx(&cfg, calib_stream_kernel, tx, tw, a));
+    return launch_status(cudaLaunchKernelEx(&cfg, calib_rows_kernel, a));
 }
 
 }  // namespace

@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict__ yr, int64_t N,
                     const __grid_constant__ ChunkPlan plan, int64_t n_chunks, double* __restrict__ partial,
                     double* __restrict__ num_out, double* __restrict__ den_out, double* __restrict__ rel_out,
-                    uint32_t* err, int64_t ext_part, int64_t ext_out) {
+                    uint32_t* err, int64_t ext_part, int64_t ext_out, int64_t skip_chunk, long long wait_limit) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStreamSlots * 2 * kChunkBytes);
     uint64_t* empty = full + kStreamSlots;
@@ -189,6 +189,11 @@ score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict_
     __shared__ double sh[kThreads / 32];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // Time-out test (armed from the host, one call): CTA 0's producer leaves its
+    // chunk number `skip_chunk` uncopied and the CTA's waits give up after
+    // `wait_limit` cycles; -1 = off.
+    const int64_t skip = blockIdx.x == 0 ? skip_chunk : -1;
+    const long long limit = skip >= 0 ? wait_limit : kWaitLimitCycles;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStreamSlots; ++s) {
             mbar_init(&full[s], 1);
@@ -207,7 +212,8 @@ score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict_
             for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++i) {
                 const int s = i % kStreamSlots;
                 const uint32_t ph = (i / kStreamSlots) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, err, kErrWaitEmpty)) break;
+                if (!mbar_wait_limit(&empty[s], ph ^ 1, abort_flag, err, kErrWaitEmpty, limit)) break;
+                if (i == skip) continue;              // time-out test: this chunk never arrives
                 while (seg + 1 < plan.n && c >= plan.chunk_prefix[seg + 1]) ++seg;   // c increases
                 const int64_t e0 = (c - plan.chunk_prefix[seg]) * kElemsPerChunk;
                 const int64_t e1 = min(e0 + kElemsPerChunk, plan.elems[seg]);
@@ -222,6 +228,7 @@ score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict_
                 }
             }
             for (int j = (i > kStreamSlots ? i - kStreamSlots : 0); j < i; ++j) {   // bounded drain
+                if (j == skip) continue;
                 const long long t0 = clock64();
                 while (!mbar_try_wait(&full[j % kStreamSlots], (j / kStreamSlots) & 1) &&
                        clock64() - t0 < kWaitLimitCycles) {}
@@ -233,7 +240,7 @@ score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict_
         for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++i) {
             const int s = i % kStreamSlots;
             const uint32_t ph = (i / kStreamSlots) & 1;
-            if (!mbar_wait(&full[s], ph, abort_flag, err, kErrWaitFull)) break;
+            if (!mbar_wait_limit(&full[s], ph, abort_flag, err, kErrWaitFull, limit)) break;
             const uint32_t n = n_elems[s];
             const uint8_t* qa = smem + s * 2 * kChunkBytes;
             const uint8_t* qb = qa + kChunkBytes;
@@ -293,6 +300,10 @@ score_stream_kernel(const uint16_t* __restrict__ yq, const uint16_t* __restrict_
 
 }  // namespace
 
+// One-shot time-out test arming (see svdq_debug_arm_score_timeout).
+std::atomic<long long> g_arm_skip{-1};
+std::atomic<long long> g_arm_limit{0};
+
 // Shared by the entry point below; `partial` must hold 2 doubles per chunk.
 int score_lambda_launch(const void* Yq, const void* Yref, int64_t M, int64_t N, int64_t ld,
                         const svdq_seg* segs, int n_seg, double* num, double* den, double* rel,
@@ -326,9 +337,11 @@ int score_lambda_launch(const void* Yq, const void* Yref, int64_t M, int64_t N, 
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
+        const int64_t skip = g_arm_skip.exchange(-1);     // armed by the time-out test for this one call
+        const long long limit = skip >= 0 ? g_arm_limit.load() : kWaitLimitCycles;
         return launch_status(cudaLaunchKernelEx(&cfg, score_stream_kernel, static_cast<const uint16_t*>(Yq),
                                                 static_cast<const uint16_t*>(Yref), N, plan, chunks, partial, num,
-                                                den, rel, err, ext_part, ext_out));
+                                                den, rel, err, ext_part, ext_out, skip, limit));
     } else {
         score_partial_kernel<<<static_cast<unsigned>(chunks), kThreads, 0, cs>>>(
             static_cast<const uint16_t*>(Yq), static_cast<const uint16_t*>(Yref), N, ld, plan, partial, ext_part, err);
@@ -362,6 +375,13 @@ size_t score_partial_bytes(const svdq_seg* segs, int n_seg, int64_t N) {
 }
 
 }  // namespace svdq
+
+extern "C" int svdq_debug_arm_score_timeout(int64_t chunk, int64_t wait_limit_cycles) {
+    if (chunk < 0 || wait_limit_cycles < 100000) return SVDQ_ERR_INVALID_ARG;
+    svdq::g_arm_limit.store(wait_limit_cycles);
+    svdq::g_arm_skip.store(chunk);
+    return SVDQ_OK;
+}
 
 extern "C" size_t svdq_score_workspace_bytes(const svdq_seg* segs, int n_seg, int64_t N) {
     const size_t b = svdq::score_partial_bytes(segs, n_seg, N);

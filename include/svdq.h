@@ -395,21 +395,22 @@ int svdq_bits_lost(const float* amax_x, int64_t ld_amax, int n_mod, const float*
 int svdq_device_error(void* stream, uint32_t* code);
 
 /*
- * svdq_debug_arm_calib_timeout -- test hook for the bounded waits (no page has
- * a counterpart).  Arms the next svdq_calib_lambda call in this process, on
- * whichever device it runs: in that call the first CTA's loader leaves its
- * ring unit number `unit` (0-based, within that CTA's range of 32-row x
- * 256-channel units) unloaded, and the CTA's waits give up after
- * `wait_limit_cycles` SM cycles instead of the usual ~2 s.  The consumer wait
- * for the missing unit therefore runs out: the kernel records code 1 ("a
- * consumer waited too long for a TMA stage") in the error word, stops its
- * other roles, waits for its own copies in flight and returns.  Nothing is
+ * svdq_debug_arm_score_timeout -- test hook for the bounded waits (no page has
+ * a counterpart).  Arms the next svdq_score_lambda (or _static) call in this
+ * process whose rows are stored back to back (ld == N, N % 8 == 0: the
+ * streaming kernel), on whichever device it runs: in that call the first CTA's
+ * loader leaves its chunk number `chunk` (0-based, within that CTA's chunks)
+ * uncopied, and the CTA's waits give up after `wait_limit_cycles` SM cycles
+ * instead of the usual ~2 s.  The consumer wait for the missing chunk therefore
+ * runs out: the kernel records code 1 ("a consumer waited too long for a TMA
+ * stage") in the error word, stops its other roles, waits for its own copies in
+ * flight, meets the other CTAs at the grid barrier and returns.  Nothing is
  * faulted and the context stays usable; that call's outputs are not valid.
- * One-shot: the following calls run normally.  Returns SVDQ_ERR_INVALID_ARG
- * for unit < 0 or a limit below 100000 cycles.  A unit at or past the CTA's
- * range arms nothing that call.
+ * One-shot: the following calls run normally.  Returns SVDQ_ERR_INVALID_ARG for
+ * chunk < 0 or a limit below 100000 cycles.  A chunk at or past the CTA's range
+ * arms nothing that call.
  */
-int svdq_debug_arm_calib_timeout(int64_t unit, int64_t wait_limit_cycles);
+int svdq_debug_arm_score_timeout(int64_t chunk, int64_t wait_limit_cycles);
 
 /*
  * The debug library.  libsvdq_debug.so is the same source compiled with
