@@ -9,24 +9,26 @@
 // "DeltaQuant on MiniMax-H3", section "The activation scale bound held": the
 // tensor scale is static and saturated groups are counted at run time.
 //
-// Work split: the rows are cut into G groups of R consecutive rows (R <= 128,
+// Work split: the rows are cut into G groups of R consecutive rows (R <= 112,
 // the last group shorter) and K into S slices of consecutive 64-channel chunks
 // (S <= 4, the CTAs of one thread-block cluster): one CTA per (group, slice).
 // R and S are chosen so that G * S comes close to the SM count (at most one
-// CTA fits per SM): 148 CTAs of 111 rows at 4096 rows (S = 4) and at 16384
-// rows (S = 1), 147 of 84 rows at 12288 rows.  Whole 128-row tiles would leave
-// 20 to 52 SMs without work at these sizes.  The partial D tiles of a cluster
-// are summed in cluster-rank order through distributed shared memory, so D is
-// deterministic.
+// CTA fits per SM): 148 CTAs of 111 rows at 4096 rows (S = 4), 147 of 112
+// rows at 16384 rows (S = 1), 147 of 84 rows at 12288 rows.  Whole 128-row
+// tiles would leave 20 to 52 SMs without work at these sizes.  The partial D
+// tiles of a cluster are summed in cluster-rank order through distributed
+// shared memory, so D is deterministic.
 //
-// Layout of one CTA (26 warps) over its group's rows and its slice of K:
-//   warp 24      TMA producer: R x 64 bf16 tiles of X (128-byte swizzle), the
+// Layout of one CTA (30 warps) over its group's rows and its slice of K:
+//   warp 28      TMA producer: R x 64 bf16 tiles of X (128-byte swizzle), the
 //                matching r x 64 tile of the down weight and 64 values of
-//                1/lambda into a 9-stage ring (a multiple of the 3 quantiser teams)
-//   warp 25      tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
+//                1/lambda into an 8-stage ring (a multiple of the 4 quantiser teams)
+//   warp 29      tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
 //                (M = 128: rows of a stage slot past R are never stored)
-//   warps 0..23  quantisers, in three teams of 8 that take the stages in
-//                turn; a lane owns one 16-channel group in each of two rows
+//   warps 0..27  quantisers, in four teams of 7 that take the stages in
+//                turn (the time per stage is set by how many stages are being
+//                quantised at once, not by the rows of a stage: four teams of
+//                112 rows beat three of 128); a lane owns one 16-channel group in each of two rows
 //                (two independent dependency chains), reads them from the
 //                swizzled tile, multiplies by 1/lambda and later by 1/S with
 //                packed f32x2 multiplies, forms the E4M3 scales of both rows
@@ -49,18 +51,25 @@ namespace {
 
 constexpr int kBM = 128;               // rows of a stage slot (the MMA's M); a group holds at most this many
 constexpr int kBK = 64;                // channels per stage (128 bytes of bf16)
-constexpr int kStages = 9;
-constexpr int kTeams = 3;             // teams of quantiser warps take stages in turn
-constexpr int kTeamWarps = 8;         // per stage: 16 rows x 4 groups of 16 channels per warp
-constexpr int kQuantWarps = kTeams * kTeamWarps;
+// Quantiser teams take the stages in turn; each warp of a team takes 16 rows
+// of a stage (4 groups of 16 channels).  Groups of up to 112 rows: four teams
+// of 7 warps over an 8-stage ring; of up to 128 rows: three teams of 8 over 9
+// stages (the host picks by the rows; a template parameter, so the ring and
+// team arithmetic stays constant).  The time per stage is set by how many
+// stages are being quantised at once, so the four-team shape is the faster one.
+constexpr int kStages = 9;            // ring slots laid out (the 4-team shape uses 8)
+constexpr int kQuantWarps = 28;
+constexpr int kGroupRows = 7 * 16;    // rows a group holds with four teams
 constexpr int kProducerWarp = kQuantWarps;
 constexpr int kMmaWarp = kQuantWarps + 1;
 constexpr int kThreads = (kQuantWarps + 2) * 32;
-// Stage i sits in slot i % kStages and is quantised by team i % kTeams.  A
+// Stage i sits in slot i % stages and is quantised by team i % teams.  A
 // parity wait only tells the current phase from the one before it, so a slot
-// must always be consumed by the same team: otherwise a team a whole ring lap
-// ahead could take the slot's unfinished phase for its own (completed) one.
-static_assert(kStages % kTeams == 0, "every slot is consumed by one team");
+// must always be consumed by the same team (stages is a multiple of teams):
+// otherwise a team a whole ring lap ahead could take the slot's unfinished
+// phase for its own (completed) one.
+static_assert(kStages % 3 == 0 && 8 <= kStages && 4 * 7 <= kQuantWarps && 3 * 8 <= kQuantWarps,
+              "both team shapes fit the warps and the ring");
 constexpr int kMaxSplit = 4;          // CTAs of a cluster along K
 constexpr uint32_t kXTileBytes = kBM * kBK * 2;  // 16 KB
 
@@ -123,11 +132,15 @@ __device__ __forceinline__ uint32_t scale_byte_checked(float a, float d, float r
     return cvt_e4m3x2(t, 0.0f) & 0xFFu;
 }
 
-template <int R>
+template <int R, int kTeamWarps>
 __global__ void __launch_bounds__(kThreads)
 quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_down,
                     QuantArgs args) {
     using L = QSmem<R>;
+    static_assert(kTeamWarps == 7 || kTeamWarps == 8, "the two team shapes");
+    constexpr int kTeams = kQuantWarps / kTeamWarps;                 // 4 or 3
+    constexpr int kStagesT = kTeamWarps == 7 ? 8 : 9;                // a multiple of the teams
+    static_assert(kStagesT % kTeams == 0 && kStagesT <= kStages, "every slot is consumed by one team");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
@@ -150,7 +163,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
     const int n_local = c_end - c_begin;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kStagesT; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kTeamWarps + (R > 0 ? 1 : 0));
         }
@@ -176,8 +189,8 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
             const uint32_t x_bytes = static_cast<uint32_t>(args.rows) * kBK * 2;
             int issued = 0;
             for (int i = 0; i < n_local; ++i) {
-                const int s = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
+                const int s = i % kStagesT;
+                const uint32_t ph = (i / kStagesT) & 1;
                 if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, args.err, kErrWaitEmpty)) break;
                 const int col = (c_begin + i) * kBK;
                 mbar_arrive_expect_tx(&full[s], x_bytes + L::kDownTileBytes + (args.inv_lambda ? kBK * 4 : 0));
@@ -190,17 +203,18 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 ++issued;
             }
             // Wait (bounded) for the copies still in flight before the CTA may exit.
-            for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i) {
+            for (int i = (issued > kStagesT ? issued - kStagesT : 0); i < issued; ++i) {
                 const long long t0 = clock64();
-                while (!mbar_try_wait(&full[i % kStages], (i / kStages) & 1) && clock64() - t0 < kWaitLimitCycles) {}
+                while (!mbar_try_wait(&full[i % kStagesT], (i / kStagesT) & 1) &&
+                       clock64() - t0 < kWaitLimitCycles) {}
             }
         }
     } else if (warp == kMmaWarp) {
         if (R > 0 && lane == 0) {
             const uint32_t idesc = idesc_bf16(kBM, R);
             for (int i = 0; i < n_local; ++i) {
-                const int s = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
+                const int s = i % kStagesT;
+                const uint32_t ph = (i / kStagesT) & 1;
                 if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(smem + L::kXOff + s * kXTileBytes);
@@ -237,7 +251,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         // of the tile, channels 16 b .. 16 b + 15 of the stage; the group's two
         // 16-byte halves are chunks 2b and 2b+1 of the row's 128-byte line
         // (both rows have the same swizzle phase, r0 % 8 == (r0 + 8) % 8).
-        const int team = warp / kTeamWarps;
+        const int team = warp / kTeamWarps;      // >= teams: a spare warp, no stages
         const int rw = lane >> 2;
         const int b = lane & 3;
         const int r0 = (warp % kTeamWarps) * 16 + rw;
@@ -254,9 +268,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         // quantise: it only keeps the ring's protocol (wait for each of its
         // team's stages, release it), so the work per stage follows the rows.
         const bool idle = (warp % kTeamWarps) * 16 >= box_rows;
-        for (int i = team; i < n_local; i += kTeams) {
-            const int s = i % kStages;
-            const uint32_t ph = (i / kStages) & 1;
+        for (int i = team < kTeams ? team : n_local; i < n_local; i += kTeams) {
+            const int s = i % kStagesT;
+            const uint32_t ph = (i / kStagesT) & 1;
             if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
             if (idle) {
                 __syncwarp();
@@ -483,9 +497,13 @@ int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const Quan
     a.n_chunks = static_cast<int>(K / kBK);
     const int64_t sms = device_sm_count() > 0 ? device_sm_count() : 148;
     const uint32_t smem = QSmem<R>::kBytes + 1024;
-    auto kern = quantize_act_kernel<R>;
-    static std::atomic<uint64_t> smem_set{0};
-    if (!set_dynamic_smem_once(kern, smem, smem_set)) return SVDQ_ERR_CUDA;
+    // both team shapes: the same threads and shared memory (the ring is laid out
+    // for 9 stages), so the cluster occupancy below holds for either
+    auto kern4 = quantize_act_kernel<R, 7>;
+    auto kern3 = quantize_act_kernel<R, 8>;
+    static std::atomic<uint64_t> smem_set4{0}, smem_set3{0};
+    if (!set_dynamic_smem_once(kern4, smem, smem_set4) || !set_dynamic_smem_once(kern3, smem, smem_set3))
+        return SVDQ_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
@@ -503,12 +521,13 @@ int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const Quan
         cfg.gridDim = dim3(1, kMaxSplit, 1);
         attr[0].val.clusterDim.y = kMaxSplit;
         cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess) max_clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, kern3, &cfg) != cudaSuccess) max_clusters = 0;
     }
     const QuantPlan plan = plan_quantize(M, a.n_chunks, sms, max_clusters);
     if (plan.groups > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED;
     a.split = plan.split;
     a.rows = plan.rows;
+
     CUtensorMap tx, td;
     if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, K, M, ldx * 2, kBK,
                         static_cast<uint32_t>(plan.rows), CU_TENSOR_MAP_SWIZZLE_128B))
@@ -524,7 +543,8 @@ int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const Quan
     cfg.gridDim = dim3(static_cast<unsigned>(plan.groups), static_cast<unsigned>(plan.split), 1);
     attr[0].val.clusterDim.y = (R > 0) ? plan.split : 1;
     cfg.numAttrs = 2;
-    return launch_status(cudaLaunchKernelEx(&cfg, kern, tx, td, a));
+    return launch_status(plan.rows <= kGroupRows ? cudaLaunchKernelEx(&cfg, kern4, tx, td, a)
+                                                 : cudaLaunchKernelEx(&cfg, kern3, tx, td, a));
 }
 
 }  // namespace
