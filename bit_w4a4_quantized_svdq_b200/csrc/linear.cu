@@ -525,9 +525,12 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------------ block-scale writers
         // Each warp copies the stage's scale atoms from the shared-memory ring
-        // into its own tensor-memory lane quarter with tcgen05.st (every quarter
-        // holds the full set, the layout the block-scaled MMA reads), then
-        // arrives on the stage's barrier.  Unlike a shared->tensor copy issued by
+        // into its own tensor-memory lane quarter with tcgen05.st, then arrives
+        // on the stage's barrier.  The block-scaled MMA of lane quarter q reads
+        // the W scales of all 256 columns (so every quarter holds all of them)
+        // and, of the four A-scale columns of an MMA (rows 32 j + lane in column
+        // j), only column q: each writer stores just that one (the same output
+        // bit for bit as storing all four).  Unlike a shared->tensor copy issued by
         // the MMA thread, these stores run alongside the MMAs instead of in front
         // of them.  Ring slot: released after the stores of its last stage.
         // Tensor-memory buffer s: written only after the MMAs of its previous
@@ -555,7 +558,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                 // buffer: A scales of MMA kk at 4 kk + (row / 32); W scales of MMA
                 // kk at 16 + 8 kk + (row / 32), rows 128..255 at + 4.  Lane i reads
                 // row i of each 512-byte atom: its 4 words are the 4 columns.
-                uint32_t ra[kMx ? 4 : 16], rb[kMx ? 8 : 32];
+                uint32_t ra[4], rb[kMx ? 8 : 32];
                 if constexpr (kMx) {
                     // MXFP8: the stage's one A atom and one W atom per 128-row block
                     // (slot layout: A [2 stages][512], then W [2 row blocks][2 stages][512]).
@@ -572,10 +575,10 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                     const uint8_t* sfb = smem + L::kOffSf + slot * kSfSlot + kSfaPair + (kb & 1) * 2048;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint4 a = *reinterpret_cast<const uint4*>(sfa + q * 512 + lane * 16);
+                        // A: only this lane quarter's rows (word `warp & 3` of the lane's 16 bytes)
+                        ra[q] = *reinterpret_cast<const uint32_t*>(sfa + q * 512 + lane * 16 + (warp & 3) * 4);
                         const uint4 x = *reinterpret_cast<const uint4*>(sfb + q * 512 + lane * 16);
                         const uint4 y = *reinterpret_cast<const uint4*>(sfb + 4096 + q * 512 + lane * 16);
-                        ra[4 * q] = a.x; ra[4 * q + 1] = a.y; ra[4 * q + 2] = a.z; ra[4 * q + 3] = a.w;
                         rb[8 * q] = x.x; rb[8 * q + 1] = x.y; rb[8 * q + 2] = x.z; rb[8 * q + 3] = x.w;
                         rb[8 * q + 4] = y.x; rb[8 * q + 5] = y.y; rb[8 * q + 6] = y.z; rb[8 * q + 7] = y.w;
                     }
@@ -592,7 +595,11 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
                                             rb[4], rb[5], rb[6], rb[7], 0u, 0u, 0u, 0u};
                     tmem_st_32x32b_x16(base, r);
                 } else {
-                    tmem_st_32x32b_x16(base, ra);
+                    // A scales of MMA kk sit in columns 4 kk .. 4 kk + 3 (rows 32 j + lane in
+                    // column 4 kk + j); lane quarter q reads only column 4 kk + q, so each
+                    // writer stores that one.  W scales: all 32 columns in every quarter.
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) tmem_st_32x32b_x1(base + 4 * q + (warp & 3), ra[q]);
                     tmem_st_32x32b_x32(base + kTmemSfbOff, rb);
                 }
                 tmem_st_wait();

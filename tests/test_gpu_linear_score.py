@@ -132,6 +132,25 @@ def test_repeatable_many_tiles(lib):
     assert lib.svdq_device_error() == 0
 
 
+@pytest.mark.parametrize("k", [256, 512])
+def test_plain_linear_repeatable_many_tiles(lib, k):
+    """The plain linear, bf16 and fp32 output, at one and two 256-channel stages
+    per tile (ring slots and scale slots reused at the fastest rate): twenty
+    calls are bitwise equal.  A ring slot released while loads from it are still
+    in flight shows up here as a 32-row block of one call that differs."""
+    m, n, r = 5120, 5120, 32
+    x = S.random_bf16((m, k), 41, 1.0)
+    w = S.random_bf16((n, k), 42, 0.02)
+    args = _operands(lib, x, w, S.random_bf16((n,), 43, 0.1), r)
+    for out_dtype in (torch.bfloat16, torch.float32):
+        y0 = lib.svdq_linear(*args, out_dtype=out_dtype)
+        for _ in range(20):
+            y = lib.svdq_linear(*args, out_dtype=out_dtype)
+            assert torch.equal(y.view(torch.int32 if out_dtype == torch.float32 else torch.int16),
+                               y0.view(torch.int32 if out_dtype == torch.float32 else torch.int16))
+    assert lib.svdq_device_error() == 0
+
+
 def test_rejects_bad_arguments(lib):
     m, n, k = 128, 256, 256
     x = S.random_bf16((m, k), 21, 1.0)

@@ -92,3 +92,17 @@ def test_linear_large_sampled(lib):
     np.testing.assert_array_equal(qa["codes"].cpu().numpy()[rows], a_c)
     check_linear_bf16(host_bits(y)[rows], O.mx_linear(a_c, a_s, w_c, w_s, L.bias))
     assert lib.svdq_device_error() == 0
+
+
+def test_linear_repeatable_many_tiles(lib):
+    """One 128-channel stage per tile (ring and scale slots reused at the fastest
+    rate), many tiles per CTA: twenty calls are bitwise equal."""
+    m, n, k = 5120, 5120, 128
+    qa = lib.svdq_quantize_mxfp8(dev_bits(_x(m, k, 51)))
+    qw = lib.svdq_quantize_mxfp8(dev_bits(S.random_bf16((n, k), 52, 0.02)))
+    bias = dev_bits(S.random_bf16((n,), 53, 0.02))
+    y0 = lib.svdq_linear_mxfp8(qa["codes"], qa["sf"], qw["codes"], qw["sf"], bias)
+    for _ in range(20):
+        y = lib.svdq_linear_mxfp8(qa["codes"], qa["sf"], qw["codes"], qw["sf"], bias)
+        assert torch.equal(y.view(torch.int16), y0.view(torch.int16))
+    assert lib.svdq_device_error() == 0
