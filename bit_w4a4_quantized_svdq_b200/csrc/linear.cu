@@ -359,8 +359,6 @@ linear_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant_
     // the stage's four MMAs of K = 32 (scale ids 0..3).
     constexpr int kStageK = kMx ? 128 : kBK;
     constexpr uint32_t kSfaPairT = kMx ? 1024 : kSfaPair;          // A scale bytes of two stages
-    constexpr uint32_t kSfSlotT = kMx ? 3072 : kSfSlot;            // A + W scale bytes of two stages
-    constexpr int kSfHalvesPerStage = kMx ? 2 : 8;                  // 256-byte scale pieces per row block
     constexpr uint32_t kTmemSfStrideT = kMx ? 16 : kTmemSfStride;
     constexpr uint32_t kTmemSfbOffT = kMx ? 4 : kTmemSfbOff;
     // a last partial stage reads zero codes and zero scales past K (TMA fill): it adds nothing
