@@ -17,12 +17,15 @@
 // rows at 16384 rows (S = 1), 147 of 84 rows at 12288 rows.  Whole 128-row
 // tiles would leave 20 to 52 SMs without work at these sizes.  The partial D
 // tiles of a cluster are summed in cluster-rank order through distributed
-// shared memory, so D is deterministic.
+// shared memory, so D is deterministic.  Without a split along K (S = 1) the
+// CTA needs no D partial in shared memory: its room goes to a deeper ring of
+// 12 stages of 112-row slots, and D goes from tensor memory to global memory.
 //
 // Layout of one CTA (30 warps) over its group's rows and its slice of K:
 //   warp 28      TMA producer: R x 64 bf16 tiles of X (128-byte swizzle), the
 //                matching r x 64 tile of the down weight and 64 values of
-//                1/lambda into an 8-stage ring (a multiple of the 4 quantiser teams)
+//                1/lambda into an 8-stage ring, or the 12-stage one without a
+//                split (a multiple of the 4 quantiser teams)
 //   warp 29      tcgen05 issuer: D_partial(tmem, fp32) += X_tile * down_tile^T
 //                (M = 128: rows of a stage slot past R are never stored)
 //   warps 0..27  quantisers, in four teams of 7 that take the stages in
@@ -38,7 +41,7 @@
 //                non-negative E4M3 bytes (S = RN(dec(byte) * s_g), 1/S = RN(1/S)),
 //                built once at CTA start;
 //                warps 0..3 (one per tensor-memory lane quarter) finally read
-//                D_partial from tensor memory.
+//                D_partial from tensor memory (and, without a split, store it).
 // The kernel is a programmatic dependent of the one before it in the stream:
 // barrier set-up, tensor-memory allocation and the tensor-map prefetch run
 // before griddepcontrol.wait, and it lets its own dependent (the linear) start
@@ -56,7 +59,8 @@ constexpr int kBK = 64;                // channels per stage (128 bytes of bf16)
 // of 7 warps over an 8-stage ring; of up to 128 rows: three teams of 8 over 9
 // stages (the host picks by the rows; a template parameter, so the ring and
 // team arithmetic stays constant).  The time per stage is set by how many
-// stages are being quantised at once, so the four-team shape is the faster one.
+// stages are being quantised at once, so the four-team shape is the faster one,
+// and the deep ring (12 stages, no split) faster still: more stages in flight.
 constexpr int kStages = 9;            // ring slots laid out (the 4-team shape uses 8)
 constexpr int kQuantWarps = 28;
 constexpr int kGroupRows = 7 * 16;    // rows a group holds with four teams
@@ -71,20 +75,38 @@ constexpr int kThreads = (kQuantWarps + 2) * 32;
 static_assert(kStages % 3 == 0 && 8 <= kStages && 4 * 7 <= kQuantWarps && 3 * 8 <= kQuantWarps,
               "both team shapes fit the warps and the ring");
 constexpr int kMaxSplit = 4;          // CTAs of a cluster along K
-constexpr uint32_t kXTileBytes = kBM * kBK * 2;  // 16 KB
+constexpr int kDeepStages = 12;       // the deep ring: groups of <= 112 rows, no split along K
 
-template <int R>
+// Shared-memory layout: kNumStages slots of kSlotRows x 64 bf16 of X (the MMA
+// reads 128 rows from a slot; rows past the group's are never stored, and a
+// 112-row slot's last ones lie in the next slot or, for the last slot, in the
+// down tiles: in bounds either way), the matching down tiles, the D partial
+// when a cluster sums D along K (kPart), 1/lambda per stage, the 1/S table and
+// the barriers.
+template <int R, int kSlotRows, int kNumStages, bool kPart>
 struct QSmem {
+    static constexpr uint32_t kXTile = kSlotRows * kBK * 2;                        // 16 or 14 KB (1 KB multiples)
+    static constexpr int kStagesL = kNumStages;
     static constexpr uint32_t kDownTileBytes = R * kBK * 2;
     static constexpr uint32_t kXOff = 0;
-    static constexpr uint32_t kDownOff = kStages * kXTileBytes;
+    static constexpr uint32_t kDownOff = kNumStages * kXTile;
     static constexpr uint32_t kPartStride = R + 4;                                 // floats per row (padded)
-    static constexpr uint32_t kPartOff = kDownOff + kStages * kDownTileBytes;     // D partial [128][R + 4] fp32
-    static constexpr uint32_t kIlamOff = kPartOff + (R > 0 ? kBM * kPartStride * 4 : 0);   // 1/lambda, 64 fp32 per stage
-    static constexpr uint32_t kTabOff = kIlamOff + kStages * kBK * 4;              // 1/S per E4M3 byte, 128 fp32
-    static constexpr uint32_t kBarOff = kTabOff + 128 * 4;
+    static constexpr uint32_t kPartOff = kDownOff + kNumStages * kDownTileBytes;  // D partial [128][R + 4] fp32
+    static constexpr uint32_t kIlamOff = kPartOff + (kPart && R > 0 ? kBM * kPartStride * 4 : 0);   // 1/lambda, 64 fp32 per stage
+    static constexpr uint32_t kTabOff = kIlamOff + kNumStages * kBK * 4;           // 1/S per E4M3 byte, 128 fp32
+    static constexpr uint32_t kBarOff = kTabOff + 128 * 4;                         // full, empty [kNumStages], dfull, ...
     static constexpr uint32_t kBytes = kBarOff + 256;
+    static_assert(kXTile % 1024 == 0, "slots keep the 128-byte swizzle's 1 KB alignment");
+    static_assert(2 * kNumStages * 8 + 24 <= 256, "the barriers fit their area");
+    static_assert(kBytes + 1024 <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
 };
+
+// The three shapes: kTeamWarps = 8 (three teams, 9 stages of 128-row slots);
+// kTeamWarps = 7 (four teams, 8 of the 9 laid-out stages); kDeep (four teams of 7
+// over 12 stages of 112-row slots, no D partial in shared memory: D goes from
+// tensor memory straight to global memory, so only without a split along K).
+template <int R, int kTeamWarps, bool kDeep>
+using QLayout = QSmem<R, kDeep ? kGroupRows : kBM, kDeep ? kDeepStages : kStages, !kDeep>;
 
 struct QuantArgs {
     const float* inv_lambda;
@@ -132,20 +154,21 @@ __device__ __forceinline__ uint32_t scale_byte_checked(float a, float d, float r
     return cvt_e4m3x2(t, 0.0f) & 0xFFu;
 }
 
-template <int R, int kTeamWarps>
+template <int R, int kTeamWarps, bool kDeep>
 __global__ void __launch_bounds__(kThreads)
 quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_down,
                     QuantArgs args) {
-    using L = QSmem<R>;
+    using L = QLayout<R, kTeamWarps, kDeep>;
     static_assert(kTeamWarps == 7 || kTeamWarps == 8, "the two team shapes");
+    static_assert(!kDeep || kTeamWarps == 7, "the deep ring is laid out for 112-row groups");
     constexpr int kTeams = kQuantWarps / kTeamWarps;                 // 4 or 3
-    constexpr int kStagesT = kTeamWarps == 7 ? 8 : 9;                // a multiple of the teams
-    static_assert(kStagesT % kTeams == 0 && kStagesT <= kStages, "every slot is consumed by one team");
+    constexpr int kStagesT = kDeep ? kDeepStages : (kTeamWarps == 7 ? 8 : 9);   // a multiple of the teams
+    static_assert(kStagesT % kTeams == 0 && kStagesT <= L::kStagesL, "every slot is consumed by one team");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-    uint64_t* empty = full + kStages;
-    uint64_t* dfull = empty + kStages;
+    uint64_t* empty = full + L::kStagesL;
+    uint64_t* dfull = empty + L::kStagesL;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dfull + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -196,7 +219,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 mbar_arrive_expect_tx(&full[s], x_bytes + L::kDownTileBytes + (args.inv_lambda ? kBK * 4 : 0));
                 if (args.inv_lambda)
                     bulk_load(smem + L::kIlamOff + s * kBK * 4, args.inv_lambda + col, kBK * 4, &full[s]);
-                tma_load_2d(smem + L::kXOff + s * kXTileBytes, &tmap_x, &full[s], col,
+                tma_load_2d(smem + L::kXOff + s * L::kXTile, &tmap_x, &full[s], col,
                             static_cast<int32_t>(row_base));
                 if (R > 0)
                     tma_load_2d(smem + L::kDownOff + s * L::kDownTileBytes, &tmap_down, &full[s], col, 0);
@@ -217,7 +240,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 const uint32_t ph = (i / kStagesT) & 1;
                 if (!mbar_wait(&full[s], ph, abort_flag, args.err, kErrWaitFull)) break;
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(smem + L::kXOff + s * kXTileBytes);
+                const uint32_t a0 = smem_u32(smem + L::kXOff + s * L::kXTile);
                 const uint32_t b0 = smem_u32(smem + L::kDownOff + s * L::kDownTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk)
@@ -278,7 +301,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
                 continue;
             }
             const int chunk = c_begin + i;
-            const uint8_t* tile = smem + L::kXOff + s * kXTileBytes;
+            const uint8_t* tile = smem + L::kXOff + s * L::kXTile;
             const uint4 u0 = *reinterpret_cast<const uint4*>(tile + r0 * 128 + ph0);
             const uint4 u1 = *reinterpret_cast<const uint4*>(tile + r0 * 128 + ph1);
             const uint4 v0 = *reinterpret_cast<const uint4*>(tile + (r0 + 8) * 128 + ph0);
@@ -366,7 +389,30 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         for (int o = 16; o > 0; o >>= 1) sat += __shfl_xor_sync(0xffffffffu, sat, o);
         if (lane == 0 && sat && args.sat_count) atomicAdd(args.sat_count, sat);
 
-        if (R > 0 && warp < 4) {   // one warp per tensor-memory lane quarter
+        if (kDeep && R > 0 && warp < 4) {
+            // No split along K: this CTA's D rows go from tensor memory straight to
+            // global memory (one warp per lane quarter, a thread per row).
+            const int row = warp * 32 + lane;
+            const int64_t grow = row_base + row;
+            const bool row_ok = row < args.rows && grow < args.M;
+            if (mbar_wait(dfull, 0, abort_flag, args.err, kErrWaitMma)) {
+                tc_fence_after();
+                const uint32_t taddr = tmem_d + (static_cast<uint32_t>(warp * 32) << 16);
+                uint32_t v[R > 16 ? 32 : 16];
+                if constexpr (R == 32) tmem_ld_32x32b_x32(taddr, v);
+                else tmem_ld_32x32b_x16(taddr, v);
+                tmem_ld_wait(v);
+                if (row_ok) {
+                    float4* dst = reinterpret_cast<float4*>(args.D + grow * R);
+#pragma unroll
+                    for (int q = 0; q < R / 4; ++q)
+                        if (store_ok(grow * R + 4 * q, 4, args.ext_d, args.err, kSiteQuantD))
+                            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                 __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+                }
+            }
+            tc_fence_before();
+        } else if (R > 0 && warp < 4) {   // one warp per tensor-memory lane quarter
             float* part = reinterpret_cast<float*>(smem + L::kPartOff) + (warp * 32 + lane) * L::kPartStride;
             if (mbar_wait(dfull, 0, abort_flag, args.err, kErrWaitMma)) {
                 tc_fence_after();
@@ -405,7 +451,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_con
         // issues all its 16-byte loads from the peers' shared memory first and
         // then adds them, so the loads' latencies overlap.
         cluster_sync_all();
-        if (warp < 4) {
+        if (!kDeep && warp < 4) {
             constexpr int kNq = R / 4;                           // float4 groups per row
             constexpr int kMaxQ = (kNq + 1) / 2 + 1;             // groups one CTA takes (split >= 2), or all
             const int split = args.split;
@@ -496,13 +542,17 @@ int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const Quan
     QuantArgs a = base;
     a.n_chunks = static_cast<int>(K / kBK);
     const int64_t sms = device_sm_count() > 0 ? device_sm_count() : 148;
-    const uint32_t smem = QSmem<R>::kBytes + 1024;
-    // both team shapes: the same threads and shared memory (the ring is laid out
-    // for 9 stages), so the cluster occupancy below holds for either
-    auto kern4 = quantize_act_kernel<R, 7>;
-    auto kern3 = quantize_act_kernel<R, 8>;
-    static std::atomic<uint64_t> smem_set4{0}, smem_set3{0};
-    if (!set_dynamic_smem_once(kern4, smem, smem_set4) || !set_dynamic_smem_once(kern3, smem, smem_set3))
+    // The three-team and the four-team shape share threads and shared memory
+    // (the ring is laid out for 9 stages), so the cluster occupancy below holds
+    // for either; the deep shape runs without clusters.
+    const uint32_t smem = QLayout<R, 8, false>::kBytes + 1024;
+    const uint32_t smem_deep = QLayout<R, 7, true>::kBytes + 1024;
+    auto kern4 = quantize_act_kernel<R, 7, false>;
+    auto kern3 = quantize_act_kernel<R, 8, false>;
+    auto kern_deep = quantize_act_kernel<R, 7, true>;
+    static std::atomic<uint64_t> smem_set4{0}, smem_set3{0}, smem_set_deep{0};
+    if (!set_dynamic_smem_once(kern4, smem, smem_set4) || !set_dynamic_smem_once(kern3, smem, smem_set3) ||
+        !set_dynamic_smem_once(kern_deep, smem_deep, smem_set_deep))
         return SVDQ_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -543,6 +593,11 @@ int launch_quantize(const void* X, int64_t M, int64_t K, int64_t ldx, const Quan
     cfg.gridDim = dim3(static_cast<unsigned>(plan.groups), static_cast<unsigned>(plan.split), 1);
     attr[0].val.clusterDim.y = (R > 0) ? plan.split : 1;
     cfg.numAttrs = 2;
+    // groups of up to 112 rows whose D needs no sum across a cluster: the deep ring
+    if (plan.rows <= kGroupRows && (R == 0 || plan.split == 1)) {
+        cfg.dynamicSmemBytes = smem_deep;
+        return launch_status(cudaLaunchKernelEx(&cfg, kern_deep, tx, td, a));
+    }
     return launch_status(plan.rows <= kGroupRows ? cudaLaunchKernelEx(&cfg, kern4, tx, td, a)
                                                  : cudaLaunchKernelEx(&cfg, kern3, tx, td, a));
 }
