@@ -52,7 +52,7 @@ FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (
 # ncu capture of the current kernel (summaries under profiles/); None until the
 # current kernel has been captured on that workload.
 LINEAR_TRAFFIC_BYTES = {3: 496.65e6 + 155.86e6}
-QUANTIZE_TRAFFIC_BYTES: dict = {}
+QUANTIZE_TRAFFIC_BYTES = {3: 673.66e6 + 171.37e6}
 # Our kernels per step: calib (zeroing + stream), quantize, linear, score (one
 # cooperative kernel when rows are back to back).
 LAUNCHES_PER_STEP = 5
