@@ -13,9 +13,10 @@
 // the last group shorter) and K into S slices of consecutive 64-channel chunks
 // (S <= 4, the CTAs of one thread-block cluster): one CTA per (group, slice).
 // R and S are chosen so that G * S comes close to the SM count (at most one
-// CTA fits per SM): 148 CTAs of 111 rows at 4096 rows (S = 4), 147 of 112
-// rows at 16384 rows (S = 1), 147 of 84 rows at 12288 rows.  Whole 128-row
-// tiles would leave 20 to 52 SMs without work at these sizes.  The partial D
+// CTA fits per SM), with no more clusters than fit at once: 128 CTAs of 128
+// rows at 4096 rows (S = 4: 32 clusters of 4 fit, 37 do not), 147 of 112 rows
+// at 16384 rows (S = 1), 140 of 88 rows at 12288 rows.  Whole 128-row tiles
+// would leave 20 to 52 SMs without work at the larger sizes.  The partial D
 // tiles of a cluster are summed in cluster-rank order through distributed
 // shared memory, so D is deterministic.  Without a split along K (S = 1) the
 // CTA needs no D partial in shared memory: its room goes to a deeper ring of
