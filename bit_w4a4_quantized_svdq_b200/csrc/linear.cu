@@ -37,10 +37,11 @@
 //         the operand copies never queue behind them
 // Instantiations (linear_kernel<out fp32, score, MXFP8>):
 //   <0|1, 0, 0>  svdq_linear: the NVFP4 linear, bf16 or fp32 output
-//   <0, 1, 0>    svdq_linear_score: the same, with the tile scored against a bf16
-//                reference in the epilogue (reference strips by TMA into the low-rank
-//                area, per-row exact fp32 pair sums, per-segment fp64 sums, a grid
-//                barrier and a final sum in CTA order); writing Y is optional
+//   <0, 1, 0>    svdq_linear_score: the same over a three-stage ring, with the tile
+//                scored against a bf16 reference in the epilogue (reference strips by
+//                TMA into a 48 KB epilogue area, per-row exact fp32 pair sums,
+//                per-segment fp64 sums, a grid barrier and a final sum in CTA order);
+//                writing Y is optional
 //   <0, 0, 1>    svdq_linear_mxfp8: E4M3 operands with E8M0 scales per 32 on
 //                kind::mxf8f6f4 MMAs; 128 channels per stage, one scale atom per 128
 //                rows per stage serving its four K = 32 MMAs through the scale ids;

@@ -5,10 +5,14 @@
 // rows per modality).
 //
 // Bandwidth-bound two-pass reduction with a fixed order, so results are
-// bitwise reproducible: pass 1 gives every (segment, row chunk) one block that
-// writes fp64 partial sums to the caller's workspace (8 independent 16-byte
-// loads per thread and input in flight); pass 2 sums each
-// segment's partials in index order and forms num, den and rel.
+// bitwise reproducible: pass 1 writes one fp64 partial sum per (segment,
+// 16384-element chunk) to the caller's workspace; pass 2 sums each segment's
+// partials in index order and forms num, den and rel.  Pass 1 has two forms
+// that reduce a chunk with the same thread mapping and tree, so they agree bit
+// for bit: rows stored back to back stream through persistent CTAs (a producer
+// warp bulk-copies whole chunks into a shared-memory ring, eight consumer warps
+// reduce them, a grid barrier, then the final sums); strided rows take one block
+// per chunk with 8 independent 16-byte loads per thread and input in flight.
 #include <mutex>
 
 #include <cooperative_groups.h>
