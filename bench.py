@@ -197,9 +197,11 @@ def run_reference(args):
     cfg = args.config
     layer = S.make_layer(cfg)
     arm = OracleArm(layer)
+    # W untimed warm-up steps on the timed sample (a step costs ~2 s on 16 host
+    # threads, most of it the oracle reading and dequantising the whole weight)
     rows = min(layer.m, 128)
-    for _ in range(min(args.warmup, 1)):
-        arm.run(8)
+    for _ in range(args.warmup):
+        arm.run(rows)
     times, vals = [], []
     for _ in range(args.steps):
         v, dt, rows = arm.run(rows)
