@@ -373,6 +373,30 @@ def test_score_identities():
     assert np.array_equal(n2[::-1], num) and np.array_equal(d2[::-1], den)
 
 
+def test_score_closed_form_per_segment():
+    # Yref = 1 everywhere; segment s adds d_s to every element of its rows (exact in
+    # bf16), so num_s = rows_s * N * d_s^2, den_s = rows_s * N and rel_s = d_s.  A
+    # segment that took a row of its neighbour, or lost one, changes its sums.
+    n = 8
+    segs = [(0, 3), (3, 7), (7, 12), (12, 12)]
+    d = [0.5, 0.25, 2.0]
+    yref = np.ones((12, n), np.float32)
+    yq = yref.copy()
+    for (b, e), ds in zip(segs, d):
+        yq[b:e] += np.float32(ds)
+    num, den, rel = O.score(S.f32_to_bf16_bits(yq), S.f32_to_bf16_bits(yref), segs)
+    rows = [e - b for b, e in segs[:3]]
+    assert num[:3].tolist() == [r * n * ds * ds for r, ds in zip(rows, d)]
+    assert den[:3].tolist() == [float(r * n) for r in rows]
+    assert rel[:3].tolist() == d
+    # an empty segment: nothing to compare, rel 0 (both sums 0)
+    assert (num[3], den[3], rel[3]) == (0.0, 0.0, 0.0)
+    # a segment whose reference is all zero but whose output is not: rel is +inf
+    z = np.zeros((2, n), np.float32)
+    _, _, r_inf = O.score(S.f32_to_bf16_bits(z + 1), S.f32_to_bf16_bits(z), [(0, 2)])
+    assert r_inf[0] == math.inf
+
+
 # --------------------------------------------------------------------------
 # Storage layouts
 # --------------------------------------------------------------------------
