@@ -171,6 +171,26 @@ def test_quantize_blocks_bruteforce(s_g):
         assert codes[0].tolist() == want_codes
 
 
+def test_elements_are_multiplied_by_the_rounded_reciprocal():
+    # Reading R4: q = RN32(x * RN32(1/S)), not RN32(x / S).  At s_g = 0.76333332
+    # the block maximum 34.5 sets the scale byte 0x4F (7.5), S = RN32(7.5 s_g); for
+    # 7.15625, 14.3125 and 28.625 the product lands one fp32 ulp above the E2M1
+    # midpoints 1.25, 2.5 and 5 and rounds up (codes 3, 5, 7), while the quotient
+    # rounds to the midpoint itself and would tie to the even codes 2, 4, 6.
+    s_g = np.float32(0.7633333206176758)
+    x = np.zeros(16, np.float32)
+    x[:4] = [34.5, 7.15625, 14.3125, 28.625]
+    bits = S.f32_to_bf16_bits(x)
+    assert np.array_equal(S.bf16_bits_to_f32(bits), x)
+    codes, sf, _ = O.quantize_blocks(bits[None, :], None, s_g)
+    assert int(sf[0, 0]) == 0x4F and O.E4M3_VALUES[0x4F] == 7.5
+    assert codes[0, 1:4].tolist() == [3, 5, 7]
+    scale = np.float32(np.float32(7.5) * s_g)
+    assert [int(O.e2m1_encode(np.array([np.float32(v / scale)]))[0]) for v in x[1:4]] == [2, 4, 6]
+    want_codes, want_sf = _brute_block(x, s_g)
+    assert codes[0].tolist() == want_codes and want_sf == 0x4F
+
+
 def test_quantize_uses_the_group_of_16_consecutive_channels():
     # one large value per group: every group gets its own scale
     x = np.zeros((1, 64), np.float32)
@@ -188,6 +208,12 @@ def test_saturation_count():
     x[1, 17] = 1e4          # second block of row 1 needs a scale above 448 at s_g = 1
     _, sf, n_sat = O.quantize_blocks(S.f32_to_bf16_bits(x), None, np.float32(1.0))
     assert n_sat == 1 and sf[1, 1] == 0x7E
+    # a block whose scale is exactly 448 (absmax 2688 = 6 * 448 at s_g = 1) is not
+    # saturated; the next bf16 value, 2704, needs 450.67 and is
+    y = np.ones((1, 32), np.float32)
+    y[0, 3], y[0, 20] = 2688.0, 2704.0
+    _, sf, n_sat = O.quantize_blocks(S.f32_to_bf16_bits(y), None, np.float32(1.0))
+    assert n_sat == 1 and sf[0].tolist() == [0x7E, 0x7E]
 
 
 # --------------------------------------------------------------------------
@@ -290,6 +316,21 @@ def test_full_rank_branch_reconstructs_the_layer():
     assert rel[n] < 2e-2 and rel[0] > 3 * rel[n]
 
 
+def test_weight_tensor_scale_closed_form():
+    # Reading R3 for weights: s_gW = max|R| / (6 * 448) of the 4-bit weight R; at
+    # rank 0, R = W diag(lambda).  The largest |W lambda| is 10.5 * 2 = 21, so
+    # s_gW = 21 / 2688 = 2^-7; that element's block scale is then exactly 448
+    # (byte 0x7E, S = 3.5) and the element itself the largest E2M1 value, 6.
+    rng = np.random.default_rng(4)
+    w = (0.02 * rng.standard_normal((16, 32))).astype(np.float32)
+    w[5, 7] = 10.5
+    lam = np.ones(32, np.float32)
+    lam[7] = 2.0
+    conv = O.convert_weight(S.f32_to_bf16_bits(w), lam, 0)
+    assert conv["s_g"] == np.float32(2.0 ** -7)
+    assert conv["sf"][5, 0] == 0x7E and conv["codes"][5, 7] == 7
+
+
 def test_lowrank_down_folds_lambda():
     rng = np.random.default_rng(4)
     x = S.f32_to_bf16_bits(rng.standard_normal((6, 32)).astype(np.float32))
@@ -332,15 +373,15 @@ def test_zero_activations_give_zero_codes_and_bias_output():
 def test_calib_lambda_closed_forms():
     x = np.zeros((3, 4), np.float32)
     w = np.zeros((2, 4), np.float32)
-    x[:, 0] = [1, -4, 2]; w[:, 0] = [1, -0.5]            # 4 / 1   -> lambda 2
+    x[:, 0] = [1, -16, 2]; w[:, 0] = [1, -0.5]           # 16 / 1  -> lambda 4
     x[:, 1] = [2, 0, 0];  w[:, 1] = [1, 0]               # 2 / 1   -> sqrt(2)
     x[:, 2] = 0;          w[:, 2] = [3, 1]               # zero activation column -> 1
     x[:, 3] = [0, 9, 0];  w[:, 3] = 0                    # zero weight column -> 1
     c = O.calib(S.f32_to_bf16_bits(x), None, S.f32_to_bf16_bits(w))
-    assert c["lam"].tolist() == [2.0, np.float32(math.sqrt(2.0)), 1.0, 1.0]
-    assert c["ax"].tolist() == [4.0, 2.0, 0.0, 9.0]
-    assert c["inv_lam"][0] == 0.5
-    # s_g = max(ax / lambda) / (6 * 448): max(2, 2/sqrt2, 0, 9) = 9
+    assert c["lam"].tolist() == [4.0, np.float32(math.sqrt(2.0)), 1.0, 1.0]
+    assert c["ax"].tolist() == [16.0, 2.0, 0.0, 9.0]
+    assert c["inv_lam"][0] == 0.25
+    # s_g = max(ax / lambda) / (6 * 448): max(4, 2/sqrt2, 0, 9) = 9, not max(ax) = 16
     assert c["s_g"] == np.float32(np.float32(9.0) / np.float32(2688.0))
 
 
