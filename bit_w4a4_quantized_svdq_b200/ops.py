@@ -80,6 +80,35 @@ def _check_bf16(t: torch.Tensor, name: str) -> None:
         raise ValueError(f"{name} must be a CUDA tensor")
 
 
+_BF16_TYPES = (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def _check_dense(t: Optional[torch.Tensor], dtypes, min_numel: int, name: str, optional: bool = False) -> None:
+    """A dense (contiguous) tensor of one of `dtypes` holding at least `min_numel`
+    elements: the kernels read such arguments through a bare pointer, so a wrong
+    type or a short buffer is refused here rather than read past its end."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if t.dtype not in dtypes:
+        want = " or ".join(str(d) for d in dtypes)
+        raise TypeError(f"{name} must be {want}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, the call reads {min_numel}")
+
+
+def _check_matrix(t: Optional[torch.Tensor], dtypes, rows: int, cols: int, name: str) -> None:
+    """A contiguous [rows, cols] tensor of one of `dtypes` (None passes)."""
+    if t is None:
+        return
+    _check_dense(t, dtypes, 0, name)
+    if tuple(t.shape) != (rows, cols):
+        raise ValueError(f"{name} must be [{rows}, {cols}], got {list(t.shape)}")
+
+
 def _row_stride(t: torch.Tensor, name: str) -> int:
     if t.dim() != 2 or t.stride(1) != 1:
         raise ValueError(f"{name} must be a row-major 2-D tensor")
@@ -146,15 +175,44 @@ def svdq_quantize_act(x: torch.Tensor, inv_lambda: Optional[torch.Tensor], s_g: 
     m, k = x.shape
     ldx = _row_stride(x, "x")
     r = 0 if down is None else int(down.shape[0])
+    _check_dense(inv_lambda, (torch.float32,), k, "inv_lambda", optional=True)
+    _check_dense(s_g, (torch.float32,), 1, "s_g")
+    _check_matrix(down, _BF16_TYPES, r, k, "down")
+    _check_dense(sat_count, (torch.int32, torch.uint32), 1, "sat_count", optional=True)
     dev = x.device
     if out is None:
         out = dict(codes=_lib.out_empty((m, k // 2), torch.uint8, dev),
                    sf=_lib.out_empty(sf_bytes(m, k), torch.uint8, dev),
                    d=_lib.out_empty((m, r), torch.float32, dev) if r else None)
+    _check_dense(out["codes"], (torch.uint8,), m * (k // 2), "out['codes']")
+    _check_dense(out["sf"], (torch.uint8,), sf_bytes(m, k), "out['sf']")
+    _check_dense(out.get("d"), (torch.float32,), m * r, "out['d']", optional=r == 0)
     _lib.check("svdq_quantize_act", lib.svdq_quantize_act(
         _ptr(x), m, k, ldx, _ptr(inv_lambda), _ptr(s_g), _ptr(down), r,
         _ptr(out["codes"]), _ptr(out["sf"]), _ptr(out["d"]), _ptr(sat_count), _stream(stream)))
     return out
+
+
+def _check_linear_operands(a_codes, a_sf, s_g_act, d, w_codes, w_sf, s_g_w, up, bias):
+    """Shapes and types of the NVFP4 linear's operands; returns (m, n, k, r)."""
+    if a_codes.dim() != 2 or w_codes.dim() != 2:
+        raise ValueError("a_codes and w_codes must be 2-D [rows, K/2] byte tensors")
+    m, kh = a_codes.shape
+    n = w_codes.shape[0]
+    k = 2 * kh
+    _check_matrix(a_codes, (torch.uint8,), m, kh, "a_codes")
+    _check_matrix(w_codes, (torch.uint8,), n, kh, "w_codes")
+    _check_dense(a_sf, (torch.uint8,), sf_bytes(m, k), "a_sf")
+    _check_dense(w_sf, (torch.uint8,), sf_bytes(n, k), "w_sf")
+    _check_dense(s_g_act, (torch.float32,), 1, "s_g_act")
+    _check_dense(s_g_w, (torch.float32,), 1, "s_g_w")
+    r = 0 if d is None else int(d.shape[-1])
+    if d is not None:
+        _check_matrix(d, (torch.float32,), m, r, "d")
+    if up is not None:
+        _check_matrix(up, _BF16_TYPES, n, r, "up")
+    _check_dense(bias, _BF16_TYPES, n, "bias", optional=True)
+    return m, n, k, r
 
 
 @_on_tensor_device
@@ -164,12 +222,11 @@ def svdq_linear(a_codes: torch.Tensor, a_sf: torch.Tensor, s_g_act: torch.Tensor
                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Y = s_g_act s_g_w deq(A) deq(W)^T + D up^T + bias."""
     lib = _lib.load()
-    m, kh = a_codes.shape
-    n = w_codes.shape[0]
-    k = 2 * kh
-    r = 0 if d is None else int(d.shape[1])
+    m, n, k, r = _check_linear_operands(a_codes, a_sf, s_g_act, d, w_codes, w_sf, s_g_w, up, bias)
     if out is None:
         out = _lib.out_empty((m, n), out_dtype, a_codes.device)
+    if out.dtype not in (torch.bfloat16, torch.float32) or out.dim() != 2 or tuple(out.shape) != (m, n):
+        raise ValueError(f"out must be a bf16 or float32 [{m}, {n}] tensor")
     ldy = _row_stride(out, "out")
     code = {torch.bfloat16: 0, torch.float32: 1}[out.dtype]
     _lib.check("svdq_linear", lib.svdq_linear(
@@ -192,10 +249,7 @@ def svdq_linear_score(a_codes: torch.Tensor, a_sf: torch.Tensor, s_g_act: torch.
     yref.  Returns (out or None, num, den, rel); write_out=False skips the output."""
     lib = _lib.load()
     _check_bf16(yref, "yref")
-    m, kh = a_codes.shape
-    n = w_codes.shape[0]
-    k = 2 * kh
-    r = 0 if d is None else int(d.shape[1])
+    m, n, k, r = _check_linear_operands(a_codes, a_sf, s_g_act, d, w_codes, w_sf, s_g_w, up, bias)
     if tuple(yref.shape) != (m, n):
         raise ValueError(f"yref must be [{m}, {n}], got {tuple(yref.shape)}")
     dev = a_codes.device
@@ -203,6 +257,8 @@ def svdq_linear_score(a_codes: torch.Tensor, a_sf: torch.Tensor, s_g_act: torch.
         out = _lib.out_empty((m, n), torch.bfloat16, dev)
     if not write_out:
         out = None
+    if out is not None and (out.dtype not in _BF16_TYPES or tuple(out.shape) != (m, n)):
+        raise ValueError(f"out must be a bf16 [{m}, {n}] tensor")
     ldy = _row_stride(out, "out") if out is not None else n
     arr, n_seg = _lib.seg_array(segs)
     num = _lib.out_empty(n_seg, torch.float64, dev)
@@ -276,6 +332,9 @@ def svdq_residual(w: torch.Tensor, lam: Optional[torch.Tensor], down: Optional[t
     _check_bf16(w, "w")
     n, k = w.shape
     r = 0 if down is None else int(down.shape[0])
+    _check_dense(lam, (torch.float32,), k, "lam", optional=True)
+    _check_matrix(down, _BF16_TYPES, r, k, "down")
+    _check_matrix(up, _BF16_TYPES, n, r, "up")
     out = _lib.out_empty((n, k), torch.bfloat16, w.device)
     _lib.check("svdq_residual", lib.svdq_residual(
         _ptr(w), n, k, _row_stride(w, "w"), _ptr(lam), _ptr(down), _ptr(up), r, _ptr(out), _stream(stream)))
@@ -341,6 +400,8 @@ def svdq_quantize_mxfp8(x: torch.Tensor, out: Optional[dict] = None, stream=None
     if out is None:
         out = dict(codes=_lib.out_empty((m, k), torch.uint8, x.device),
                    sf=_lib.out_empty(nbytes, torch.uint8, x.device))
+    _check_dense(out["codes"], (torch.uint8,), m * k, "out['codes']")
+    _check_dense(out["sf"], (torch.uint8,), nbytes, "out['sf']")
     _lib.check("svdq_quantize_mxfp8", lib.svdq_quantize_mxfp8(
         _ptr(x), m, k, _row_stride(x, "x"), _ptr(out["codes"]), _ptr(out["sf"]), _stream(stream)))
     return out
@@ -352,10 +413,19 @@ def svdq_linear_mxfp8(a_codes: torch.Tensor, a_sf: torch.Tensor, w_codes: torch.
                       stream=None) -> torch.Tensor:
     """Y bf16 [M, N] = dequant(A) dequant(W)^T + bias on the MXFP8 tensor-core path."""
     lib = _lib.load()
+    if a_codes.dim() != 2 or w_codes.dim() != 2:
+        raise ValueError("a_codes and w_codes must be 2-D [rows, K] byte tensors")
     m, k = a_codes.shape
     n = w_codes.shape[0]
+    _check_matrix(a_codes, (torch.uint8,), m, k, "a_codes")
+    _check_matrix(w_codes, (torch.uint8,), n, k, "w_codes")
+    _check_dense(a_sf, (torch.uint8,), mxfp8_sf_bytes(m, k), "a_sf")
+    _check_dense(w_sf, (torch.uint8,), mxfp8_sf_bytes(n, k), "w_sf")
+    _check_dense(bias, _BF16_TYPES, n, "bias", optional=True)
     if out is None:
         out = _lib.out_empty((m, n), torch.bfloat16, a_codes.device)
+    if out.dtype not in _BF16_TYPES or tuple(out.shape) != (m, n):
+        raise ValueError(f"out must be a bf16 [{m}, {n}] tensor")
     _lib.check("svdq_linear_mxfp8", lib.svdq_linear_mxfp8(
         _ptr(a_codes), _ptr(a_sf), _ptr(w_codes), _ptr(w_sf), _ptr(bias), _ptr(out), _row_stride(out, "out"),
         m, n, k, _stream(stream)))

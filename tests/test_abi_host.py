@@ -222,3 +222,46 @@ def test_wrappers_reject_tensors_on_different_devices():
         ops.svdq_quantize_act(cpu.view(torch.int16), None, f32)
     with pytest.raises(ValueError, match="CUDA tensors"):
         ops.svdq_calib_lambda(cpu.view(torch.int16), None, None)
+
+
+def test_binding_refuses_wrong_types_and_short_buffers():
+    """Arguments the kernels read through a bare pointer are checked for dtype,
+    dense layout and size before any launch (the checks need no device)."""
+    import torch
+
+    from bit_w4a4_quantized_svdq_b200 import ops
+
+    m, n, k, r = 4, 256, 128, 16
+    sfa, sfw = ops.sf_bytes(m, k), ops.sf_bytes(n, k)
+    good = dict(a_codes=torch.zeros((m, k // 2), dtype=torch.uint8), a_sf=torch.zeros(sfa, dtype=torch.uint8),
+                s_g_act=torch.ones(1), d=torch.zeros((m, r)), w_codes=torch.zeros((n, k // 2), dtype=torch.uint8),
+                w_sf=torch.zeros(sfw, dtype=torch.uint8), s_g_w=torch.ones(()),
+                up=torch.zeros((n, r), dtype=torch.int16), bias=torch.zeros(n, dtype=torch.bfloat16))
+    assert ops._check_linear_operands(**good) == (m, n, k, r)
+    assert ops._check_linear_operands(**dict(good, d=None, up=None, bias=None)) == (m, n, k, 0)
+    bad = [
+        (dict(s_g_act=torch.ones(1, dtype=torch.float64)), TypeError),        # wrong dtype
+        (dict(a_sf=torch.zeros(sfa - 1, dtype=torch.uint8)), ValueError),     # short scale buffer
+        (dict(w_sf=torch.zeros(sfa, dtype=torch.uint8)), ValueError),         # the activation's size, not W's
+        (dict(d=torch.zeros((m, r)).t().contiguous().t()), ValueError),       # not contiguous
+        (dict(d=torch.zeros((m + 1, r))), ValueError),                        # wrong rows
+        (dict(up=torch.zeros((n, r + 16), dtype=torch.int16)), ValueError),   # rank differs from D's
+        (dict(up=torch.zeros((n, r), dtype=torch.float16)), TypeError),       # not bf16
+        (dict(bias=torch.zeros(n - 1, dtype=torch.int16)), ValueError),       # short bias
+        (dict(w_codes=torch.zeros((n, k // 2 + 1), dtype=torch.uint8)), ValueError),  # K differs from A's
+        (dict(a_codes=torch.zeros((m, k // 2), dtype=torch.int8)), TypeError),
+    ]
+    for change, err in bad:
+        with pytest.raises(err):
+            ops._check_linear_operands(**dict(good, **change))
+    # 1/lambda and the tensor scale of the activation quantiser
+    ops._check_dense(torch.ones((3, k))[1], (torch.float32,), k, "inv_lambda")   # a row of a candidate grid
+    ops._check_dense(torch.ones(()), (torch.float32,), 1, "s_g")                  # a 0-dim scale
+    with pytest.raises(ValueError):
+        ops._check_dense(torch.ones(k - 1), (torch.float32,), k, "inv_lambda")
+    with pytest.raises(ValueError):
+        ops._check_dense(None, (torch.float32,), 1, "s_g")
+    ops._check_dense(None, (torch.float32,), k, "inv_lambda", optional=True)
+    ops._check_matrix(torch.zeros((r, k), dtype=torch.int16), ops._BF16_TYPES, r, k, "down")
+    with pytest.raises(ValueError):
+        ops._check_matrix(torch.zeros((k, r), dtype=torch.int16).t(), ops._BF16_TYPES, r, k, "down")
