@@ -49,6 +49,9 @@ Readings where the pages are silent:
      the down factor is stored with lambda folded in (L1s = diag(1/lambda) L1)
      as a [r, K] "down" weight and L2^T as an [N, r] "up" weight, both bf16.
   R10 rel-L2 of a segment is ||Yq - Yref||_F / ||Yref||_F over its rows.
+  R11 fp64 results stored as bf16 (the residual, the layer output compared
+      in bf16) are rounded fp64 -> fp32 -> bf16, each step to nearest, ties
+      to even.
   R15 The bits-lost proxy uses per-modality channel absmax statistics: the
       channel's absmax is RN32(ax_j * (1/lambda_j)) (the smoothed statistic
       the kernel's group scale sees; max over rows commutes with the monotone
@@ -77,11 +80,14 @@ Readings where the pages are silent:
       exact product) rounded to nearest, ties to even, saturating at 448, sign
       kept (-0 -> 0x80).  No smoothing, no low-rank branch, no tensor scale.
 
-Pins (``tests/test_oracle_pins.py``) hold every function to something other
-than itself: independent float-format rounding, torch's float8 conversion,
-exact rational brute force on tiny blocks, exactly representable inputs whose
-W4A4 product equals a plain fp64 matmul, full-rank low-rank branches, and
-reduction identities.  The scale-factor memory layout (``sf_to_mma_layout``)
+Pins (``tests/test_oracle_*.py``) hold every function to something other
+than itself: independent float-format rounding, the bf16 format's definition,
+torch's float8 conversion, exact rational brute force on tiny blocks, exactly
+representable inputs whose W4A4 product equals a plain fp64 matmul, full-rank
+low-rank branches, closed forms, worked values that separate each reading
+from its nearest alternative, and reduction identities.
+``tests/oracle_mutation_audit.py`` plants plausible slips in a copy of this
+module and checks that each one fails a pin.  The scale-factor memory layout (``sf_to_mma_layout``)
 is a hardware operand layout, not a page formula: it is pinned as a
 bijection and by the GPU GEMM that consumes it.
 """
