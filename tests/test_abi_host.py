@@ -265,3 +265,26 @@ def test_binding_refuses_wrong_types_and_short_buffers():
     ops._check_matrix(torch.zeros((r, k), dtype=torch.int16), ops._BF16_TYPES, r, k, "down")
     with pytest.raises(ValueError):
         ops._check_matrix(torch.zeros((k, r), dtype=torch.int16).t(), ops._BF16_TYPES, r, k, "down")
+
+
+def test_header_is_plain_c():
+    """include/svdq.h compiles as C99 (and as C++) in a unit that takes the
+    address of every entry point it declares, so the boundary needs no C++."""
+    import shutil
+    import subprocess
+    import tempfile
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    names = _declared_functions()
+    body = ("#include \"svdq.h\"\ntypedef void (*any_fn)(void);\n" +
+            "".join(f"any_fn p_{n} = (any_fn)&{n};\n" for n in names))
+    with tempfile.TemporaryDirectory() as d:
+        for lang, std, ext in (("c", "-std=c99", "c"), ("c++", "-std=c++17", "cc")):
+            src = os.path.join(d, f"unit.{ext}")
+            with open(src, "w") as f:
+                f.write(body)
+            res = subprocess.run([cc, "-x", lang, std, "-Wall", "-Werror", "-pedantic", "-c", src,
+                                  "-I", os.path.join(ROOT, "include"), "-o", os.path.join(d, f"unit_{ext}.o")],
+                                 capture_output=True, text=True)
+            assert res.returncode == 0, res.stderr
