@@ -564,8 +564,9 @@ def run_gpu(args):
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             # a bounded row sample of the same workload: about 10-20 s of host work
+            # (each run also reads and dequantises the whole weight, ~1.5-2 s)
             arm = OracleArm(layer)
-            rows = min(layer.m, 384)
+            rows = min(layer.m, 2048)
             runs = [arm.run(rows) for _ in range(2)]
             dt = sum(x[1] for x in runs)
             cpu = {"value": 2 * 2.0 * rows * n * k / dt / 1e12, "unit": UNIT, "cores": _oracle_threads(),
